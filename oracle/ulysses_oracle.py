@@ -1,0 +1,277 @@
+"""Plain CPU oracle for the Ulysses sequence-parallel attention layer (fp64).
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+use it.  It shares no code with the CUDA library; both sides see the same
+seeded inputs and nothing else.
+
+Sources (web pages, cited by title and section):
+
+* "hao-ai-lab FastVideo, compare main...perf/ulysses-h3-adaptive" -- the fused
+  Ulysses all-to-all.  The shape comment above ``ulysses_a2a_tuned`` in
+  ``csrc/comm/ulysses_all_to_all.cu`` fixes the two modes:
+  mode 0 maps ``[B, S_local, H, D]`` to ``[B, S_global, H_local, D]`` and mode 1
+  is its inverse, with ``H_local = H / world``.  ``docs/contributing/
+  ulysses_performance.md`` ("Ulysses performance on GB200") fixes the 1 GiB
+  per-rank window and the per-plane exchange (896,000,000 bytes per plane at
+  250,000 tokens, 56 heads, head dim 128, sequence parallelism 4).
+  ``ulysses_a2a.py`` (``MAX_WINDOW_BYTES``, ``_call_signature``, ``run_armed``)
+  gives the window arithmetic and the one-launch-per-plane loop.
+* "hao-ai-lab FastVideo, compare aryan/h3-nvfp4-stack-speedups...main" --
+  ``DistributedAttention.forward_stacked`` in ``fastvideo/attention/layer.py``
+  (stack Q/K/V, all-to-all with scatter_dim=2 / gather_dim=1, backend
+  attention, inverse all-to-all) and the FA4 wrappers in
+  ``flash_attn_cute.py`` (softmax attention with ``softmax_scale``, non-causal,
+  varlen through ``cu_seqlens``).
+
+Readings where the pages leave a step open (each one is also listed in the
+design notes of the repository):
+
+* The all-to-all body is not printed.  We take the standard reading of the
+  mode-0 shape map: source rank q contributes its local tokens as global rows
+  ``q*Nl + i`` (rank order), and destination rank r receives heads
+  ``[r*Hl, (r+1)*Hl)``.
+* N not divisible by P is padded to ``Np = P*ceil(N/P)`` rows; pad rows are
+  moved by the repack like any other row, never attended to as keys, and
+  produce zero output rows.
+* Sequence-sharded layout is token-interleaved ``[Np, C, H, D]`` (planes Q, K,
+  V[, G]); head-sharded layout is ``[P, C, Np, Hl, D]``.
+
+Everything here is written for clarity, not speed.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+# 1 GiB registered window per rank ("Ulysses performance on GB200": each rank
+# keeps at most 1 GiB of registered window storage; ``MAX_WINDOW_BYTES`` in
+# ulysses_a2a.py).
+MAX_WINDOW_BYTES = 1024 ** 3
+BF16_BYTES = 2
+
+
+# ---------------------------------------------------------------------------
+# Sizes and window arithmetic
+# ---------------------------------------------------------------------------
+
+def local_tokens(N: int, P: int) -> int:
+    """Nl = ceil(N / P): tokens owned by each virtual rank before the repack."""
+    if P < 1 or N < 0:
+        raise ValueError("need P >= 1 and N >= 0")
+    return -(-N // P)
+
+
+def padded_tokens(N: int, P: int) -> int:
+    """Np = P * Nl: the padded global sequence length every buffer is sized for."""
+    return P * local_tokens(N, P)
+
+
+def plane_bytes_per_rank(N: int, H: int, D: int, P: int, elem_bytes: int = BF16_BYTES) -> int:
+    """Bytes one virtual rank sends (and receives) for ONE plane.
+
+    Sequence side: Nl tokens x H heads x D; head side: Np tokens x H/P heads x D.
+    Both are equal.  ulysses_a2a.py sizes the chunked window as
+    ``nbytes // planes`` for an operand ``[planes, S_local, H, D]``.
+    """
+    return local_tokens(N, P) * H * D * elem_bytes
+
+
+def auto_plane_chunk(N: int, H: int, D: int, P: int, planes: int,
+                     window_bytes: int = MAX_WINDOW_BYTES) -> int:
+    """Largest number of planes per launch whose per-rank bytes fit the window.
+
+    Returns 0 when a single plane already exceeds the window (the call must be
+    refused, as ulysses_a2a.py declines operands whose window exceeds the cap).
+    """
+    per_plane = plane_bytes_per_rank(N, H, D, P)
+    if per_plane > window_bytes:
+        return 0
+    if per_plane == 0:
+        return planes
+    return min(planes, window_bytes // per_plane)
+
+
+# ---------------------------------------------------------------------------
+# bf16 helpers (bit patterns held as uint16)
+# ---------------------------------------------------------------------------
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening: a bf16 pattern is the top half of an IEEE binary32."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 -> fp32 (round to nearest even) -> bf16 (round to nearest even).
+
+    Used only to build bf16 inputs for closed-form tests; NaN maps to the
+    canonical quiet NaN 0x7FC0.
+    """
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    rounded = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    nan = np.isnan(f)
+    rounded[nan] = 0x7FC0
+    return rounded
+
+
+# ---------------------------------------------------------------------------
+# Repack (the all-to-all index map), exact on bit patterns
+# ---------------------------------------------------------------------------
+
+def repack_fwd(S: np.ndarray, P: int) -> np.ndarray:
+    """Ulysses mode 0 on one GPU: sequence-sharded -> head-sharded.
+
+    S: ``[Np, C, H, D]`` uint16 (bf16 bits).  Rank q owns rows ``[q*Nl, (q+1)*Nl)``.
+    Returns T: ``[P, C, Np, Hl, D]`` with ``T[r, c, n, j, d] = S[n, c, r*Hl + j, d]``.
+
+    Written as the reshape/transpose of the mode-0 shape comment in
+    ``ulysses_all_to_all.cu``: every source rank's ``[Nl, H, D]`` block is split
+    along heads into P pieces; piece r goes to rank r, where the pieces from
+    all source ranks are stacked in source-rank order along the sequence.
+    """
+    Np, C, H, D = S.shape
+    if Np % P or H % P:
+        raise ValueError("Np and H must be divisible by P")
+    Nl, Hl = Np // P, H // P
+    # [src rank q, local token i, plane c, dest rank r, local head j, d]
+    x = S.reshape(P, Nl, C, P, Hl, D)
+    # -> [dest rank r, plane c, src rank q, local token i, local head j, d]
+    x = x.transpose(3, 2, 0, 1, 4, 5)
+    return np.ascontiguousarray(x).reshape(P, C, Np, Hl, D)
+
+
+def repack_bwd(T: np.ndarray) -> np.ndarray:
+    """Ulysses mode 1: head-sharded ``[P, C, Np, Hl, D]`` -> ``[Np, C, P*Hl, D]``.
+
+    ``S[n, c, r*Hl + j, d] = T[r, c, n, j, d]``: the inverse of :func:`repack_fwd`.
+    """
+    P, C, Np, Hl, D = T.shape
+    Nl = Np // P
+    x = T.reshape(P, C, P, Nl, Hl, D)           # [r, c, q, i, j, d]
+    x = x.transpose(2, 3, 1, 0, 4, 5)            # [q, i, c, r, j, d]
+    return np.ascontiguousarray(x).reshape(Np, C, P * Hl, D)
+
+
+# ---------------------------------------------------------------------------
+# Attention (fp64 definition)
+# ---------------------------------------------------------------------------
+
+def segments_from_cu_seqlens(cu_seqlens, N: int) -> list[tuple[int, int]]:
+    """Turn ``cu_seqlens`` prefix sums into ``[(start, end), ...]``.
+
+    ``cu_seqlens`` is the varlen metadata of the FA4 wrappers (int32 prefix sums
+    of packed sequence lengths, first entry 0, last entry the total).  None
+    means one sequence of length N.
+    """
+    if cu_seqlens is None:
+        return [(0, N)]
+    cu = [int(v) for v in cu_seqlens]
+    if len(cu) < 2 or cu[0] != 0 or cu[-1] != N or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must start at 0, be non-decreasing and end at N")
+    return [(a, b) for a, b in zip(cu, cu[1:])]
+
+
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
+    """Softmax attention of query rows ``q [R, D]`` over keys ``k, v [M, D]`` in fp64.
+
+    ``o = softmax(scale * q k^T) v`` row by row (non-causal: every key counts).
+    The row maximum is subtracted before ``exp``; this changes nothing
+    mathematically and keeps fp64 finite.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if k.shape[0] == 0:
+        return np.zeros((q.shape[0], v.shape[1]), dtype=np.float64)
+    z = scale * (q @ k.T)                        # [R, M] logits
+    z = z - z.max(axis=1, keepdims=True)
+    p = np.exp(z)
+    return (p @ v) / p.sum(axis=1, keepdims=True)
+
+
+def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
+                    rows: np.ndarray | None = None) -> np.ndarray:
+    """Step two of the layer: attention on every head-sharded slab.
+
+    T: head-sharded ``[P, C, Np, Hl, D]`` uint16; planes 0, 1, 2 are Q, K, V
+    (a fourth plane, the gate, is ignored).  Query row n attends to the keys of
+    its own segment (all keys ``< N`` without ``cu_seqlens``).  Rows ``n >= N``
+    are padding and give zero.
+
+    Returns fp64 ``[P, R, Hl, D]`` for the selected rows (all ``Np`` rows when
+    ``rows`` is None).
+    """
+    P, C, Np, Hl, D = T.shape
+    if C < 3:
+        raise ValueError("need Q, K and V planes")
+    segs = segments_from_cu_seqlens(cu_seqlens, N)
+    rows = np.arange(Np) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros((P, rows.size, Hl, D), dtype=np.float64)
+    seg_of = np.full(rows.size, -1, dtype=np.int64)
+    for s, (a, b) in enumerate(segs):
+        seg_of[(rows >= a) & (rows < b)] = s
+    for r in range(P):
+        for j in range(Hl):
+            for s, (a, b) in enumerate(segs):
+                sel = np.nonzero(seg_of == s)[0]
+                if sel.size == 0:
+                    continue
+                q = bf16_bits_to_f64(T[r, 0, rows[sel], j, :])
+                k = bf16_bits_to_f64(T[r, 1, a:b, j, :])
+                v = bf16_bits_to_f64(T[r, 2, a:b, j, :])
+                out[r, sel, j, :] = attention_rows(q, k, v, scale)
+    return out
+
+
+def output_repack_bwd(O_heads: np.ndarray) -> np.ndarray:
+    """Step three on the attention output: ``[P, R, Hl, D] -> [R, P*Hl, D]``.
+
+    The same index map as :func:`repack_bwd` with one plane, applied to fp64
+    values (row selection already done).
+    """
+    P, R, Hl, D = O_heads.shape
+    return np.ascontiguousarray(O_heads.transpose(1, 0, 2, 3)).reshape(R, P * Hl, D)
+
+
+def layer_fwd(S: np.ndarray, P: int, N: int, scale: float, cu_seqlens=None,
+              rows: np.ndarray | None = None) -> np.ndarray:
+    """The whole layer: repack -> attention per slab -> inverse repack.
+
+    S: sequence-sharded ``[Np, C, H, D]`` uint16.  Returns fp64 ``[R, H, D]``
+    (sequence-sharded output rows, all ``Np`` rows when ``rows`` is None).
+    """
+    T = repack_fwd(S, P)
+    O = attention_heads(T, N, scale, cu_seqlens=cu_seqlens, rows=rows)
+    return output_repack_bwd(O)
+
+
+def sample_rows(N: int, count: int, seed: int, cu_seqlens=None) -> np.ndarray:
+    """The seeded subset of query rows checked on large N.
+
+    ``count`` rows drawn without replacement from ``[0, N)`` with
+    ``numpy.random.default_rng(seed + 10_000)``; rows 0 and N-1 and the first
+    and last row of every segment are always included.  Sorted.
+    """
+    if count >= N:
+        return np.arange(N)
+    rng = np.random.default_rng(seed + 10_000)
+    chosen = set(int(x) for x in rng.choice(N, size=count, replace=False))
+    forced = {0, N - 1}
+    for a, b in segments_from_cu_seqlens(cu_seqlens, N):
+        if b > a:
+            forced.update((a, b - 1))
+    return np.array(sorted(chosen | forced), dtype=np.int64)
+
+
+def attention_flops(N: int, H: int, D: int, cu_seqlens=None) -> float:
+    """Algorithmic attention FLOPs: 4 * L^2 * H * D summed over sequences."""
+    return float(sum(4 * (b - a) ** 2 * H * D for a, b in segments_from_cu_seqlens(cu_seqlens, N)))
+
+
+def softmax_scale(D: int) -> float:
+    """1/sqrt(D): the scale of the Ulysses layer (1/sqrt(128) for D = 128)."""
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,277 @@
+"""Pins for the CPU oracle: facts fixed by the pages and by mathematics.
+
+Each test checks the oracle against something other than itself: byte counts
+the pages print, the inverse/identity properties of the all-to-all, a
+brute-force index loop, closed-form softmax results, and the Ulysses
+invariant that the whole layer equals plain multi-head attention on the
+unsharded sequence.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import ulysses_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _bits(rng, shape):
+    # arbitrary 16-bit patterns, NaN/Inf/denormal included: the repack is a bit copy
+    return rng.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+
+
+def _bf16_normal(rng, shape, scale=1.0):
+    return orc.f64_to_bf16_bits(rng.standard_normal(shape) * scale)
+
+
+# ---------------------------------------------------------------- window bytes
+
+def test_window_bytes_match_printed_values():
+    g = json.load(open(os.path.join(GOLDEN, "window_bytes.json")))
+    for case in g["per_plane"]:
+        assert orc.plane_bytes_per_rank(case["tokens"], case["heads"], case["head_dim"], case["sp"]) == case["bytes"]
+    for case in g["whole_operand"]:
+        per_plane = orc.plane_bytes_per_rank(case["tokens"], case["heads"], case["head_dim"], case["sp"])
+        assert per_plane * case["planes"] == case["bytes"]
+    b = g["half_gib_boundary"]
+    lim = b["limit_bytes"]
+    lo, hi = b["below"], b["above"]
+    assert orc.plane_bytes_per_rank(lo["tokens"], lo["heads"], lo["head_dim"], lo["sp"]) <= lim
+    assert orc.plane_bytes_per_rank(hi["tokens"], hi["heads"], hi["head_dim"], hi["sp"]) > lim
+    assert orc.MAX_WINDOW_BYTES == g["window_cap_bytes"]["value"]
+
+
+def test_auto_plane_chunk_one_plane_per_launch_at_250k():
+    # 896,000,000 B per plane: two planes exceed 1 GiB, so one plane per launch
+    assert orc.auto_plane_chunk(250_000, 56, 128, 4, planes=4) == 1
+    # 32,000 tokens: all four planes (458,752,000 B) fit in one window
+    assert orc.auto_plane_chunk(32_000, 56, 128, 4, planes=4) == 4
+    # a plane larger than the window cannot be exchanged at all
+    assert orc.auto_plane_chunk(400_000, 56, 128, 4, planes=3) == 0
+
+
+def test_padding_sizes():
+    assert orc.padded_tokens(19_394, 4) == 19_396
+    assert orc.padded_tokens(1024, 2) == 1024
+    assert orc.padded_tokens(104_448, 8) == 104_448
+    assert orc.local_tokens(19_394, 4) == 4849
+
+
+# ---------------------------------------------------------------- repack
+
+@pytest.mark.parametrize("P,C,Nl,H,D", [(1, 3, 5, 4, 8), (2, 3, 4, 8, 4), (4, 4, 3, 8, 2), (8, 3, 2, 56, 2)])
+def test_repack_round_trip_is_identity(P, C, Nl, H, D):
+    rng = np.random.default_rng(P * 100 + C)
+    S = _bits(rng, (P * Nl, C, H, D))
+    T = orc.repack_fwd(S, P)
+    assert T.shape == (P, C, P * Nl, H // P, D)
+    assert np.array_equal(orc.repack_bwd(T), S)
+    # and the other way round
+    T2 = _bits(rng, T.shape)
+    assert np.array_equal(orc.repack_fwd(orc.repack_bwd(T2), P), T2)
+
+
+def test_repack_p1_is_identity():
+    rng = np.random.default_rng(7)
+    S = _bits(rng, (9, 4, 6, 8))
+    T = orc.repack_fwd(S, 1)
+    assert np.array_equal(T[0].transpose(1, 0, 2, 3), S)
+
+
+def _brute_force_fwd(S, P):
+    # literal per-element loop over the destination index set
+    Np, C, H, D = S.shape
+    Hl = H // P
+    T = np.zeros((P, C, Np, Hl, D), dtype=S.dtype)
+    for r in range(P):
+        for c in range(C):
+            for n in range(Np):
+                for j in range(Hl):
+                    for d in range(D):
+                        T[r, c, n, j, d] = S[n, c, r * Hl + j, d]
+    return T
+
+
+def _per_rank_all_to_all(S, P):
+    # the mode-0 shape map as P separate ranks: rank q holds x_q [C, Nl, H, D]
+    # (sequence shard); it sends head block r to rank r, which concatenates the
+    # blocks it receives in source-rank order along the sequence
+    Np, C, H, D = S.shape
+    Nl, Hl = Np // P, H // P
+    local = [S[q * Nl:(q + 1) * Nl].transpose(1, 0, 2, 3) for q in range(P)]
+    out = []
+    for r in range(P):
+        recv = [local[q][:, :, r * Hl:(r + 1) * Hl, :] for q in range(P)]
+        out.append(np.concatenate(recv, axis=1))   # [C, Np, Hl, D]
+    return np.stack(out)
+
+
+def test_repack_matches_brute_force_loop_and_per_rank_exchange():
+    rng = np.random.default_rng(11)
+    for P, C, Nl, H, D in [(2, 3, 3, 4, 2), (4, 4, 2, 8, 3), (3, 3, 2, 6, 2)]:
+        S = _bits(rng, (P * Nl, C, H, D))
+        T = orc.repack_fwd(S, P)
+        assert np.array_equal(T, _brute_force_fwd(S, P))
+        assert np.array_equal(T, _per_rank_all_to_all(S, P))
+
+
+def test_repack_rejects_indivisible_heads():
+    with pytest.raises(ValueError):
+        orc.repack_fwd(np.zeros((4, 3, 6, 2), np.uint16), 4)
+
+
+# ---------------------------------------------------------------- bf16 helpers
+
+def test_bf16_widening_known_patterns():
+    bits = np.array([0x3F80, 0xC000, 0x0000, 0x8000, 0x3F81, 0x7F80, 0x0001], dtype=np.uint16)
+    f = orc.bf16_bits_to_f64(bits)
+    assert f[0] == 1.0 and f[1] == -2.0 and f[2] == 0.0 and math.copysign(1, f[3]) == -1
+    assert f[4] == 1.0 + 2.0 ** -7
+    assert math.isinf(f[5])
+    assert f[6] == 2.0 ** -133
+
+
+def test_bf16_rounding_ties_to_even():
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties to the even pattern 0x3F80
+    assert orc.f64_to_bf16_bits(np.array([1.0 + 2.0 ** -8]))[0] == 0x3F80
+    # 1 + 3*2^-8 is halfway between 1+2^-7 (odd, 0x3F81) and 1+2^-6 (even, 0x3F82)
+    assert orc.f64_to_bf16_bits(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 0x3F82
+    assert orc.f64_to_bf16_bits(np.array([-2.0]))[0] == 0xC000
+    assert orc.f64_to_bf16_bits(np.array([float("nan")]))[0] == 0x7FC0
+
+
+# ---------------------------------------------------------------- attention closed forms
+
+S128 = 1.0 / math.sqrt(128.0)
+
+
+def test_scale_is_one_over_sqrt_128():
+    assert orc.softmax_scale(128) == S128
+
+
+def test_two_keys_weights_three_to_one():
+    # logits differ by ln 3 after scaling => weights exactly 3/4 and 1/4
+    D = 128
+    q = np.zeros((1, D)); q[0, 0] = 1.0
+    k = np.zeros((2, D)); k[0, 0] = math.log(3.0) * math.sqrt(128.0)
+    v = np.zeros((2, D)); v[0, :] = 4.0; v[1, :] = -8.0
+    o = orc.attention_rows(q, k, v, S128)
+    assert np.allclose(o, 0.75 * 4.0 + 0.25 * -8.0, rtol=0, atol=1e-13)
+
+
+def test_uniform_keys_give_mean_of_v():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((5, 16))
+    k = np.tile(rng.standard_normal((1, 16)), (9, 1))
+    v = rng.standard_normal((9, 16))
+    o = orc.attention_rows(q, k, v, 0.3)
+    assert np.allclose(o, np.tile(v.mean(axis=0), (5, 1)), rtol=0, atol=1e-13)
+
+
+def test_single_key_returns_its_value():
+    rng = np.random.default_rng(4)
+    v = rng.standard_normal((1, 8))
+    o = orc.attention_rows(rng.standard_normal((3, 8)), rng.standard_normal((1, 8)), v, 1.0)
+    assert np.allclose(o, np.tile(v, (3, 1)), rtol=0, atol=1e-15)
+
+
+def test_key_permutation_invariance():
+    rng = np.random.default_rng(5)
+    q, k, v = rng.standard_normal((4, 8)), rng.standard_normal((12, 8)), rng.standard_normal((12, 8))
+    perm = rng.permutation(12)
+    assert np.allclose(orc.attention_rows(q, k, v, 0.5), orc.attention_rows(q, k[perm], v[perm], 0.5),
+                       rtol=0, atol=1e-13)
+
+
+def _brute_force_softmax(q, k, v, scale):
+    out = []
+    for qi in q:
+        logits = [scale * math.fsum(float(a) * float(b) for a, b in zip(qi, kj)) for kj in k]
+        m = max(logits)
+        w = [math.exp(z - m) for z in logits]
+        tot = math.fsum(w)
+        out.append([math.fsum(wj * float(vj[d]) for wj, vj in zip(w, v)) / tot for d in range(v.shape[1])])
+    return np.array(out)
+
+
+@pytest.mark.parametrize("M", [1, 7, 64])
+def test_matches_brute_force_softmax(M):
+    rng = np.random.default_rng(M)
+    q, k, v = rng.standard_normal((6, 16)), rng.standard_normal((M, 16)), rng.standard_normal((M, 16))
+    assert np.allclose(orc.attention_rows(q, k, v, 0.25), _brute_force_softmax(q, k, v, 0.25),
+                       rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- layer invariants
+
+def _plain_mha(S, N, scale, segs):
+    # multi-head attention on the unsharded sequence, head by head (no repack)
+    Np, C, H, D = S.shape
+    out = np.zeros((Np, H, D))
+    for h in range(H):
+        for a, b in segs:
+            q = orc.bf16_bits_to_f64(S[a:b, 0, h])
+            k = orc.bf16_bits_to_f64(S[a:b, 1, h])
+            v = orc.bf16_bits_to_f64(S[a:b, 2, h])
+            out[a:b, h] = _brute_force_softmax(q, k, v, scale) if b - a <= 8 else orc.attention_rows(q, k, v, scale)
+    return out
+
+
+@pytest.mark.parametrize("P,N,H,C", [(2, 16, 4, 3), (4, 14, 8, 4), (1, 9, 2, 3), (3, 10, 6, 3)])
+def test_layer_equals_plain_multi_head_attention(P, N, H, C):
+    rng = np.random.default_rng(P * 31 + N)
+    D = 8
+    Np = orc.padded_tokens(N, P)
+    S = _bf16_normal(rng, (Np, C, H, D))
+    S[N:] = 0                                      # pad rows are zero in the input
+    got = orc.layer_fwd(S, P, N, 0.35)
+    want = _plain_mha(S, N, 0.35, [(0, N)])
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+    assert np.all(got[N:] == 0.0)                   # pad query rows give zero
+
+
+def test_varlen_equals_independent_segments():
+    rng = np.random.default_rng(21)
+    P, H, D, C = 2, 4, 8, 3
+    cu = [0, 5, 6, 13, 16]
+    N = cu[-1]
+    S = _bf16_normal(rng, (N, C, H, D))
+    got = orc.layer_fwd(S, P, N, 0.5, cu_seqlens=cu)
+    want = _plain_mha(S, N, 0.5, list(zip(cu, cu[1:])))
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+    # a segment of length one returns its own value row
+    assert np.allclose(got[5], orc.bf16_bits_to_f64(S[5, 2]), atol=1e-15)
+
+
+def test_padding_keys_never_attended():
+    # padded rows hold large values; results must not change
+    rng = np.random.default_rng(22)
+    P, N, H, D = 4, 10, 4, 8
+    Np = orc.padded_tokens(N, P)
+    S = _bf16_normal(rng, (Np, 3, H, D))
+    S[N:] = 0
+    base = orc.layer_fwd(S, P, N, 0.4)
+    S2 = S.copy()
+    S2[N:] = orc.f64_to_bf16_bits(np.full((Np - N, 3, H, D), 50.0))
+    got = orc.layer_fwd(S2, P, N, 0.4)
+    assert np.array_equal(got[:N], base[:N]) and np.all(got[N:] == 0)
+
+
+def test_row_sampling_matches_full_rows():
+    rng = np.random.default_rng(23)
+    P, N, H, D = 2, 40, 4, 8
+    S = _bf16_normal(rng, (N, 3, H, D))
+    rows = orc.sample_rows(N, 9, seed=1, cu_seqlens=[0, 17, 40])
+    assert {0, 16, 17, 39} <= set(rows.tolist())
+    full = orc.layer_fwd(S, P, N, 0.3, cu_seqlens=[0, 17, 40])
+    part = orc.layer_fwd(S, P, N, 0.3, cu_seqlens=[0, 17, 40], rows=rows)
+    assert np.array_equal(part, full[rows])
+
+
+def test_flop_count():
+    assert orc.attention_flops(1024, 8, 128) == 4 * 1024 ** 2 * 8 * 128
+    cu = [0, 52224, 83456, 104448]
+    assert orc.attention_flops(104448, 56, 128, cu) == sum(4 * L ** 2 * 56 * 128 for L in (52224, 31232, 20992))

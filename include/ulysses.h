@@ -1,0 +1,191 @@
+/*
+ * ulysses.h -- C ABI of the one-GPU Ulysses sequence-parallel attention layer
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The layer (DistributedAttention.forward_stacked, "hao-ai-lab FastVideo,
+ * compare aryan/h3-nvfp4-stack-speedups...main", fastvideo/attention/layer.py)
+ * has three steps, all run by kernels of this library:
+ *
+ *   1. repack_fwd  -- the Ulysses all-to-all in mode 0 (scatter heads, gather
+ *      sequence): P sequence-sharded slabs become P head-sharded slabs.
+ *      Shapes from the mode comment above ulysses_a2a_tuned ("hao-ai-lab
+ *      FastVideo, compare main...perf/ulysses-h3-adaptive",
+ *      csrc/comm/ulysses_all_to_all.cu):  [B, S_local, H, D] -> [B, S_global, H_local, D].
+ *   2. attn_fwd    -- non-causal softmax attention per head-sharded slab
+ *      (the FA4 backend of flash_attn_cute.py: softmax_scale, varlen through
+ *      cu_seqlens).
+ *   3. repack_bwd  -- mode 1, the inverse map, applied to the attention output.
+ *
+ * All P "virtual ranks" are slabs of one GPU's memory; there is no collective.
+ *
+ * Notation: N real tokens, P virtual ranks, H heads, D = 128 head dim,
+ * Hl = H / P, C planes (3 = Q,K,V; 4 = Q,K,V,G), Nl = ceil(N / P),
+ * Np = P * Nl (padded token count).  All tensors are bf16, row-major.
+ *
+ *   sequence-sharded input  S : Np rows; element (n, c, h, d) at
+ *                               n*token_stride + c*plane_stride + h*D + d
+ *                               (default token_stride = C*H*D, plane_stride = H*D,
+ *                               i.e. [Np, C, H, D]); rank q owns rows [q*Nl, (q+1)*Nl).
+ *   head-sharded            T : [P, C, Np, Hl, D];  T[r,c,n,j,d] = S[n,c,r*Hl+j,d]
+ *   head-sharded output   O_T : [P, Np, Hl, D]
+ *   sequence output       O_S : [Np, H, D]
+ *
+ * Rows n in [N, Np) are padding: the repack moves them like any other row,
+ * attention never uses them as keys and writes zero output rows for them.
+ *
+ * Conventions for every call:
+ *   - pointers named dev_* or taking tensors are caller-owned DEVICE memory on
+ *     the current device, 16-byte aligned; outputs must not overlap inputs;
+ *   - `stream` is a cudaStream_t (CUstream) passed as void*; NULL is the
+ *     legacy default stream;
+ *   - calls are asynchronous on `stream`, allocate nothing and do not
+ *     synchronise (except ulysses_last_device_error);
+ *   - invalid arguments are reported through the return code, never abort.
+ */
+#ifndef ULYSSES_H_
+#define ULYSSES_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+enum {
+  ULYSSES_OK = 0,
+  ULYSSES_ERR_ARG = 1,          /* null/overlapping pointer, bad size, bad cu_seqlens */
+  ULYSSES_ERR_DIVISIBILITY = 2, /* H % P != 0 (heads must split evenly across ranks) */
+  ULYSSES_ERR_ALIGN = 3,        /* pointer or stride not a multiple of 16 bytes */
+  ULYSSES_ERR_WINDOW = 4,       /* one plane per rank exceeds the 1 GiB window */
+  ULYSSES_ERR_WORKSPACE = 5,    /* workspace smaller than ulysses_workspace_bytes() */
+  ULYSSES_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed (or no device) */
+  ULYSSES_ERR_DEVICE = 7,       /* a kernel reported an error (see ulysses_last_device_error) */
+  ULYSSES_ERR_UNSUPPORTED = 8   /* D != 128, too many sequences, ... */
+};
+
+/* Per-rank window cap: at most 1 GiB moved per rank per repack launch
+ * ("Ulysses performance on GB200": each rank keeps at most 1 GiB of window
+ * storage and exchanges one plane at a time; MAX_WINDOW_BYTES in ulysses_a2a.py). */
+#define ULYSSES_MAX_WINDOW_BYTES (1024LL * 1024LL * 1024LL)
+/* Most packed sequences one plan accepts (cu_seqlens has num_seqs + 1 entries). */
+#define ULYSSES_MAX_SEQS 64
+
+typedef struct ulysses_plan_s ulysses_plan_t;
+
+/*
+ * Create a plan (host object owned by the library; free with
+ * ulysses_plan_destroy).  The plan is immutable and may be shared by any
+ * number of calls; backward reuses the forward plan, as _FusedUlyssesA2A does
+ * ("Outputs own their storage, and backward uses the plan saved by its forward").
+ *
+ *   N            real tokens (>= 1)
+ *   H, D, P      heads, head dim (must be 128), virtual ranks (1 <= P <= H, H % P == 0)
+ *   planes       C: 3 (Q,K,V) or 4 (Q,K,V,G; G is moved but not attended); 1..8 accepted
+ *   token_stride, plane_stride
+ *                element strides of the sequence-sharded input; 0, 0 selects
+ *                [Np, C, H, D].  Must be multiples of 8 elements (16 bytes).
+ *   plane_chunk  planes per repack launch; 0 = the largest count whose bytes
+ *                per rank fit in 1 GiB
+ *   cu_seqlens_host, num_seqs
+ *                host array of num_seqs+1 int32 prefix sums (first 0, last N,
+ *                non-decreasing) for packed varlen sequences attended
+ *                block-diagonally; NULL/0 = one sequence of length N.
+ *
+ * Errors: ARG, DIVISIBILITY, ALIGN, WINDOW (one plane per rank > 1 GiB, or a
+ * plane_chunk whose bytes exceed it), UNSUPPORTED.  On success *out is set.
+ * The plan holds a 16-byte device error word on the device current at
+ * creation; without a CUDA device the plan is still created so its sizes can
+ * be queried, and every launch returns ULYSSES_ERR_CUDA.
+ */
+int ulysses_plan(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
+                 int64_t token_stride, int64_t plane_stride, int64_t plane_chunk,
+                 const int32_t* cu_seqlens_host, int32_t num_seqs);
+
+void ulysses_plan_destroy(ulysses_plan_t* plan);
+
+/* Np = P * ceil(N / P): rows every buffer is sized for. */
+int64_t ulysses_plan_padded_tokens(const ulysses_plan_t* plan);
+
+/* Planes moved per repack launch (the window chunk the plan chose). */
+int32_t ulysses_plan_plane_chunk(const ulysses_plan_t* plan);
+
+/* Bytes one rank exchanges per plane: Nl * H * D * 2. */
+int64_t ulysses_plan_window_bytes_per_plane(const ulysses_plan_t* plan);
+
+/* Workspace for ulysses_layer_fwd with fused = 0: T (P*C*Np*Hl*D) plus
+ * O_T (P*Np*Hl*D) bf16 elements, each region 256-byte aligned.  0 bytes are
+ * needed with fused = 1. */
+size_t ulysses_workspace_bytes(const ulysses_plan_t* plan);
+
+/*
+ * Step 1, Ulysses mode 0: src_seq (sequence-sharded, plan strides, C planes)
+ * -> dst_heads T [P, C, Np, Hl, D].  One launch per plane chunk, each moving
+ * at most 1 GiB per rank (the per-plane loop of run_armed in ulysses_a2a.py).
+ * Bit-exact copy.  Errors: ARG, ALIGN, CUDA.
+ */
+int ulysses_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads, void* stream);
+
+/*
+ * Step 3, Ulysses mode 1 (the inverse map): src_heads [P, planes, Np, Hl, D]
+ * -> dst_seq.  With planes == C, dst_seq uses the plan's input strides (a full
+ * round trip restores the input bit for bit).  With planes < C, dst_seq is a
+ * dense [Np, planes, H, D] buffer; planes == 1 gives the layer output
+ * [Np, H, D].  Errors: ARG, ALIGN, CUDA.
+ */
+int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* dst_seq, int32_t planes,
+                       void* stream);
+
+/*
+ * Step 2: out_heads O_T [P, Np, Hl, D] = softmax(softmax_scale * Q K^T) V for
+ * every rank r and local head j, with Q, K, V the planes 0, 1, 2 of
+ * qkv_heads T [P, C, Np, Hl, D].  Non-causal; query row n attends to the keys
+ * of its cu_seqlens segment (all keys < N without cu_seqlens).  fp32
+ * accumulation and softmax, bf16 probabilities for the second product, bf16
+ * output; pad rows [N, Np) are written as zeros.  Errors: ARG, ALIGN, CUDA.
+ */
+int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, float softmax_scale,
+                     void* stream);
+
+/*
+ * The whole layer with softmax_scale = 1/sqrt(D):  out_seq O_S [Np, H, D]
+ * from qkv_seq (sequence-sharded, plan strides).
+ *   fused = 0: repack_fwd -> attn_fwd -> repack_bwd(planes = 1) through the
+ *              caller's workspace (>= ulysses_workspace_bytes()).
+ *   fused = 1: one attention launch whose tensor maps read qkv_seq directly
+ *              and whose epilogue writes O_S; the head-sharded copies never
+ *              exist.  workspace may be NULL.  Same arithmetic, same tile
+ *              order: the output equals the fused = 0 output bit for bit.
+ * Errors: ARG, ALIGN, WORKSPACE, CUDA.
+ */
+int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
+                      size_t workspace_bytes, int32_t fused, void* stream);
+
+/*
+ * ulysses_layer_fwd from HOST buffers: copies host_qkv_seq (pinned host
+ * memory, the plan's input layout) into dev_qkv_seq, runs the layer into
+ * dev_out_seq, and copies O_S back to host_out_seq, all on `stream`
+ * (asynchronous: synchronise before reading host_out_seq).  Device buffers
+ * and workspace are the caller's.  Errors: as ulysses_layer_fwd.
+ */
+int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
+                           void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
+                           int32_t fused, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the plan's device error word.
+ * Returns 0 when no kernel reported an error, otherwise the error bits
+ * (1 = a pipeline wait timed out and the kernel gave up; 2 = a work unit
+ * decoded outside the problem), or -1 if the synchronisation itself failed.
+ */
+int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream);
+
+/* Static description of a return code. */
+const char* ulysses_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ULYSSES_H_ */

@@ -1,0 +1,145 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Small cases span several tiles and ragged tails; the oracle finishes them in
+seconds.  Repack: bit-exact.  Attention: max-abs <= 2e-2 and mean-abs <= 2e-3
+against the fp64 oracle (the layer's stated tolerance); pad rows exactly zero.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import ulysses_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+
+# (P, N, H, C, layout, cu_seqlens, seed)
+CASES = [
+    pytest.param(2, 1024, 8, 3, "token", None, 0, id="tiny-P2-N1024-H8"),
+    pytest.param(4, 1001, 8, 3, "token", None, 5, id="ragged-P4-N1001"),
+    pytest.param(1, 300, 2, 3, "token", None, 6, id="P1-N300"),
+    pytest.param(4, 777, 8, 4, "token", None, 7, id="qkvg-P4-N777"),
+    pytest.param(2, 640, 4, 3, "plane", None, 8, id="plane-major-P2"),
+    pytest.param(2, 1000, 4, 3, "token", [0, 300, 301, 777, 1000], 9, id="varlen-4seq"),
+    pytest.param(8, 2048, 16, 3, "token", [0, 1024, 1536, 2048], 10, id="varlen-P8"),
+    pytest.param(1, 1, 1, 3, "token", None, 11, id="N1"),
+    pytest.param(4, 5, 4, 3, "token", None, 12, id="N5-P4"),
+]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _strides(layout, N, P, C, H):
+    Np = orc.padded_tokens(N, P)
+    if layout == "token":
+        return 0, 0
+    return H * 128, Np * H * 128
+
+
+def _seq_as_token_major(bits, layout):
+    # oracle input is always [Np, C, H, D]
+    return bits if layout == "token" else np.ascontiguousarray(bits.transpose(1, 0, 2, 3))
+
+
+def _run(P, N, H, C, layout, cu, seed):
+    torch = _torch()
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    dev = torch.device("cuda", 0)
+    ts, ps = _strides(layout, N, P, C, H)
+    plan = U.ulysses_plan(N, H, 128, P, C, ts, ps, 0, cu)
+    Np = plan.padded_tokens
+    S = inputs.qkv_seq(N, H, P, C, seed, dev, layout=layout)
+    Hl = H // P
+    T = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
+    U.ulysses_repack_fwd(plan, S, T)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
+    U.ulysses_attn_fwd(plan, T, OT, 1.0 / math.sqrt(128))
+    back = torch.empty_like(S)
+    U.ulysses_repack_bwd(plan, T, back, C)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+    U.ulysses_layer_fwd(plan, S, OS, ws, fused=0)
+    OSf = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=dev)
+    U.ulysses_layer_fwd(plan, S, OSf, None, fused=1)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    return plan, S, T, OT, back, OS, OSf
+
+
+def _bits(t):
+    from ulysses_sequence_attention_repack_b200 import inputs
+    return inputs.host_bits(t)
+
+
+def _f32(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("P,N,H,C,layout,cu,seed", CASES)
+def test_repack_attention_layer_against_oracle(gpu, P, N, H, C, layout, cu, seed):
+    plan, S, T, OT, back, OS, OSf = _run(P, N, H, C, layout, cu, seed)
+    S_bits = _seq_as_token_major(_bits(S), layout)
+    # step 1: bit-exact
+    T_ref = orc.repack_fwd(S_bits, P)
+    assert np.array_equal(_bits(T), T_ref)
+    # step 3 on all planes: exact round trip
+    assert np.array_equal(_bits(back), _bits(S))
+    # step 2 against fp64 attention on the same bytes
+    scale = 1.0 / math.sqrt(128)
+    O_ref = orc.attention_heads(T_ref, N, scale, cu_seqlens=cu)
+    O_gpu = _f32(OT)
+    err = np.abs(O_gpu - O_ref)
+    assert err.max() <= MAX_ABS, err.max()
+    assert err.mean() <= MEAN_ABS, err.mean()
+    assert np.all(O_gpu[:, N:] == 0)
+    # the whole layer: oracle composition, and fused == unfused bit for bit
+    L_ref = orc.output_repack_bwd(O_ref)
+    L_gpu = _f32(OS)
+    errl = np.abs(L_gpu - L_ref)
+    assert errl.max() <= MAX_ABS and errl.mean() <= MEAN_ABS
+    assert np.array_equal(_bits(OS), _bits(OSf))
+    # step 3 on the attention output equals the layer output bit for bit
+    assert np.array_equal(_bits(OS), orc.repack_bwd(_bits(OT)[:, None])[:, 0])
+
+
+def test_sharp_softmax_diagnostic(gpu):
+    """Q scaled by 8: peaked rows exercise the running-max rescale path."""
+    torch = _torch()
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    dev = torch.device("cuda", 0)
+    P, N, H = 2, 1024, 4
+    plan = U.ulysses_plan(N, H, 128, P, 3)
+    S = inputs.qkv_seq(N, H, P, 3, 21, dev)
+    S[:, 0] *= 8
+    OS = torch.empty((N, H, 128), dtype=torch.bfloat16, device=dev)
+    U.ulysses_layer_fwd(plan, S, OS, None, fused=1)
+    torch.cuda.synchronize()
+    ref = orc.layer_fwd(_bits(S), P, N, 1.0 / math.sqrt(128))
+    err = np.abs(_f32(OS) - ref)
+    assert err.max() <= 4 * MAX_ABS and err.mean() <= MEAN_ABS
+
+
+def test_uniform_keys_give_mean_of_v(gpu):
+    torch = _torch()
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    dev = torch.device("cuda", 0)
+    P, N, H = 2, 700, 4
+    plan = U.ulysses_plan(N, H, 128, P, 3)
+    S = inputs.qkv_seq(N, H, P, 3, 22, dev)
+    S[:N, 1] = S[0:1, 1]      # every key equal
+    OS = torch.empty((N, H, 128), dtype=torch.bfloat16, device=dev)
+    U.ulysses_layer_fwd(plan, S, OS, None, fused=1)
+    torch.cuda.synchronize()
+    v = _f32(S[:N, 2])                                 # [N, H, D]
+    want = np.broadcast_to(v.mean(axis=0, keepdims=True), v.shape)
+    err = np.abs(_f32(OS) - want)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS

@@ -1,0 +1,23 @@
+"""One-GPU Ulysses sequence-parallel attention layer for NVIDIA B200 (sm_100a).
+
+The layer (repack -> attention -> inverse repack) runs in the kernels of
+``libulysses.so``; this package is its Python binding.  Entry points keep the
+names of the C ABI declared in ``include/ulysses.h``.
+"""
+from ._lib import (  # noqa: F401
+    EXPORTS,
+    MAX_SEQS,
+    MAX_WINDOW_BYTES,
+    Plan,
+    UlyssesError,
+    library_path,
+    load,
+    strerror,
+    ulysses_attn_fwd,
+    ulysses_last_device_error,
+    ulysses_layer_fwd,
+    ulysses_layer_fwd_host,
+    ulysses_plan,
+    ulysses_repack_bwd,
+    ulysses_repack_fwd,
+)

@@ -1,0 +1,212 @@
+"""ctypes binding of libulysses.so: argument marshalling only.
+
+Every function has the name of the C entry point it calls and takes torch
+tensors (device memory), plain ints and an optional CUDA stream; all work
+happens in the library's kernels.  There is no fallback: if the library
+cannot be loaded, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from . import build as _build
+
+
+# return codes, as in include/ulysses.h
+ULYSSES_OK = 0
+ULYSSES_ERR_ARG = 1
+ULYSSES_ERR_DIVISIBILITY = 2
+ULYSSES_ERR_ALIGN = 3
+ULYSSES_ERR_WINDOW = 4
+ULYSSES_ERR_WORKSPACE = 5
+ULYSSES_ERR_CUDA = 6
+ULYSSES_ERR_DEVICE = 7
+ULYSSES_ERR_UNSUPPORTED = 8
+MAX_SEQS = 64
+MAX_WINDOW_BYTES = 1024 ** 3
+
+EXPORTS = (
+    "ulysses_plan", "ulysses_plan_destroy", "ulysses_plan_padded_tokens", "ulysses_plan_plane_chunk",
+    "ulysses_plan_window_bytes_per_plane", "ulysses_workspace_bytes", "ulysses_repack_fwd",
+    "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
+    "ulysses_last_device_error", "ulysses_strerror",
+)
+
+
+class UlyssesError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: error {code}: {strerror(code)}")
+
+
+_lock = threading.Lock()
+_handle: ctypes.CDLL | None = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load() -> ctypes.CDLL:
+    """Load (building first if the sources are newer) and type the library."""
+    global _handle
+    with _lock:
+        if _handle is not None:
+            return _handle
+        path = _build.ensure_built()
+        if not os.path.exists(path):
+            raise ImportError(f"libulysses.so missing at {path}")
+        lib = ctypes.CDLL(path)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        lib.ulysses_plan.argtypes = [ctypes.POINTER(vp), i64, i32, i32, i32, i32, i64, i64, i64,
+                                     ctypes.POINTER(ctypes.c_int32), i32]
+        lib.ulysses_plan.restype = ctypes.c_int
+        lib.ulysses_plan_destroy.argtypes = [vp]
+        lib.ulysses_plan_destroy.restype = None
+        lib.ulysses_plan_padded_tokens.argtypes = [vp]
+        lib.ulysses_plan_padded_tokens.restype = i64
+        lib.ulysses_plan_plane_chunk.argtypes = [vp]
+        lib.ulysses_plan_plane_chunk.restype = i32
+        lib.ulysses_plan_window_bytes_per_plane.argtypes = [vp]
+        lib.ulysses_plan_window_bytes_per_plane.restype = i64
+        lib.ulysses_workspace_bytes.argtypes = [vp]
+        lib.ulysses_workspace_bytes.restype = sz
+        lib.ulysses_repack_fwd.argtypes = [vp, vp, vp, vp]
+        lib.ulysses_repack_fwd.restype = ctypes.c_int
+        lib.ulysses_repack_bwd.argtypes = [vp, vp, vp, i32, vp]
+        lib.ulysses_repack_bwd.restype = ctypes.c_int
+        lib.ulysses_attn_fwd.argtypes = [vp, vp, vp, ctypes.c_float, vp]
+        lib.ulysses_attn_fwd.restype = ctypes.c_int
+        lib.ulysses_layer_fwd.argtypes = [vp, vp, vp, vp, sz, i32, vp]
+        lib.ulysses_layer_fwd.restype = ctypes.c_int
+        lib.ulysses_layer_fwd_host.argtypes = [vp, vp, vp, vp, vp, vp, sz, i32, vp]
+        lib.ulysses_layer_fwd_host.restype = ctypes.c_int
+        lib.ulysses_last_device_error.argtypes = [vp, vp]
+        lib.ulysses_last_device_error.restype = ctypes.c_int
+        lib.ulysses_strerror.argtypes = [ctypes.c_int]
+        lib.ulysses_strerror.restype = ctypes.c_char_p
+        _handle = lib
+        return lib
+
+
+def strerror(code: int) -> str:
+    return load().ulysses_strerror(int(code)).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != ULYSSES_OK:
+        raise UlyssesError(code, where)
+
+
+def _ptr(t) -> int | None:
+    """Device (or host) address of a tensor, or an int address as given."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Plan:
+    """Owner of a ulysses_plan_t*; destroyed with the object."""
+
+    def __init__(self, handle: int, N: int, H: int, D: int, P: int, planes: int, cu_seqlens):
+        self._h = ctypes.c_void_p(handle)
+        self.N, self.H, self.D, self.P, self.planes = N, H, D, P, planes
+        self.cu_seqlens = None if cu_seqlens is None else [int(x) for x in cu_seqlens]
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if not self._h:
+            raise ValueError("plan destroyed")
+        return self._h
+
+    @property
+    def padded_tokens(self) -> int:
+        return load().ulysses_plan_padded_tokens(self.handle)
+
+    @property
+    def plane_chunk(self) -> int:
+        return load().ulysses_plan_plane_chunk(self.handle)
+
+    @property
+    def window_bytes_per_plane(self) -> int:
+        return load().ulysses_plan_window_bytes_per_plane(self.handle)
+
+    @property
+    def workspace_bytes(self) -> int:
+        return load().ulysses_workspace_bytes(self.handle)
+
+    def destroy(self) -> None:
+        if self._h:
+            load().ulysses_plan_destroy(self._h)
+            self._h = ctypes.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
+
+
+def ulysses_plan(N: int, H: int, D: int, P: int, planes: int, token_stride: int = 0, plane_stride: int = 0,
+                 plane_chunk: int = 0, cu_seqlens=None) -> Plan:
+    lib = load()
+    h = ctypes.c_void_p()
+    if cu_seqlens is None:
+        arr, ns = None, 0
+    else:
+        vals = [int(x) for x in cu_seqlens]
+        arr = (ctypes.c_int32 * len(vals))(*vals)
+        ns = len(vals) - 1
+    code = lib.ulysses_plan(ctypes.byref(h), int(N), int(H), int(D), int(P), int(planes), int(token_stride),
+                            int(plane_stride), int(plane_chunk), arr, ns)
+    _check(code, "ulysses_plan")
+    return Plan(h.value, N, H, D, P, planes, cu_seqlens)
+
+
+def ulysses_repack_fwd(plan: Plan, src_seq, dst_heads, stream=None) -> None:
+    _check(load().ulysses_repack_fwd(plan.handle, _ptr(src_seq), _ptr(dst_heads), _stream(stream)),
+           "ulysses_repack_fwd")
+
+
+def ulysses_repack_bwd(plan: Plan, src_heads, dst_seq, planes: int, stream=None) -> None:
+    _check(load().ulysses_repack_bwd(plan.handle, _ptr(src_heads), _ptr(dst_seq), int(planes), _stream(stream)),
+           "ulysses_repack_bwd")
+
+
+def ulysses_attn_fwd(plan: Plan, qkv_heads, out_heads, softmax_scale: float, stream=None) -> None:
+    _check(load().ulysses_attn_fwd(plan.handle, _ptr(qkv_heads), _ptr(out_heads), float(softmax_scale),
+                                   _stream(stream)), "ulysses_attn_fwd")
+
+
+def ulysses_layer_fwd(plan: Plan, qkv_seq, out_seq, workspace=None, workspace_bytes: int | None = None,
+                      fused: int = 0, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().ulysses_layer_fwd(plan.handle, _ptr(qkv_seq), _ptr(out_seq), _ptr(workspace),
+                                    int(workspace_bytes), int(fused), _stream(stream)), "ulysses_layer_fwd")
+
+
+def ulysses_layer_fwd_host(plan: Plan, host_qkv_seq, host_out_seq, dev_qkv_seq, dev_out_seq, workspace=None,
+                           workspace_bytes: int | None = None, fused: int = 0, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().ulysses_layer_fwd_host(plan.handle, _ptr(host_qkv_seq), _ptr(host_out_seq), _ptr(dev_qkv_seq),
+                                         _ptr(dev_out_seq), _ptr(workspace), int(workspace_bytes), int(fused),
+                                         _stream(stream)), "ulysses_layer_fwd_host")
+
+
+def ulysses_last_device_error(plan: Plan, stream=None) -> int:
+    return load().ulysses_last_device_error(plan.handle, _stream(stream))

@@ -1,0 +1,352 @@
+// C ABI of the one-GPU Ulysses layer: plan validation, buffer checks and the
+// launch sequence of the three steps.  Declarations and argument contracts
+// are in include/ulysses.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+namespace {
+
+constexpr int32_t kHeadDim = 128;
+constexpr int32_t kMaxHeads = 1024;
+constexpr int32_t kMaxPlanes = 8;
+constexpr int64_t kMaxRows = (int64_t(1) << 31) - 4096;   // kernels index rows with int32
+
+inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlap(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + static_cast<uintptr_t>(bbytes) && y < x + static_cast<uintptr_t>(abytes);
+}
+
+// bytes spanned by the sequence-sharded buffer with the given strides
+inline int64_t seq_extent_bytes(const ulysses_plan_t* p, int32_t planes, int64_t tok, int64_t pl) {
+  return ((p->Np - 1) * tok + static_cast<int64_t>(planes - 1) * pl + static_cast<int64_t>(p->H) * p->D) * 2;
+}
+inline int64_t heads_bytes(const ulysses_plan_t* p, int32_t planes) {
+  return static_cast<int64_t>(p->P) * planes * p->Np * p->Hl * p->D * 2;
+}
+inline int64_t out_seq_bytes(const ulysses_plan_t* p) { return p->Np * p->H * p->D * 2; }
+
+// Launch-time device check: the plan's error word lives on one device.
+int device_ready(const ulysses_plan_t* p) {
+  if (!p || !p->dev_err) return ULYSSES_ERR_CUDA;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return ULYSSES_ERR_CUDA;
+  }
+  return dev == p->device ? ULYSSES_OK : ULYSSES_ERR_ARG;
+}
+
+int status_of(cudaError_t e) {
+  if (e == cudaSuccess) return ULYSSES_OK;
+  cudaGetLastError();
+  return ULYSSES_ERR_CUDA;
+}
+
+int repack_fwd_impl(const ulysses_plan_t* p, const void* src, void* dst, cudaStream_t st) {
+  for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
+    const int32_t cc = std::min(p->plane_chunk, p->C - c0);
+    int s = status_of(ulysses::launch_repack(0, src, dst, p->Np, p->H, p->P, p->C, c0, cc, p->token_stride,
+                                             p->plane_stride, st));
+    if (s != ULYSSES_OK) return s;
+  }
+  return ULYSSES_OK;
+}
+
+// dst layout for mode 1 with `planes` planes (see ulysses_repack_bwd)
+void bwd_dst_strides(const ulysses_plan_t* p, int32_t planes, int64_t* tok, int64_t* pl) {
+  if (planes == p->C) {
+    *tok = p->token_stride;
+    *pl = p->plane_stride;
+  } else {
+    *tok = static_cast<int64_t>(planes) * p->H * p->D;
+    *pl = static_cast<int64_t>(p->H) * p->D;
+  }
+}
+
+int repack_bwd_impl(const ulysses_plan_t* p, const void* src, void* dst, int32_t planes, cudaStream_t st) {
+  int64_t tok, pl;
+  bwd_dst_strides(p, planes, &tok, &pl);
+  // same window rule as the forward direction: at most plane_chunk planes per launch
+  for (int32_t c0 = 0; c0 < planes; c0 += p->plane_chunk) {
+    const int32_t cc = std::min(p->plane_chunk, planes - c0);
+    int s = status_of(ulysses::launch_repack(1, src, dst, p->Np, p->H, p->P, planes, c0, cc, tok, pl, st));
+    if (s != ULYSSES_OK) return s;
+  }
+  return ULYSSES_OK;
+}
+
+int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, float scale, cudaStream_t st) {
+  ulysses::AttnLaunch a;
+  a.base = base;
+  a.fused = fused;
+  a.Np = p->Np;
+  a.N = p->N;
+  a.H = p->H;
+  a.P = p->P;
+  a.Hl = p->Hl;
+  a.C = p->C;
+  a.tok_stride = p->token_stride;
+  a.plane_stride = p->plane_stride;
+  a.out = out;
+  if (fused) {   // O_S [Np, H, D], head h = r*Hl + j
+    a.o_stride_r = static_cast<int64_t>(p->Hl) * p->D;
+    a.o_stride_n = static_cast<int64_t>(p->H) * p->D;
+  } else {       // O_T [P, Np, Hl, D]
+    a.o_stride_r = p->Np * p->Hl * p->D;
+    a.o_stride_n = static_cast<int64_t>(p->Hl) * p->D;
+  }
+  a.o_stride_j = p->D;
+  a.scale = scale;
+  a.plan = p;
+  return status_of(ulysses::launch_attn(a, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int ulysses_plan(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
+                 int64_t token_stride, int64_t plane_stride, int64_t plane_chunk, const int32_t* cu_seqlens_host,
+                 int32_t num_seqs) {
+  if (!out) return ULYSSES_ERR_ARG;
+  *out = nullptr;
+  if (D != kHeadDim) return ULYSSES_ERR_UNSUPPORTED;
+  if (N < 1 || H < 1 || P < 1 || planes < 1 || planes > kMaxPlanes) return ULYSSES_ERR_ARG;
+  if (H > kMaxHeads) return ULYSSES_ERR_UNSUPPORTED;
+  if (P > H || H % P != 0) return ULYSSES_ERR_DIVISIBILITY;
+  const int64_t Nl = (N + P - 1) / P;
+  const int64_t Np = Nl * P;
+  if (Np > kMaxRows) return ULYSSES_ERR_UNSUPPORTED;
+
+  // strides of the sequence-sharded input (elements)
+  const int64_t row = static_cast<int64_t>(H) * D;
+  if (token_stride == 0 && plane_stride == 0) {
+    token_stride = planes * row;
+    plane_stride = row;
+  }
+  if (token_stride <= 0 || plane_stride <= 0) return ULYSSES_ERR_ARG;
+  if (token_stride % 8 || plane_stride % 8) return ULYSSES_ERR_ALIGN;
+  const bool token_major = plane_stride >= row && token_stride >= (planes - 1) * plane_stride + row;
+  const bool plane_major = token_stride >= row && plane_stride >= (Np - 1) * token_stride + row;
+  if (!token_major && !plane_major && planes > 1) return ULYSSES_ERR_ARG;   // rows would overlap
+  if (planes == 1 && token_stride < row) return ULYSSES_ERR_ARG;
+
+  // window: bytes per rank per plane, and planes per launch
+  const int64_t per_plane = Nl * row * 2;
+  if (per_plane > ULYSSES_MAX_WINDOW_BYTES) return ULYSSES_ERR_WINDOW;
+  int64_t chunk = plane_chunk;
+  if (chunk == 0) chunk = std::min<int64_t>(planes, ULYSSES_MAX_WINDOW_BYTES / per_plane);
+  if (chunk < 1 || chunk > planes) return ULYSSES_ERR_ARG;
+  if (chunk * per_plane > ULYSSES_MAX_WINDOW_BYTES) return ULYSSES_ERR_WINDOW;
+
+  // packed sequences
+  ulysses::Segment segs[ULYSSES_MAX_SEQS];
+  int32_t nseq = 0;
+  if (cu_seqlens_host == nullptr || num_seqs == 0) {
+    if (cu_seqlens_host == nullptr && num_seqs != 0) return ULYSSES_ERR_ARG;
+    segs[0] = {0, static_cast<int32_t>(N)};
+    nseq = 1;
+  } else {
+    if (num_seqs < 0) return ULYSSES_ERR_ARG;
+    if (num_seqs > ULYSSES_MAX_SEQS) return ULYSSES_ERR_UNSUPPORTED;
+    if (cu_seqlens_host[0] != 0 || cu_seqlens_host[num_seqs] != N) return ULYSSES_ERR_ARG;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+      if (cu_seqlens_host[s + 1] < cu_seqlens_host[s]) return ULYSSES_ERR_ARG;
+      segs[s] = {cu_seqlens_host[s], cu_seqlens_host[s + 1]};
+    }
+    nseq = num_seqs;
+  }
+
+  ulysses_plan_t* p = new (std::nothrow) ulysses_plan_t;
+  if (!p) return ULYSSES_ERR_ARG;
+  std::memset(p, 0, sizeof(*p));
+  p->N = N;
+  p->Np = Np;
+  p->Nl = Nl;
+  p->H = H;
+  p->D = D;
+  p->P = P;
+  p->Hl = H / P;
+  p->C = planes;
+  p->token_stride = token_stride;
+  p->plane_stride = plane_stride;
+  p->plane_chunk = static_cast<int32_t>(chunk);
+  p->num_seqs = nseq;
+  std::memcpy(p->segs, segs, sizeof(ulysses::Segment) * nseq);
+  p->device = -1;
+  p->dev_err = nullptr;
+
+  // device error word (16 bytes) on the current device; absent without a GPU
+  int dev = -1;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    void* e = nullptr;
+    if (cudaMalloc(&e, 16) == cudaSuccess) {
+      if (cudaMemset(e, 0, 16) == cudaSuccess) {
+        p->dev_err = static_cast<unsigned int*>(e);
+        p->device = dev;
+      } else {
+        cudaFree(e);
+      }
+    }
+  }
+  cudaGetLastError();   // a missing device is not an error of plan creation
+  *out = p;
+  return ULYSSES_OK;
+}
+
+void ulysses_plan_destroy(ulysses_plan_t* plan) {
+  if (!plan) return;
+  if (plan->dev_err) {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != plan->device) cudaSetDevice(plan->device);
+    cudaFree(plan->dev_err);
+    if (cur >= 0 && cur != plan->device) cudaSetDevice(cur);
+    cudaGetLastError();
+  }
+  delete plan;
+}
+
+int64_t ulysses_plan_padded_tokens(const ulysses_plan_t* plan) { return plan ? plan->Np : -1; }
+
+int32_t ulysses_plan_plane_chunk(const ulysses_plan_t* plan) { return plan ? plan->plane_chunk : -1; }
+
+int64_t ulysses_plan_window_bytes_per_plane(const ulysses_plan_t* plan) {
+  return plan ? plan->Nl * plan->H * plan->D * 2 : -1;
+}
+
+size_t ulysses_workspace_bytes(const ulysses_plan_t* plan) {
+  if (!plan) return 0;
+  return static_cast<size_t>(align_up(heads_bytes(plan, plan->C), 256) + align_up(heads_bytes(plan, 1), 256));
+}
+
+int ulysses_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads, void* stream) {
+  if (!plan || !src_seq || !dst_heads) return ULYSSES_ERR_ARG;
+  if (!aligned16(src_seq) || !aligned16(dst_heads)) return ULYSSES_ERR_ALIGN;
+  if (overlap(src_seq, seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride), dst_heads,
+              heads_bytes(plan, plan->C)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  return repack_fwd_impl(plan, src_seq, dst_heads, static_cast<cudaStream_t>(stream));
+}
+
+int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* dst_seq, int32_t planes,
+                       void* stream) {
+  if (!plan || !src_heads || !dst_seq) return ULYSSES_ERR_ARG;
+  if (planes < 1 || planes > plan->C) return ULYSSES_ERR_ARG;
+  if (!aligned16(src_heads) || !aligned16(dst_seq)) return ULYSSES_ERR_ALIGN;
+  int64_t tok, pl;
+  bwd_dst_strides(plan, planes, &tok, &pl);
+  if (overlap(src_heads, heads_bytes(plan, planes), dst_seq, seq_extent_bytes(plan, planes, tok, pl)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  return repack_bwd_impl(plan, src_heads, dst_seq, planes, static_cast<cudaStream_t>(stream));
+}
+
+int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, float softmax_scale,
+                     void* stream) {
+  if (!plan || !qkv_heads || !out_heads) return ULYSSES_ERR_ARG;
+  if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
+  if (!aligned16(qkv_heads) || !aligned16(out_heads)) return ULYSSES_ERR_ALIGN;
+  if (overlap(qkv_heads, heads_bytes(plan, plan->C), out_heads, heads_bytes(plan, 1))) return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  return attn_impl(plan, qkv_heads, 0, out_heads, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
+                      size_t workspace_bytes, int32_t fused, void* stream) {
+  if (!plan || !qkv_seq || !out_seq) return ULYSSES_ERR_ARG;
+  if (plan->C < 3 || (fused != 0 && fused != 1)) return ULYSSES_ERR_ARG;
+  if (!aligned16(qkv_seq) || !aligned16(out_seq)) return ULYSSES_ERR_ALIGN;
+  const int64_t in_bytes = seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride);
+  if (overlap(qkv_seq, in_bytes, out_seq, out_seq_bytes(plan))) return ULYSSES_ERR_ARG;
+  const float scale = 1.0f / std::sqrt(static_cast<float>(plan->D));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fused) {
+    int s = device_ready(plan);
+    if (s != ULYSSES_OK) return s;
+    return attn_impl(plan, qkv_seq, 1, out_seq, scale, st);
+  }
+  if (!workspace) return ULYSSES_ERR_WORKSPACE;
+  if (workspace_bytes < ulysses_workspace_bytes(plan)) return ULYSSES_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ULYSSES_ERR_ALIGN;
+  const int64_t ws = static_cast<int64_t>(ulysses_workspace_bytes(plan));
+  if (overlap(workspace, ws, qkv_seq, in_bytes) || overlap(workspace, ws, out_seq, out_seq_bytes(plan)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  uint8_t* T = static_cast<uint8_t*>(workspace);
+  uint8_t* OT = T + align_up(heads_bytes(plan, plan->C), 256);
+  if ((s = repack_fwd_impl(plan, qkv_seq, T, st)) != ULYSSES_OK) return s;
+  if ((s = attn_impl(plan, T, 0, OT, scale, st)) != ULYSSES_OK) return s;
+  return repack_bwd_impl(plan, OT, out_seq, 1, st);
+}
+
+int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
+                           void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
+                           int32_t fused, void* stream) {
+  if (!plan || !host_qkv_seq || !host_out_seq || !dev_qkv_seq || !dev_out_seq) return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t in_bytes = seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride);
+  if (cudaMemcpyAsync(dev_qkv_seq, host_qkv_seq, static_cast<size_t>(in_bytes), cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return status_of(cudaErrorUnknown);
+  s = ulysses_layer_fwd(plan, dev_qkv_seq, dev_out_seq, workspace, workspace_bytes, fused, stream);
+  if (s != ULYSSES_OK) return s;
+  if (cudaMemcpyAsync(host_out_seq, dev_out_seq, static_cast<size_t>(out_seq_bytes(plan)), cudaMemcpyDeviceToHost,
+                      st) != cudaSuccess)
+    return status_of(cudaErrorUnknown);
+  return ULYSSES_OK;
+}
+
+int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream) {
+  if (!plan || !plan->dev_err) return -1;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, plan->dev_err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  if (v != 0 && cudaMemset(plan->dev_err, 0, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return static_cast<int>(v);
+}
+
+const char* ulysses_strerror(int code) {
+  switch (code) {
+    case ULYSSES_OK: return "ok";
+    case ULYSSES_ERR_ARG: return "invalid argument (null or overlapping pointer, bad size or cu_seqlens)";
+    case ULYSSES_ERR_DIVISIBILITY: return "heads are not divisible by the number of ranks";
+    case ULYSSES_ERR_ALIGN: return "pointer or stride is not 16-byte aligned";
+    case ULYSSES_ERR_WINDOW: return "one plane per rank exceeds the 1 GiB window";
+    case ULYSSES_ERR_WORKSPACE: return "workspace missing or too small";
+    case ULYSSES_ERR_CUDA: return "CUDA call failed or no CUDA device";
+    case ULYSSES_ERR_DEVICE: return "a kernel reported an error";
+    case ULYSSES_ERR_UNSUPPORTED: return "unsupported configuration";
+    default: return "unknown error code";
+  }
+}
+
+}  // extern "C"

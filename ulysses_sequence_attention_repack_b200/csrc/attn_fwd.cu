@@ -1,0 +1,524 @@
+// Non-causal softmax attention for the Ulysses layer on sm_100a.
+//
+//   O[n, :] = sum_{m in K(n)} softmax_m(scale * <Q_n, K_m>) V_m
+//
+// (the FA4 backend call of flash_attn_cute.py in "hao-ai-lab FastVideo,
+// compare aryan/h3-nvfp4-stack-speedups...main": softmax_scale, non-causal,
+// varlen through cu_seqlens).  K(n) is the key range of the packed sequence
+// holding row n.  Computed flash-style: keys are visited in tiles of 128 and
+// the softmax is kept online (running max and sum), so the N x N score matrix
+// never leaves the SM.
+//
+// Design (one persistent CTA per SM, 10 warps):
+//   warp 9      TMA producer: Q tiles (2 x 128 rows) and a 2-stage K ring and
+//               V ring, 128-byte swizzled, completion counted on mbarriers.
+//   warp 8      tcgen05 issuer (one lane): S_i = Q_i K^T into TMEM (fp32),
+//               then O_i += P_i V with P_i read from TMEM (bf16, aliased over
+//               S_i) and V from shared memory.  Two Q tiles ping-pong so the
+//               tensor core works on one tile while the other is in softmax.
+//   warps 0-7   two softmax warpgroups, one per Q tile; thread t of a group
+//               owns query row t, so row max and row sum need no shuffles.
+//               The running max is only moved (and O rescaled in TMEM) when
+//               it grows by more than 8 in log2 units; the final 1/l uses the
+//               same stale max, so the result is unchanged.
+// TMEM: S0 | S1 | O0 | O1, 128 fp32 columns each (all 512 columns).
+//
+// Every wait is bounded: on timeout the kernel sets an error bit, skips the
+// remaining work, waits (bounded) for its own in-flight copies and MMAs,
+// frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace ulysses {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+constexpr int BM = 128;            // query rows per tile
+constexpr int BN = 128;            // keys per tile
+constexpr int HD = 128;            // head dim
+constexpr int kUnitRows = 2 * BM;  // query rows per work unit (two tiles)
+constexpr uint32_t kHalfBytes = BM * 64 * 2;   // one 128-row x 64-column swizzled box: 16 KB
+constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 x 128 bf16: 32 KB
+constexpr int kStages = 2;
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s per wait
+
+// shared memory map (offsets from a 1024-aligned base)
+constexpr uint32_t kOffQ = 0;                                  // [2 tiles][2 halves] 64 KB
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;             // [stages] 64 KB
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;       // [stages] 64 KB
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+// barrier indices
+enum {
+  B_QFULL0 = 0, B_QFULL1, B_QEMPTY,
+  B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1,
+  B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,
+  B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1,
+  B_OFULL0, B_OFULL1, B_OEMPTY0, B_OEMPTY1,
+  B_DONE, B_COUNT
+};
+constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;           // TMEM base address
+constexpr uint32_t kOffAbort = kOffSlot + 4;
+constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;          // + alignment slack
+
+// TMEM columns
+constexpr uint32_t kColS0 = 0, kColO0 = 256;
+
+constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);    // Q, K both K-major (head dim contiguous)
+constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, 0, 1);   // P from TMEM, V MN-major (head dim contiguous)
+
+struct SegDesc {
+  int32_t start;       // first query row and first key
+  int32_t kv_end;      // one past the last key
+  int32_t q_end;       // one past the last query row this segment writes (Np for the last segment)
+  int32_t nqb;         // 256-row query blocks
+  int32_t unit_base;   // first work unit of this segment
+};
+
+struct AttnParams {
+  __nv_bfloat16* out;
+  unsigned int* err;
+  int64_t o_stride_r, o_stride_n, o_stride_j;
+  int32_t N, Np;
+  int32_t Hl, P, fused;
+  int32_t num_units, nseg;
+  float scale_log2;
+  SegDesc seg[ULYSSES_MAX_SEQS];   // longest first
+};
+
+struct Unit {
+  int seg, r, j, q0;
+};
+
+__device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& w) {
+  int s = 0;
+  while (s + 1 < p.nseg && u >= p.seg[s + 1].unit_base) ++s;
+  const int local = u - p.seg[s].unit_base;
+  const int nqb = p.seg[s].nqb;
+  const int rh = local / nqb;         // (rank, head) major, query block minor: CTAs running
+  const int qb = local - rh * nqb;    // side by side share one head's K/V in L2
+  w.seg = s;
+  w.r = rh / p.Hl;
+  w.j = rh - w.r * p.Hl;
+  w.q0 = p.seg[s].start + qb * kUnitRows;
+  return local >= 0 && w.r < p.P;
+}
+
+// waits that ignore the abort flag (used for draining in-flight work)
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kOffBar;
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffSlot);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  WaitGuard g{abort_flag, p.err, kWaitLimitNs};
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(BAR(B_QFULL0), 1);
+    mbar_init(BAR(B_QFULL1), 1);
+    mbar_init(BAR(B_QEMPTY), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(BAR(B_KFULL0 + s), 1);
+      mbar_init(BAR(B_KEMPTY0 + s), 1);
+      mbar_init(BAR(B_VFULL0 + s), 1);
+      mbar_init(BAR(B_VEMPTY0 + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(B_SFULL0 + i), 1);
+      mbar_init(BAR(B_PFULL0 + i), BM);
+      mbar_init(BAR(B_OFULL0 + i), 1);
+      mbar_init(BAR(B_OEMPTY0 + i), BM);
+    }
+    mbar_init(BAR(B_DONE), 1);
+    fence_mbar_init();
+  }
+  if (warp == kTmaWarp && lane == 0) prefetch_tmap(&tmap);
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kc = 0, vc = 0, uc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+        Unit w;
+        if (!decode_unit(p, u, w)) {
+          atomicOr(p.err, kErrBadUnit);
+          break;
+        }
+        const SegDesc& sd = p.seg[w.seg];
+        const int hc = p.fused ? w.r * p.Hl + w.j : w.j;   // head coordinate
+        const int rc = p.fused ? 0 : w.r;                  // rank coordinate
+        if (uc > 0 && !(ok = mbar_wait(BAR(B_QEMPTY), (uc - 1) & 1, g))) break;
+        for (int i = 0; i < 2; ++i) {
+          mbar_arrive_expect_tx(BAR(B_QFULL0 + i), kTileBytes);
+          for (int h = 0; h < 2; ++h)
+            tma_load_5d(sbase + kOffQ + (2 * i + h) * kHalfBytes, &tmap, BAR(B_QFULL0 + i), 64 * h, hc,
+                        w.q0 + i * BM, 0, rc);
+        }
+        const int nkv = (sd.kv_end - sd.start + BN - 1) / BN;
+        for (int t = 0; t < nkv; ++t) {
+          const int kv0 = sd.start + t * BN;
+          {
+            const uint32_t s = kc % kStages, ph = (kc / kStages) & 1;
+            if (kc >= kStages && !(ok = mbar_wait(BAR(B_KEMPTY0 + s), ph ^ 1, g))) break;
+            mbar_arrive_expect_tx(BAR(B_KFULL0 + s), kTileBytes);
+            for (int h = 0; h < 2; ++h)
+              tma_load_5d(sbase + kOffK + s * kTileBytes + h * kHalfBytes, &tmap, BAR(B_KFULL0 + s), 64 * h, hc,
+                          kv0, 1, rc);
+            ++kc;
+          }
+          {
+            const uint32_t s = vc % kStages, ph = (vc / kStages) & 1;
+            if (vc >= kStages && !(ok = mbar_wait(BAR(B_VEMPTY0 + s), ph ^ 1, g))) break;
+            mbar_arrive_expect_tx(BAR(B_VFULL0 + s), kTileBytes);
+            for (int h = 0; h < 2; ++h)
+              tma_load_5d(sbase + kOffV + s * kTileBytes + h * kHalfBytes, &tmap, BAR(B_VFULL0 + s), 64 * h, hc,
+                          kv0, 2, rc);
+            ++vc;
+          }
+        }
+      }
+      // drain: every copy this thread issued has landed before the CTA exits
+      if (uc > 0) {
+        drain_wait(BAR(B_QFULL0), (uc - 1) & 1);
+        drain_wait(BAR(B_QFULL1), (uc - 1) & 1);
+      }
+      for (uint32_t n = (kc > kStages ? kc - kStages : 0); n < kc; ++n)
+        drain_wait(BAR(B_KFULL0 + n % kStages), (n / kStages) & 1);
+      for (uint32_t n = (vc > kStages ? vc - kStages : 0); n < vc; ++n)
+        drain_wait(BAR(B_VFULL0 + n % kStages), (n / kStages) & 1);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ tcgen05 issuer
+    if (lane == 0) {
+      uint32_t kc = 0, vc = 0, uc = 0, pc = 0;
+      bool ok = true;
+      auto issue_s = [&](int i, uint32_t ks) {
+        const uint32_t qa = sbase + kOffQ + 2 * i * kHalfBytes;
+        const uint32_t ka = sbase + kOffK + ks * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          mma_ss(tmem + kColS0 + 128 * i, desc_sw128(qa + off, 16, 1024), desc_sw128(ka + off, 16, 1024),
+                 kIdescS, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int i, uint32_t vs, uint32_t acc) {
+        const uint32_t va = sbase + kOffV + vs * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          mma_ts(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 8 * kk,
+                 desc_sw128(va + kk * 2048, kHalfBytes, 1024), kIdescPV, (acc | kk) != 0);
+        }
+      };
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+        Unit w;
+        if (!decode_unit(p, u, w)) break;
+        const SegDesc& sd = p.seg[w.seg];
+        const int nkv = (sd.kv_end - sd.start + BN - 1) / BN;
+        if (!(ok = mbar_wait(BAR(B_QFULL0), uc & 1, g))) break;
+        if (!(ok = mbar_wait(BAR(B_QFULL1), uc & 1, g))) break;
+        uint32_t ks = kc % kStages;
+        if (!(ok = mbar_wait(BAR(B_KFULL0 + ks), (kc / kStages) & 1, g))) break;
+        tc_fence_after();
+        issue_s(0, ks);
+        mma_commit(BAR(B_SFULL0));
+        issue_s(1, ks);
+        mma_commit(BAR(B_SFULL1));
+        mma_commit(BAR(B_KEMPTY0 + ks));
+        ++kc;
+        if (nkv == 1) mma_commit(BAR(B_QEMPTY));
+        for (int t = 0; ok && t < nkv; ++t) {
+          const uint32_t vs = vc % kStages;
+          if (!(ok = mbar_wait(BAR(B_VFULL0 + vs), (vc / kStages) & 1, g))) break;
+          for (int i = 0; i < 2; ++i) {
+            if (t == 0 && uc > 0 && !(ok = mbar_wait(BAR(B_OEMPTY0 + i), (uc - 1) & 1, g))) break;
+            if (!(ok = mbar_wait(BAR(B_PFULL0 + i), pc & 1, g))) break;
+            tc_fence_after();
+            issue_pv(i, vs, t > 0);
+            if (t == nkv - 1) {
+              mma_commit(BAR(B_OFULL0 + i));
+            } else if (i == 0) {
+              ks = kc % kStages;
+              if (!(ok = mbar_wait(BAR(B_KFULL0 + ks), (kc / kStages) & 1, g))) break;
+              tc_fence_after();
+              issue_s(0, ks);
+              mma_commit(BAR(B_SFULL0));
+            } else {
+              issue_s(1, ks);
+              mma_commit(BAR(B_SFULL1));
+              mma_commit(BAR(B_KEMPTY0 + ks));
+              ++kc;
+              if (t + 1 == nkv - 1) mma_commit(BAR(B_QEMPTY));
+            }
+          }
+          ++pc;
+          if (!ok) break;
+          mma_commit(BAR(B_VEMPTY0 + vs));
+          ++vc;
+        }
+      }
+      // drain: all MMAs this thread issued are complete before TMEM is freed
+      mma_commit(BAR(B_DONE));
+      drain_wait(BAR(B_DONE), 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;                  // Q tile 0 or 1
+    const int row = threadIdx.x & 127;         // query row inside the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + kColS0 + 128 * wg;
+    const uint32_t tO = tmem + lane_base + kColO0 + 128 * wg;
+    const float sl2 = p.scale_log2;
+    uint32_t sc = 0, uc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+      Unit w;
+      if (!decode_unit(p, u, w)) break;
+      const SegDesc& sd = p.seg[w.seg];
+      const int nkv = (sd.kv_end - sd.start + BN - 1) / BN;
+      float m_used = -INFINITY;   // running max, log2 units (scaled)
+      float l = 0.f;              // running sum of exp2(x - m_used)
+      for (int t = 0; t < nkv; ++t) {
+        if (!(ok = mbar_wait_warp(BAR(B_SFULL0 + wg), sc & 1, g))) break;
+        ++sc;
+        tc_fence_after();
+        uint32_t sraw[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sraw[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_regs_ready(sraw[c]);
+        float* s = reinterpret_cast<float*>(&sraw[0][0]);
+        if (t == nkv - 1) {
+          const int valid = sd.kv_end - (sd.start + t * BN);   // 1..128
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_used, mx * sl2);
+        // Move the running max only when it grew by more than 8 (log2 units):
+        // probabilities stay below 2^8 and O is rescaled rarely.
+        bool need = false;
+        float f = 1.0f;
+        if (t == 0) {
+          m_used = m_new;
+        } else if (m_new - m_used > 8.0f) {
+          need = true;
+          f = ex2_approx(m_used - m_new);
+          l *= f;
+          m_used = m_new;
+        }
+        const float neg_m = -m_used;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = ex2_approx(fmaf(s[64 * half + 2 * c], sl2, neg_m));
+            const float p1 = ex2_approx(fmaf(s[64 * half + 2 * c + 1], sl2, neg_m));
+            l += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + 32 * half, pk);   // P (bf16 pairs) over the first 64 columns of S
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // O holds the sum of earlier tiles (complete: S of this tile was
+          // issued after them); scale it to the new max before the next P V.
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld();
+            tmem_regs_ready(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tO + 32 * c, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PFULL0 + wg));
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16 -> global
+      if (!(ok = mbar_wait_warp(BAR(B_OFULL0 + wg), uc & 1, g))) break;
+      tc_fence_after();
+      uint32_t oraw[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tO + 32 * c, oraw[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_regs_ready(oraw[c]);
+      tc_fence_before();
+      mbar_arrive(BAR(B_OEMPTY0 + wg));
+      const int n = w.q0 + wg * BM + row;
+      if (n < sd.q_end && n < p.Np) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + w.r * p.o_stride_r + static_cast<int64_t>(n) * p.o_stride_n +
+                                              w.j * p.o_stride_j);
+        const bool pad = n >= p.N;   // pad rows are written as zeros
+        const float inv = 1.0f / l;
+        const float* o = reinterpret_cast<const float*>(&oraw[0][0]);
+#pragma unroll
+        for (int v = 0; v < 16; ++v) {
+          uint4 q;
+          q.x = pack_bf16x2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+          q.y = pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+          q.z = pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+          q.w = pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+          if (pad) q = make_uint4(0u, 0u, 0u, 0u);
+          dst[v] = q;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
+  const ulysses_plan_t* pl = a.plan;
+  EncodeTiledFn encode = get_encode_fn();
+  if (!encode) return cudaErrorNotSupported;
+
+  // 5-D view (d, head, token, plane, rank) of the Q/K/V source
+  cuuint64_t dims[5], strides[4];
+  dims[0] = HD;
+  if (!a.fused) {
+    dims[1] = a.Hl;
+    dims[2] = a.Np;
+    dims[3] = a.C;
+    dims[4] = a.P;
+    strides[0] = HD * 2;
+    strides[1] = static_cast<cuuint64_t>(a.Hl) * HD * 2;
+    strides[2] = static_cast<cuuint64_t>(a.Np) * a.Hl * HD * 2;
+    strides[3] = static_cast<cuuint64_t>(a.C) * a.Np * a.Hl * HD * 2;
+  } else {
+    dims[1] = a.H;
+    dims[2] = a.Np;
+    dims[3] = a.C;
+    dims[4] = 1;
+    strides[0] = HD * 2;
+    strides[1] = static_cast<cuuint64_t>(a.tok_stride) * 2;
+    strides[2] = static_cast<cuuint64_t>(a.plane_stride) * 2;
+    strides[3] = std::max<cuuint64_t>(strides[1] * a.Np, strides[2] * a.C);
+  }
+  cuuint32_t box[5] = {64, 1, BM, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUtensorMap tmap;
+  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(a.base), dims, strides, box,
+                       estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.err = pl->dev_err;
+  p.o_stride_r = a.o_stride_r;
+  p.o_stride_n = a.o_stride_n;
+  p.o_stride_j = a.o_stride_j;
+  p.N = static_cast<int32_t>(a.N);
+  p.Np = static_cast<int32_t>(a.Np);
+  p.Hl = a.Hl;
+  p.P = a.P;
+  p.fused = a.fused;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+
+  // Non-empty segments, longest first.  The segment that ends at N also
+  // covers the pad query rows [N, Np), which are written as zeros.
+  int order[ULYSSES_MAX_SEQS];
+  int nseg = 0;
+  for (int s = 0; s < pl->num_seqs; ++s)
+    if (pl->segs[s].end > pl->segs[s].start) order[nseg++] = s;
+  std::stable_sort(order, order + nseg, [&](int x, int y) {
+    return (pl->segs[x].end - pl->segs[x].start) > (pl->segs[y].end - pl->segs[y].start);
+  });
+  int units = 0;
+  for (int k = 0; k < nseg; ++k) {
+    const ulysses::Segment& sg = pl->segs[order[k]];
+    SegDesc& d = p.seg[k];
+    d.start = sg.start;
+    d.kv_end = sg.end;
+    d.q_end = (sg.end == a.N) ? static_cast<int32_t>(a.Np) : sg.end;
+    d.nqb = (d.q_end - d.start + kUnitRows - 1) / kUnitRows;
+    d.unit_base = units;
+    units += d.nqb * a.P * a.Hl;
+  }
+  p.nseg = nseg;
+  p.num_units = units;
+  if (units == 0) return cudaSuccess;
+
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr_set[64] = {false};
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int grid = std::min(units, sms);
+  attn_fwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmap, p);
+  return cudaGetLastError();
+}
+
+}  // namespace ulysses

@@ -1,0 +1,53 @@
+// Host-side declarations shared by the C ABI (api.cpp) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/ulysses.h"
+
+namespace ulysses {
+
+struct Segment {
+  int32_t start, end;   // key / query range [start, end) of one packed sequence
+};
+
+}  // namespace ulysses
+
+struct ulysses_plan_s {
+  int64_t N, Np, Nl;
+  int32_t H, D, P, Hl, C;
+  int64_t token_stride, plane_stride;   // elements, sequence-sharded input
+  int32_t plane_chunk;
+  int32_t num_seqs;
+  ulysses::Segment segs[ULYSSES_MAX_SEQS];
+  int32_t device;                       // device the plan's scratch lives on (-1: none)
+  unsigned int* dev_err;                // device error word (16 bytes allocated)
+};
+
+namespace ulysses {
+
+// One repack launch over planes [c0, c0 + cc).
+//   dir = 0: seq -> heads (mode 0), dir = 1: heads -> seq (mode 1).
+//   seq side: element (n, c, h, d) at n*tok_stride + c*plane_stride + h*D + d
+//   head side: [P, Ctot, Np, Hl, D]
+cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
+                          int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream);
+
+// Attention launch description (filled by api.cpp).
+struct AttnLaunch {
+  const void* base;        // Q/K/V source buffer
+  int fused;               // 0: head-sharded T; 1: sequence-sharded S (plan strides)
+  int64_t Np, N;
+  int32_t H, P, Hl, C;
+  int64_t tok_stride, plane_stride;     // for fused = 1
+  void* out;
+  int64_t o_stride_r, o_stride_n, o_stride_j;   // elements
+  float scale;
+  const ulysses_plan_t* plan;
+};
+
+cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream);
+
+}  // namespace ulysses

@@ -1,0 +1,126 @@
+// Ulysses repack on one GPU: the all-to-all index map between the
+// sequence-sharded layout and the head-sharded layout.
+//
+//   mode 0 (dir = 0): T[r, c, n, j, d] = S[n, c, r*Hl + j, d]
+//   mode 1 (dir = 1): S[n, c, r*Hl + j, d] = T[r, c, n, j, d]
+//
+// Shapes follow the mode comment above ulysses_a2a_tuned ("hao-ai-lab
+// FastVideo, compare main...perf/ulysses-h3-adaptive",
+// csrc/comm/ulysses_all_to_all.cu): [B, S_local, H, D] <-> [B, S_global, H_local, D],
+// with each of the P source slabs contributing its rows in rank order.
+//
+// Pure data movement, HBM bound.  For one (token n, plane c) the sequence side
+// is one contiguous run of H*D*2 bytes; it splits into P contiguous runs of
+// Hl*D*2 bytes on the head side.  One warp moves one (n, c) run with 16-byte
+// vector loads and stores: 32 lanes cover 512 contiguous bytes per step on
+// both sides, and every lane keeps UNROLL loads in flight before storing.
+// Destination offsets of each head are precomputed in shared memory so the
+// inner loop has no division.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+
+namespace ulysses {
+namespace {
+
+constexpr int kRepackThreads = 256;
+constexpr int kUnroll = 8;
+constexpr int kMaxHeads = 1024;
+
+__device__ __forceinline__ int4 ld_stream(const int4* p) {
+  int4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_stream(int4* p, int4 v) {
+  asm volatile("st.global.cs.v4.s32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Element offsets are int64 throughout: the largest head-sharded buffer holds
+// 7.2e9 elements.
+template <int DIR>
+__global__ void __launch_bounds__(kRepackThreads) repack_kernel(const int4* __restrict__ src,
+                                                                int4* __restrict__ dst, int64_t Np, int32_t H,
+                                                                int32_t Hl, int32_t Ctot, int32_t c0, int32_t cc,
+                                                                int64_t tok_stride, int64_t plane_stride) {
+  // head_off[h]: element offset of head h's run inside a head-sharded row,
+  // relative to T[0, c, n, 0, 0]: r*Ctot*Np*Hl*D + j*D with r = h / Hl, j = h % Hl.
+  __shared__ int64_t head_off[kMaxHeads];
+  constexpr int D = 128;
+  const int64_t rank_stride = static_cast<int64_t>(Ctot) * Np * Hl * D;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    const int r = h / Hl, j = h - (h / Hl) * Hl;
+    head_off[h] = r * rank_stride + static_cast<int64_t>(j) * D;
+  }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = Np * cc;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int vec_per_row = H * (D / 8);   // 16-byte vectors in one (n, c) run
+
+  for (int64_t row = warp0; row < rows; row += nwarps) {
+    // plane-major over the chunk: consecutive warps take consecutive tokens
+    const int c = c0 + static_cast<int>(row / Np);
+    const int64_t n = row - (row / Np) * Np;
+    const int64_t seq_base = n * tok_stride + c * plane_stride;                 // elements
+    const int64_t head_base = (static_cast<int64_t>(c) * Np + n) * Hl * D;       // elements, + head_off[h]
+    for (int k0 = 0; k0 < vec_per_row; k0 += 32 * kUnroll) {
+      int4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int k = k0 + u * 32 + lane;
+        if (k < vec_per_row) {
+          const int h = k >> 4;
+          const int64_t seq_off = seq_base + static_cast<int64_t>(k) * 8;
+          const int64_t head_el = head_base + head_off[h] + (k & 15) * 8;
+          v[u] = ld_stream(src + ((DIR == 0 ? seq_off : head_el) >> 3));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int k = k0 + u * 32 + lane;
+        if (k < vec_per_row) {
+          const int h = k >> 4;
+          const int64_t seq_off = seq_base + static_cast<int64_t>(k) * 8;
+          const int64_t head_el = head_base + head_off[h] + (k & 15) * 8;
+          st_stream(dst + ((DIR == 0 ? head_el : seq_off) >> 3), v[u]);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
+                          int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream) {
+  if (H > kMaxHeads || P < 1 || H % P != 0) return cudaErrorInvalidValue;
+  const int64_t rows = Np * cc;
+  if (rows == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int warps_per_cta = kRepackThreads / 32;
+  // persistent grid: 8 resident CTAs of 256 threads per SM
+  const int64_t want = (rows + warps_per_cta - 1) / warps_per_cta;
+  const int grid = static_cast<int>(want < static_cast<int64_t>(sms) * 8 ? want : static_cast<int64_t>(sms) * 8);
+  const int Hl = H / P;
+  if (dir == 0) {
+    repack_kernel<0><<<grid, kRepackThreads, 0, stream>>>(static_cast<const int4*>(src), static_cast<int4*>(dst),
+                                                          Np, H, Hl, Ctot, c0, cc, tok_stride, plane_stride);
+  } else {
+    repack_kernel<1><<<grid, kRepackThreads, 0, stream>>>(static_cast<const int4*>(src), static_cast<int4*>(dst),
+                                                          Np, H, Hl, Ctot, c0, cc, tok_stride, plane_stride);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ulysses

@@ -194,7 +194,8 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) ->
 
 
 def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
-                    rows: np.ndarray | None = None) -> np.ndarray:
+                    rows: np.ndarray | None = None, workers: int = 1,
+                    row_block: int = 256) -> np.ndarray:
     """Step two of the layer: attention on every head-sharded slab.
 
     T: head-sharded ``[P, C, Np, Hl, D]`` uint16; planes 0, 1, 2 are Q, K, V
@@ -203,7 +204,9 @@ def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
     are padding and give zero.
 
     Returns fp64 ``[P, R, Hl, D]`` for the selected rows (all ``Np`` rows when
-    ``rows`` is None).
+    ``rows`` is None).  Query rows are independent, so they are evaluated
+    ``row_block`` at a time to bound memory, and ``workers`` threads may take
+    different (rank, head) slabs; neither changes any arithmetic.
     """
     P, C, Np, Hl, D = T.shape
     if C < 3:
@@ -214,16 +217,28 @@ def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
     seg_of = np.full(rows.size, -1, dtype=np.int64)
     for s, (a, b) in enumerate(segs):
         seg_of[(rows >= a) & (rows < b)] = s
-    for r in range(P):
-        for j in range(Hl):
-            for s, (a, b) in enumerate(segs):
-                sel = np.nonzero(seg_of == s)[0]
-                if sel.size == 0:
-                    continue
-                q = bf16_bits_to_f64(T[r, 0, rows[sel], j, :])
-                k = bf16_bits_to_f64(T[r, 1, a:b, j, :])
-                v = bf16_bits_to_f64(T[r, 2, a:b, j, :])
-                out[r, sel, j, :] = attention_rows(q, k, v, scale)
+
+    def one_slab(rj):
+        r, j = rj
+        for s, (a, b) in enumerate(segs):
+            sel = np.nonzero(seg_of == s)[0]
+            if sel.size == 0:
+                continue
+            k = bf16_bits_to_f64(T[r, 1, a:b, j, :])
+            v = bf16_bits_to_f64(T[r, 2, a:b, j, :])
+            for i0 in range(0, sel.size, row_block):
+                part = sel[i0:i0 + row_block]
+                q = bf16_bits_to_f64(T[r, 0, rows[part], j, :])
+                out[r, part, j, :] = attention_rows(q, k, v, scale)
+
+    slabs = [(r, j) for r in range(P) for j in range(Hl)]
+    if workers > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            list(ex.map(one_slab, slabs))
+    else:
+        for rj in slabs:
+            one_slab(rj)
     return out
 
 
@@ -238,14 +253,14 @@ def output_repack_bwd(O_heads: np.ndarray) -> np.ndarray:
 
 
 def layer_fwd(S: np.ndarray, P: int, N: int, scale: float, cu_seqlens=None,
-              rows: np.ndarray | None = None) -> np.ndarray:
+              rows: np.ndarray | None = None, workers: int = 1) -> np.ndarray:
     """The whole layer: repack -> attention per slab -> inverse repack.
 
     S: sequence-sharded ``[Np, C, H, D]`` uint16.  Returns fp64 ``[R, H, D]``
     (sequence-sharded output rows, all ``Np`` rows when ``rows`` is None).
     """
     T = repack_fwd(S, P)
-    O = attention_heads(T, N, scale, cu_seqlens=cu_seqlens, rows=rows)
+    O = attention_heads(T, N, scale, cu_seqlens=cu_seqlens, rows=rows, workers=workers)
     return output_repack_bwd(O)
 
 

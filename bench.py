@@ -1,0 +1,408 @@
+"""Benchmark of the one-GPU Ulysses attention layer (repack -> attention -> inverse repack).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config dit19k] [--impl ours|reference]
+
+One step = one pass of the whole layer over the workload's synthetic input:
+ulysses_repack_fwd (all planes) -> ulysses_attn_fwd -> ulysses_repack_bwd
+(output plane), each a C-ABI call on one stream with CUDA events between
+them.  Rank 0 prints one JSON line.  N > 1 runs N independent replicas (the
+layer has no exchange between GPUs in this build), launched with torchrun.
+
+``--impl reference`` times the CPU oracle instead, on a bounded sample of
+the same workload per step, extrapolated to the full layer.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+# name: (P, N, H, planes, seed, cu_seqlens)
+WORKLOADS = {
+    "tiny": (2, 1024, 8, 3, 0, None),
+    "dit19k": (4, 19_394, 56, 3, 1, None),
+    "clip38k": (4, 38_912, 56, 4, 2, None),
+    "long104k": (8, 104_448, 56, 3, 3, None),
+    "long104k-varlen": (8, 104_448, 56, 3, 3, [0, 52_224, 83_456, 104_448]),
+    "prof8k": (4, 8192, 56, 3, 1, None),   # small case for profiler captures (352 MB input > L2)
+}
+WORKLOAD_TEXT = {
+    "tiny": "Tiny Ulysses layer P=2 N=1024 H=8 D=128 packed QKV bf16",
+    "dit19k": "Video-DiT geometry P=4 N=19394 H=56 D=128 packed QKV bf16 [N,3,H,D]",
+    "clip38k": "Longer clip P=4 N=38912 H=56 D=128 packed QKVG bf16 [N,4,H,D]",
+    "long104k": "Long clip P=8 N=104448 H=56 D=128 packed QKV bf16",
+    "long104k-varlen": "Long clip varlen P=8 N=104448 H=56 D=128, 3 sequences 52224/31232/20992",
+    "prof8k": "Profiling case P=4 N=8192 H=56 D=128 packed QKV bf16",
+}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_flops(N, H, cu):
+    segs = [(0, N)] if cu is None else list(zip(cu, cu[1:]))
+    return float(sum(4 * (b - a) ** 2 * H * 128 for a, b in segs))
+
+
+def source_hash(name):
+    p = os.path.join(ROOT, "ulysses_sequence_attention_repack_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    rec = d.get(kernel, {}).get(workload)
+    if not rec or rec.get("source_sha256_16") != source_hash(rec["source"]):
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu_index = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [[x.strip() for x in line.split(",")] for line in out.strip().splitlines() if line.strip()]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 7:
+                continue
+            try:
+                sm.append(float(r[0]))
+                mx = float(r[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, r[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    P, N, H, C, seed, cu = WORKLOADS[args.config]
+    Hl = H // P
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu)
+    Np = plan.padded_tokens
+    S = inputs.qkv_seq(N, H, P, C, seed, dev)
+    T = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    scale = 1.0 / math.sqrt(128)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        U.ulysses_repack_fwd(plan, S, T, stream)
+        if evs:
+            evs[1].record(stream)
+        U.ulysses_attn_fwd(plan, T, OT, scale, stream)
+        if evs:
+            evs[2].record(stream)
+        U.ulysses_repack_bwd(plan, OT, OS, 1, stream)
+        if evs:
+            evs[3].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(stop)
+    t_rf = [e[0].elapsed_time(e[1]) for e in evs]
+    t_at = [e[1].elapsed_time(e[2]) for e in evs]
+    t_rb = [e[2].elapsed_time(e[3]) for e in evs]
+    if U.ulysses_last_device_error(plan) != 0:
+        raise RuntimeError("a kernel reported a device error during the timed region")
+
+    # fused variant (attention reads the sequence-sharded input directly)
+    for _ in range(3):
+        U.ulysses_layer_fwd(plan, S, OS, None, fused=1, stream=stream)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nf = max(3, args.steps // 2)
+    f0.record(stream)
+    for _ in range(nf):
+        U.ulysses_layer_fwd(plan, S, OS, None, fused=1, stream=stream)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fused_ms = f0.elapsed_time(f1) / nf
+
+    # end to end through the C ABI from pinned host buffers
+    host_in = S.cpu().pin_memory()
+    host_out = torch.empty(OS.shape, dtype=OS.dtype).pin_memory()
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev)
+    dev_in = torch.empty_like(S)
+    for _ in range(2):
+        U.ulysses_layer_fwd_host(plan, host_in, host_out, dev_in, OS, ws, fused=0, stream=stream)
+    torch.cuda.synchronize()
+    ne = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(ne):
+        U.ulysses_layer_fwd_host(plan, host_in, host_out, dev_in, OS, ws, fused=0, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / ne
+    h2d = host_in.numel() * host_in.element_size()
+    d2h = host_out.numel() * host_out.element_size()
+
+    vals = torch.tensor([total_ms, e2e_ms, fused_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, fused_ms = vals.tolist()
+    if rank != 0:
+        return None
+
+    pk, pk_kind = peaks()
+    flops = attn_flops(N, H, cu)
+    at_ms = statistics.mean(t_at)
+    rf_ms, rb_ms = statistics.mean(t_rf), statistics.mean(t_rb)
+    rf_bytes = 2 * C * Np * H * 128 * 2
+    rb_bytes = 2 * Np * H * 128 * 2
+    attn_tflops = flops / (at_ms * 1e-3) / 1e12
+    rf_gbs = rf_bytes / (rf_ms * 1e-3) / 1e9
+    rb_gbs = rb_bytes / (rb_ms * 1e-3) / 1e9
+    ms_per_step = total_ms / args.steps
+    launches_per_step = math.ceil(C / plan.plane_chunk) + 1 + 1
+    traffic = recorded_traffic("attn_fwd_kernel", args.config)
+    line = {
+        "metric": "Ulysses layer µs; attn TFLOP/s and repack GB/s vs B200 peak",
+        "value": round(ms_per_step * 1000.0, 2),
+        "unit": "us per layer",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic N(0,1) bf16, seeded",
+        "config": {"workload": WORKLOAD_TEXT[args.config], "name": args.config, "P": P, "N": N, "Np": Np,
+                   "H": H, "D": 128, "planes": C, "seed": seed, "cu_seqlens": cu,
+                   "step": "repack_fwd + attn_fwd + repack_bwd(output), one C-ABI call each",
+                   "replicas": world, "l2": f"inputs larger than L2 ({S.numel() * 2 / 1e6:.0f} MB per step)"},
+        "attn_us": round(at_ms * 1000, 2),
+        "attn_tflops": round(attn_tflops, 1),
+        "repack_fwd_us": round(rf_ms * 1000, 2),
+        "repack_fwd_gbs": round(rf_gbs, 1),
+        "repack_bwd_us": round(rb_ms * 1000, 2),
+        "repack_bwd_gbs": round(rb_gbs, 1),
+        "repack_fwd_frac": {"measured": round(rf_gbs / pk["hbm_gbs"], 3),
+                            "spec_8TBs": round(rf_gbs / SPEC_PEAKS["hbm_gbs"], 3)},
+        "attn_frac": {"measured_burst": round(attn_tflops / pk["bf16_tflops"], 3),
+                      "measured_sustained": round(attn_tflops / pk.get("bf16_tflops_sustained",
+                                                                       pk["bf16_tflops"]), 3),
+                      "spec_2250": round(attn_tflops / SPEC_PEAKS["bf16_tflops"], 3)},
+        "fused_layer_us": round(fused_ms * 1000, 2),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": round(attn_tflops, 1),
+                     "peak": pk["bf16_tflops"], "peak_kind": f"{pk_kind} bf16 burst", "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / pk["bf16_tflops"], 3), "traffic": traffic,
+                     "algorithmic_flops_per_launch": flops},
+        "e2e": {"value": round(e2e_ms * 1000, 2), "unit": "us per layer", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "path": "ulysses_layer_fwd_host (pinned host in/out)"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.config, S)
+    return line
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(config, S_bits, rows_per_head=1024, heads=4, token_frac=16):
+    """Time the oracle on a bounded sample and extrapolate to one full layer (µs)."""
+    import numpy as np
+    from oracle import ulysses_oracle as orc
+    P, N, H, C, seed, cu = WORKLOADS[config]
+    Np = S_bits.shape[0]
+    Hl = H // P
+    # repack: a token slice (multiple of P rows), scaled by the slice fraction
+    ns = max(P, (Np // token_frac) // P * P)
+    t0 = time.perf_counter()
+    Tsub = orc.repack_fwd(np.ascontiguousarray(S_bits[:ns]), P)
+    t_rf = (time.perf_counter() - t0) * (Np / ns)
+    t0 = time.perf_counter()
+    orc.repack_bwd(Tsub[:, :1])
+    t_rb = (time.perf_counter() - t0) * (Np / ns)
+    # attention: `heads` heads of rank 0, `rows_per_head` sampled rows, all keys
+    T = np.empty((1, 3, Np, heads, 128), dtype=np.uint16)
+    for c in range(3):
+        T[0, c] = S_bits[:, c, :heads, :]
+    rows = orc.sample_rows(N, rows_per_head, seed, cu)
+    t0 = time.perf_counter()
+    orc.attention_heads(T, N, 1.0 / math.sqrt(128), cu_seqlens=cu, rows=rows)
+    t_at = (time.perf_counter() - t0) * (N / rows.size) * (H / heads)
+    total_us = (t_rf + t_at + t_rb) * 1e6
+    sample = (f"repack of {ns}/{Np} tokens (x{Np / ns:.1f}); attention of {rows.size} query rows x {heads} heads "
+              f"over all keys (x{(N / rows.size) * (H / heads):.1f}); extrapolated linearly to one layer")
+    return total_us, sample
+
+
+def cpu_baseline(config, S):
+    from ulysses_sequence_attention_repack_b200 import inputs
+    S_bits = inputs.host_bits(S)
+    us, sample = oracle_sample(config, S_bits)
+    return {"value": round(us, 1), "unit": "us per layer", "cores": _cores(), "kind": "oracle",
+            "sample": sample}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, rank 0 only, on a bounded sample per step."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import torch
+    P, N, H, C, seed, cu = WORKLOADS[args.config]
+    sys.path.insert(0, ROOT)
+    from ulysses_sequence_attention_repack_b200 import inputs
+    S = inputs.qkv_seq(N, H, P, C, seed, "cpu")
+    S_bits = inputs.host_bits(S)
+    del S
+    for _ in range(args.warmup):
+        oracle_sample(args.config, S_bits, rows_per_head=128, heads=2, token_frac=64)
+    vals, sample = [], ""
+    t_start = time.perf_counter()
+    for _ in range(args.steps):
+        v, sample = oracle_sample(args.config, S_bits, rows_per_head=128, heads=2, token_frac=64)
+        vals.append(v)
+    wall = time.perf_counter() - t_start
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference",
+        "metric": "Ulysses layer µs; attn TFLOP/s and repack GB/s vs B200 peak",
+        "value": round(value, 1), "unit": "us per layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(value / 1000, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic N(0,1) bf16, seeded",
+        "config": {"workload": WORKLOAD_TEXT[args.config], "name": args.config},
+        "cpu_baseline": {"value": round(value, 1), "unit": "us per layer", "cores": _cores(), "kind": "oracle",
+                         "sample": sample, "wall_s": round(wall, 1)},
+        "e2e": {"value": round(value, 1), "unit": "us per layer", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "numpy": np.__version__, "torch": torch.__version__,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="dit19k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

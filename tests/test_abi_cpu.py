@@ -1,0 +1,119 @@
+"""Host-side tests of the C ABI (no GPU needed: nothing here launches a kernel)."""
+import os
+import re
+
+import pytest
+
+import ulysses_sequence_attention_repack_b200 as U
+from oracle import ulysses_oracle as orc
+from ulysses_sequence_attention_repack_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "ulysses.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ulysses_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = U.load()
+    syms = declared_symbols()
+    assert len(syms) >= 13
+    for name in syms:
+        assert hasattr(lib, name), name
+    assert set(syms) == set(U.EXPORTS)
+
+
+def test_library_built_for_sm100a():
+    # the build passes exactly one gencode target: sm_100a
+    from ulysses_sequence_attention_repack_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert os.path.exists(U.library_path())
+
+
+def _code(**kw):
+    args = dict(N=1024, H=8, D=128, P=2, planes=3, token_stride=0, plane_stride=0, plane_chunk=0, cu_seqlens=None)
+    args.update(kw)
+    try:
+        U.ulysses_plan(**args)
+        return 0
+    except U.UlyssesError as e:
+        return e.code
+
+
+def test_plan_validation_codes():
+    assert _code() == _lib.ULYSSES_OK
+    assert _code(D=64) == _lib.ULYSSES_ERR_UNSUPPORTED
+    assert _code(H=6, P=4) == _lib.ULYSSES_ERR_DIVISIBILITY
+    assert _code(P=16) == _lib.ULYSSES_ERR_DIVISIBILITY          # more ranks than heads
+    assert _code(P=0) == _lib.ULYSSES_ERR_ARG
+    assert _code(N=0) == _lib.ULYSSES_ERR_ARG
+    assert _code(planes=0) == _lib.ULYSSES_ERR_ARG
+    assert _code(planes=9) == _lib.ULYSSES_ERR_ARG
+    assert _code(token_stride=3 * 8 * 128 + 4, plane_stride=8 * 128) == _lib.ULYSSES_ERR_ALIGN
+    assert _code(token_stride=8 * 128, plane_stride=8 * 128) == _lib.ULYSSES_ERR_ARG   # planes overlap
+    # one plane per rank above 1 GiB: 400,000 tokens x 56 heads at SP 4
+    assert _code(N=400_000, H=56, P=4) == _lib.ULYSSES_ERR_WINDOW
+    # a chunk of two 896,000,000-byte planes exceeds the window
+    assert _code(N=250_000, H=56, P=4, planes=4, plane_chunk=2) == _lib.ULYSSES_ERR_WINDOW
+    assert _code(plane_chunk=4) == _lib.ULYSSES_ERR_ARG
+    # cu_seqlens: must start at 0, end at N, never decrease
+    assert _code(N=10, P=2, H=2, cu_seqlens=[0, 5, 10]) == _lib.ULYSSES_OK
+    assert _code(N=10, P=2, H=2, cu_seqlens=[1, 5, 10]) == _lib.ULYSSES_ERR_ARG
+    assert _code(N=10, P=2, H=2, cu_seqlens=[0, 5, 9]) == _lib.ULYSSES_ERR_ARG
+    assert _code(N=10, P=2, H=2, cu_seqlens=[0, 6, 5, 10]) == _lib.ULYSSES_ERR_ARG
+    assert _code(N=65, P=1, H=1, cu_seqlens=list(range(66))) == _lib.ULYSSES_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("N,H,P,C", [(19_394, 56, 4, 3), (38_912, 56, 4, 4), (104_448, 56, 8, 3),
+                                     (250_000, 56, 4, 4), (32_000, 56, 4, 4), (1024, 8, 2, 3), (5, 4, 4, 3)])
+def test_plan_sizes_agree_with_oracle(N, H, P, C):
+    plan = U.ulysses_plan(N, H, 128, P, C)
+    assert plan.padded_tokens == orc.padded_tokens(N, P)
+    assert plan.window_bytes_per_plane == orc.plane_bytes_per_rank(N, H, 128, P)
+    assert plan.plane_chunk == orc.auto_plane_chunk(N, H, 128, P, C)
+    Np, Hl = orc.padded_tokens(N, P), H // P
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    assert plan.workspace_bytes == up(P * C * Np * Hl * 128 * 2) + up(P * Np * Hl * 128 * 2)
+
+
+def test_window_bytes_printed_on_the_pages():
+    # 250,000 tokens, 56 heads, head dim 128, SP 4: 896,000,000 bytes per plane, one plane per launch
+    plan = U.ulysses_plan(250_000, 56, 128, 4, 4)
+    assert plan.window_bytes_per_plane == 896_000_000
+    assert plan.plane_chunk == 1
+
+
+def test_launch_argument_checks_before_any_device_work():
+    plan = U.ulysses_plan(1024, 8, 128, 2, 3)
+    lib = U.load()
+    h = plan.handle
+    # null pointers
+    assert lib.ulysses_repack_fwd(h, None, 0x10000, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_attn_fwd(h, 0x10000, None, 0.1, None) == _lib.ULYSSES_ERR_ARG
+    # misaligned pointers
+    assert lib.ulysses_repack_fwd(h, 0x10008, 0x90000000, None) == _lib.ULYSSES_ERR_ALIGN
+    assert lib.ulysses_repack_bwd(h, 0x10000, 0x90000004, 1, None) == _lib.ULYSSES_ERR_ALIGN
+    # overlapping input and output
+    assert lib.ulysses_repack_fwd(h, 0x10000, 0x10000 + 4096, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_attn_fwd(h, 0x10000, 0x10000, 0.1, None) == _lib.ULYSSES_ERR_ARG
+    # bad scale and plane count
+    assert lib.ulysses_attn_fwd(h, 0x10000, 0x90000000, -1.0, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_repack_bwd(h, 0x10000, 0x90000000, 4, None) == _lib.ULYSSES_ERR_ARG
+    # layer: missing or short workspace, bad fused flag
+    assert lib.ulysses_layer_fwd(h, 0x10000, 0x90000000, None, 0, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
+    assert lib.ulysses_layer_fwd(h, 0x10000, 0x90000000, 0xA0000000, 16, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
+    assert lib.ulysses_layer_fwd(h, 0x10000, 0x90000000, None, 0, 2, None) == _lib.ULYSSES_ERR_ARG
+    # a gate-less plan cannot run attention
+    p2 = U.ulysses_plan(1024, 8, 128, 2, 2)
+    assert lib.ulysses_attn_fwd(p2.handle, 0x10000, 0x90000000, 0.1, None) == _lib.ULYSSES_ERR_ARG
+
+
+def test_strerror_covers_every_code():
+    for code in range(9):
+        assert U.strerror(code) != "unknown error code"
+    assert U.strerror(99) == "unknown error code"

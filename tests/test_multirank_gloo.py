@@ -1,0 +1,62 @@
+"""The repack index map against a real all-to-all between processes (gloo, CPU).
+
+On P real GPUs each virtual rank is a process and step one of the layer is
+one all-to-all that scatters heads and gathers the sequence (mode 0 of the
+FastVideo Ulysses transport).  Here P CPU processes run that exchange with
+torch.distributed.all_to_all_single; each rank's received slab must equal the
+oracle's head-sharded slab for that rank bit for bit, and the inverse
+exchange must restore the input.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from oracle import ulysses_oracle as orc
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, S_bits, result_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        Np, C, H, D = S_bits.shape
+        Nl, Hl = Np // world, H // world
+        # this rank's sequence shard; bit patterns widened to int32 (gloo has no 16-bit integers)
+        x = torch.from_numpy(S_bits[rank * Nl:(rank + 1) * Nl].astype(np.int32))         # [Nl, C, H, D]
+        # head block r goes to rank r: [P, C, Nl, Hl, D], split along dim 0
+        send = x.reshape(Nl, C, world, Hl, D).permute(2, 1, 0, 3, 4).contiguous()
+        recv = torch.empty_like(send)                                                   # [P(src), C, Nl, Hl, D]
+        dist.all_to_all_single(recv, send)
+        heads = recv.permute(1, 0, 2, 3, 4).reshape(C, world * Nl, Hl, D).contiguous()  # [C, Np, Hl, D]
+        # inverse exchange (mode 1) restores the shard
+        send_b = heads.reshape(C, world, Nl, Hl, D).permute(1, 0, 2, 3, 4).contiguous()
+        recv_b = torch.empty_like(send_b)
+        dist.all_to_all_single(recv_b, send_b)
+        back = recv_b.permute(2, 1, 0, 3, 4).reshape(Nl, C, H, D)
+        np.save(os.path.join(result_dir, f"heads{rank}.npy"), heads.numpy().astype(np.uint16))
+        np.save(os.path.join(result_dir, f"back{rank}.npy"), back.numpy().astype(np.uint16))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,Nl,C,H", [(2, 5, 3, 4), (4, 3, 4, 8)])
+def test_all_to_all_processes_match_oracle_repack(tmp_path, world, Nl, C, H):
+    rng = np.random.default_rng(world)
+    S = rng.integers(0, 1 << 16, size=(world * Nl, C, H, 4), dtype=np.uint16)
+    mp.start_processes(_worker, args=(world, _free_port(), S, str(tmp_path)), nprocs=world, start_method="spawn")
+    T = orc.repack_fwd(S, world)
+    for r in range(world):
+        assert np.array_equal(np.load(tmp_path / f"heads{r}.npy"), T[r])
+        Nl_ = S.shape[0] // world
+        assert np.array_equal(np.load(tmp_path / f"back{r}.npy"), S[r * Nl_:(r + 1) * Nl_])

@@ -40,9 +40,19 @@
 namespace ulysses {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;      // 3 warpgroups
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
+// Register split: the kernel is launched with kLaunchRegs per thread
+// (384 x 168 = 64512); warpgroup 2 (TMA, MMA, two spare warps) drops to
+// kProducerRegs and the two softmax warpgroups rise to kSoftmaxRegs:
+// 128 x 72 + 256 x 216 = 64512.  The host refuses to launch if the compiled
+// register count differs, so the increase can never wait for registers that
+// were not released.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kProducerRegs = 72;
+constexpr uint32_t kSoftmaxRegs = 216;
+static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int BM = 128;            // query rows per tile
 constexpr int BN = 128;            // keys per tile
 constexpr int HD = 128;            // head dim
@@ -165,8 +175,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == kTmaWarp) {
+  if (warp >= 8) {
+   regs_dec<kProducerRegs>();
+   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t kc = 0, vc = 0, uc = 0;
@@ -220,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t n = (vc > kStages ? vc - kStages : 0); n < vc; ++n)
         drain_wait(BAR(B_VFULL0 + n % kStages), (n / kStages) & 1);
     }
-  } else if (warp == kMmaWarp) {
+   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ tcgen05 issuer
     if (lane == 0) {
       uint32_t kc = 0, vc = 0, uc = 0, pc = 0;
@@ -294,7 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(BAR(B_DONE));
       drain_wait(BAR(B_DONE), 0);
     }
+   }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------ softmax warpgroups
     const int wg = warp >> 2;                  // Q tile 0 or 1
     const int row = threadIdx.x & 127;         // query row inside the tile == TMEM lane
@@ -328,9 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (c >= valid) s[c] = -INFINITY;
         }
-        float mx = s[0];
+        // row max: eight independent 3-input max chains, then a short tree
+        float mxa[8];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int k = 0; k < 8; ++k) mxa[k] = fmax3(s[16 * k], s[16 * k + 1], s[16 * k + 2]);
+#pragma unroll
+        for (int i = 3; i < 15; i += 2)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mxa[k] = fmax3(mxa[k], s[16 * k + i], s[16 * k + i + 1]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mxa[k] = fmaxf(mxa[k], s[16 * k + 15]);
+        const float mx = fmax3(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]));
         const float m_new = fmaxf(m_used, mx * sl2);
         // Move the running max only when it grew by more than 8 (log2 units):
         // probabilities stay below 2^8 and O is rescaled rarely.
@@ -344,18 +365,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= f;
           m_used = m_new;
         }
-        const float neg_m = -m_used;
+        const f2 scale2{sl2, sl2}, negm2{-m_used, -m_used};
+        f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2_approx(fmaf(s[64 * half + 2 * c], sl2, neg_m));
-            const float p1 = ex2_approx(fmaf(s[64 * half + 2 * c + 1], sl2, neg_m));
-            l += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
+            const f2 x = ffma2(f2{s[64 * half + 2 * c], s[64 * half + 2 * c + 1]}, scale2, negm2);
+            const f2 e{ex2_approx(x.x), ex2_approx(x.y)};
+            acc[c & 3] = fadd2(acc[c & 3], e);
+            pk[c] = pack_bf16x2(e.x, e.y);
           }
           tmem_st32(tS + 32 * half, pk);   // P (bf16 pairs) over the first 64 columns of S
+        }
+        {
+          const f2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+          const f2 a = fadd2(a01, a23);
+          l += a.x + a.y;
         }
         if (__any_sync(0xffffffffu, need)) {
           // O holds the sum of earlier tiles (complete: S of this tile was
@@ -512,7 +539,11 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static bool attr_set[64] = {false};
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != static_cast<int>(kLaunchRegs)) return cudaErrorInvalidConfiguration;   // see register split
+    e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }

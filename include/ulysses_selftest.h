@@ -1,0 +1,30 @@
+/*
+ * ulysses_selftest.h -- test hooks of libulysses.so (not part of the layer).
+ *
+ * These entry points run single device helpers of the kernels on their own,
+ * so tests can compare them with reference values.
+ */
+#ifndef ULYSSES_SELFTEST_H_
+#define ULYSSES_SELFTEST_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * y[i] = 2^x[i] computed with the FMA-pipe exponential the attention softmax
+ * uses for part of its probabilities (round-to-nearest range reduction plus a
+ * degree-3 minimax polynomial; maximum relative error 7.5e-5 for
+ * -125 <= x <= 64; inputs below -125 return 2^-125).  x and y are device
+ * arrays of n floats, 4-byte aligned; asynchronous on `stream`.
+ * Returns 0, 1 for a bad argument, 6 for a CUDA launch error.
+ */
+int ulysses_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ULYSSES_SELFTEST_H_ */

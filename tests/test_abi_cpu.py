@@ -12,7 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_symbols():
-    text = open(os.path.join(ROOT, "include", "ulysses.h")).read()
+    import glob
+    text = "".join(open(h).read() for h in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(ulysses_\w+)\s*\(", text)))
 
@@ -20,7 +21,7 @@ def declared_symbols():
 def test_library_exports_every_declared_symbol():
     lib = U.load()
     syms = declared_symbols()
-    assert len(syms) >= 13
+    assert len(syms) >= 14
     for name in syms:
         assert hasattr(lib, name), name
     assert set(syms) == set(U.EXPORTS)

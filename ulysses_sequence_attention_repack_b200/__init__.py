@@ -20,4 +20,5 @@ from ._lib import (  # noqa: F401
     ulysses_plan,
     ulysses_repack_bwd,
     ulysses_repack_fwd,
+    ulysses_selftest_exp2_poly,
 )

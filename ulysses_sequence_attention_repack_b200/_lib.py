@@ -31,7 +31,7 @@ EXPORTS = (
     "ulysses_plan", "ulysses_plan_destroy", "ulysses_plan_padded_tokens", "ulysses_plan_plane_chunk",
     "ulysses_plan_window_bytes_per_plane", "ulysses_workspace_bytes", "ulysses_repack_fwd",
     "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
-    "ulysses_last_device_error", "ulysses_strerror",
+    "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
 )
 
 
@@ -87,6 +87,8 @@ def load() -> ctypes.CDLL:
         lib.ulysses_last_device_error.restype = ctypes.c_int
         lib.ulysses_strerror.argtypes = [ctypes.c_int]
         lib.ulysses_strerror.restype = ctypes.c_char_p
+        lib.ulysses_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
+        lib.ulysses_selftest_exp2_poly.restype = ctypes.c_int
         _handle = lib
         return lib
 
@@ -210,3 +212,9 @@ def ulysses_layer_fwd_host(plan: Plan, host_qkv_seq, host_out_seq, dev_qkv_seq, 
 
 def ulysses_last_device_error(plan: Plan, stream=None) -> int:
     return load().ulysses_last_device_error(plan.handle, _stream(stream))
+
+
+def ulysses_selftest_exp2_poly(x, y, stream=None) -> None:
+    """y = 2^x with the attention kernel's FMA-pipe exponential (float32 device tensors)."""
+    _check(load().ulysses_selftest_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)),
+           "ulysses_selftest_exp2_poly")

@@ -34,8 +34,15 @@
 #include <cstdint>
 #include <cstring>
 
+#include "exp2_poly.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
+
+// One pair in ULY_EMU_EVERY of each row's exponentials is computed on the FMA
+// pipe (exp2_poly2) instead of the MUFU unit.
+#ifndef ULY_EMU_EVERY
+#define ULY_EMU_EVERY 4
+#endif
 
 namespace ulysses {
 namespace {
@@ -74,6 +81,7 @@ enum {
   B_VFULL0, B_VFULL1, B_VEMPTY0, B_VEMPTY1,
   B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1,
   B_OFULL0, B_OFULL1, B_OEMPTY0, B_OEMPTY1,
+  B_PHALF0, B_PHALF1,
   B_DONE, B_COUNT
 };
 constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;           // TMEM base address
@@ -123,6 +131,29 @@ __device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& w)
   return local >= 0 && w.r < p.P;
 }
 
+// P = exp2(s * scale_log2 - m) for columns [64 half, 64 half + 64) of one row,
+// stored to TMEM as 32 bf16 pairs at P columns [32 half, 32 half + 32); the
+// row sum accumulates in acc.
+template <bool kEmu>
+__device__ __forceinline__ void exp_store_half(const float* s, int half, f2 scale2, f2 negm2, f2 (&acc)[4],
+                                               uint32_t tS) {
+  uint32_t pk[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const f2 x = ffma2(f2{s[64 * half + 2 * c], s[64 * half + 2 * c + 1]}, scale2, negm2);
+    f2 e;
+    if (kEmu && (c % ULY_EMU_EVERY) == ULY_EMU_EVERY - 1) {
+      e = exp2_poly2(x);
+    } else {
+      e.x = ex2_approx(x.x);
+      e.y = ex2_approx(x.y);
+    }
+    acc[c & 3] = fadd2(acc[c & 3], e);
+    pk[c] = pack_bf16x2(e.x, e.y);
+  }
+  tmem_st32(tS + 32 * half, pk);
+}
+
 // waits that ignore the abort flag (used for draining in-flight work)
 __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
@@ -162,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR(B_PFULL0 + i), BM);
       mbar_init(BAR(B_OFULL0 + i), 1);
       mbar_init(BAR(B_OEMPTY0 + i), BM);
+      mbar_init(BAR(B_PHALF0 + i), BM);
     }
     mbar_init(BAR(B_DONE), 1);
     fence_mbar_init();
@@ -236,23 +268,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kc = 0, vc = 0, uc = 0, pc = 0;
       bool ok = true;
+      // descriptors computed once; each group of 8 MMAs is one asm block
+      const uint64_t dQ0 = desc_sw128(sbase + kOffQ, 16, 1024);
+      const uint64_t dQ1 = desc_sw128(sbase + kOffQ + 2 * kHalfBytes, 16, 1024);
+      const uint64_t dK0 = desc_sw128(sbase + kOffK, 16, 1024);
+      const uint64_t dK1 = desc_sw128(sbase + kOffK + kTileBytes, 16, 1024);
+      const uint64_t dV0 = desc_sw128(sbase + kOffV, kHalfBytes, 1024);
+      const uint64_t dV1 = desc_sw128(sbase + kOffV + kTileBytes, kHalfBytes, 1024);
       auto issue_s = [&](int i, uint32_t ks) {
-        const uint32_t qa = sbase + kOffQ + 2 * i * kHalfBytes;
-        const uint32_t ka = sbase + kOffK + ks * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(tmem + kColS0 + 128 * i, desc_sw128(qa + off, 16, 1024), desc_sw128(ka + off, 16, 1024),
-                 kIdescS, kk > 0);
-        }
+        mma_ss_k128(tmem + kColS0 + 128 * i, i ? dQ1 : dQ0, ks ? dK1 : dK0, kIdescS, 0);
       };
-      auto issue_pv = [&](int i, uint32_t vs, uint32_t acc) {
-        const uint32_t va = sbase + kOffV + vs * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 8 * kk,
-                 desc_sw128(va + kk * 2048, kHalfBytes, 1024), kIdescPV, (acc | kk) != 0);
-        }
+      // O_i (+)= P_i V over keys [64 h, 64 h + 64): P columns [32 h, 32 h + 32),
+      // V rows 64 h.. (8 KB further in each 64-column atom: +512 descriptor units)
+      auto issue_pv_half = [&](int i, uint32_t vs, int h, uint32_t acc) {
+        mma_ts_k64(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 32 * h, (vs ? dV1 : dV0) + 512 * h, kIdescPV,
+                   acc);
       };
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
         Unit w;
@@ -276,9 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(BAR(B_VFULL0 + vs), (vc / kStages) & 1, g))) break;
           for (int i = 0; i < 2; ++i) {
             if (t == 0 && uc > 0 && !(ok = mbar_wait(BAR(B_OEMPTY0 + i), (uc - 1) & 1, g))) break;
+            if (!(ok = mbar_wait(BAR(B_PHALF0 + i), pc & 1, g))) break;
+            tc_fence_after();
+            issue_pv_half(i, vs, 0, t > 0);
             if (!(ok = mbar_wait(BAR(B_PFULL0 + i), pc & 1, g))) break;
             tc_fence_after();
-            issue_pv(i, vs, t > 0);
+            issue_pv_half(i, vs, 1, 1);
             if (t == nkv - 1) {
               mma_commit(BAR(B_OFULL0 + i));
             } else if (i == 0) {
@@ -365,25 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           l *= f;
           m_used = m_new;
         }
-        const f2 scale2{sl2, sl2}, negm2{-m_used, -m_used};
-        f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const f2 x = ffma2(f2{s[64 * half + 2 * c], s[64 * half + 2 * c + 1]}, scale2, negm2);
-            const f2 e{ex2_approx(x.x), ex2_approx(x.y)};
-            acc[c & 3] = fadd2(acc[c & 3], e);
-            pk[c] = pack_bf16x2(e.x, e.y);
-          }
-          tmem_st32(tS + 32 * half, pk);   // P (bf16 pairs) over the first 64 columns of S
-        }
-        {
-          const f2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
-          const f2 a = fadd2(a01, a23);
-          l += a.x + a.y;
-        }
         if (__any_sync(0xffffffffu, need)) {
           // O holds the sum of earlier tiles (complete: S of this tile was
           // issued after them); scale it to the new max before the next P V.
@@ -397,6 +411,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
             tmem_st32(tO + 32 * c, o);
           }
+        }
+        const f2 scale2{sl2, sl2}, negm2{-m_used, -m_used};
+        f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        // P (bf16 pairs) over the first 64 columns of S, in two halves; the
+        // first half is handed to the MMA warp before the second is computed.
+        // The masked last tile uses MUFU ex2 only, so masked keys give exact zeros.
+        const bool emu = t != nkv - 1;
+        if (emu)
+          exp_store_half<true>(s, 0, scale2, negm2, acc, tS);
+        else
+          exp_store_half<false>(s, 0, scale2, negm2, acc, tS);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(B_PHALF0 + wg));
+        if (emu)
+          exp_store_half<true>(s, 1, scale2, negm2, acc, tS);
+        else
+          exp_store_half<false>(s, 1, scale2, negm2, acc, tS);
+        {
+          const f2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+          const f2 a = fadd2(a01, a23);
+          l += a.x + a.y;
         }
         tmem_wait_st();
         tc_fence_before();

@@ -38,10 +38,12 @@
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
-// One pair in ULY_EMU_EVERY of each row's exponentials is computed on the FMA
-// pipe (exp2_poly2) instead of the MUFU unit.
+// With ULY_EMU_EVERY = k > 0, one pair in k of each row's exponentials is
+// computed on the FMA pipe (exp2_poly2) instead of the MUFU unit.  Off by
+// default: on B200 the MUFU unit is not what limits this loop, and the extra
+// FMA-pipe instructions made it slower (k = 8, 4, 2 all measured slower).
 #ifndef ULY_EMU_EVERY
-#define ULY_EMU_EVERY 4
+#define ULY_EMU_EVERY 0
 #endif
 
 namespace ulysses {
@@ -142,7 +144,7 @@ __device__ __forceinline__ void exp_store_half(const float* s, int half, f2 scal
   for (int c = 0; c < 32; ++c) {
     const f2 x = ffma2(f2{s[64 * half + 2 * c], s[64 * half + 2 * c + 1]}, scale2, negm2);
     f2 e;
-    if (kEmu && (c % ULY_EMU_EVERY) == ULY_EMU_EVERY - 1) {
+    if (kEmu && ULY_EMU_EVERY > 0 && (c % (ULY_EMU_EVERY > 0 ? ULY_EMU_EVERY : 1)) == ULY_EMU_EVERY - 1) {
       e = exp2_poly2(x);
     } else {
       e.x = ex2_approx(x.x);

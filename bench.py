@@ -35,7 +35,9 @@ WORKLOADS = {
     "long104k": (8, 104_448, 56, 3, 3, None),
     "long104k-varlen": (8, 104_448, 56, 3, 3, [0, 52_224, 83_456, 104_448]),
     "prof8k": (4, 8192, 56, 3, 1, None),   # small case for profiler captures (352 MB input > L2)
+    "stress250k": (4, 250_000, 56, 4, 4, None),   # repack fwd + bwd only, plus an N sweep
 }
+SWEEP_N = (4096, 8192, 16384, 32768, 65536, 131072, 250_000)
 WORKLOAD_TEXT = {
     "tiny": "Tiny Ulysses layer P=2 N=1024 H=8 D=128 packed QKV bf16",
     "dit19k": "Video-DiT geometry P=4 N=19394 H=56 D=128 packed QKV bf16 [N,3,H,D]",
@@ -43,6 +45,8 @@ WORKLOAD_TEXT = {
     "long104k": "Long clip P=8 N=104448 H=56 D=128 packed QKV bf16",
     "long104k-varlen": "Long clip varlen P=8 N=104448 H=56 D=128, 3 sequences 52224/31232/20992",
     "prof8k": "Profiling case P=4 N=8192 H=56 D=128 packed QKV bf16",
+    "stress250k": "Repack stress P=4 N=250000 H=56 D=128 packed QKVG bf16, one 896,000,000-byte plane per rank "
+                  "per launch; repack fwd+bwd; N sweep 4096..250000",
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
@@ -284,6 +288,72 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def run_repack_stress(args, rank, world, local_rank):
+    """Repack forward + backward at 250k tokens (QKVG), then a GB/s sweep over N."""
+    import torch
+    import torch.distributed as dist
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    P, N, H, C, seed, _ = WORKLOADS["stress250k"]
+    stream = torch.cuda.current_stream()
+
+    def time_pair(n, steps, warmup):
+        plan = U.ulysses_plan(n, H, 128, P, C)
+        Np = plan.padded_tokens
+        S = inputs.qkv_seq(n, H, P, C, seed, dev)
+        T = torch.empty((P, C, Np, H // P, 128), dtype=torch.bfloat16, device=dev)
+        back = torch.empty_like(S)
+        for _ in range(warmup):
+            U.ulysses_repack_fwd(plan, S, T, stream)
+            U.ulysses_repack_bwd(plan, T, back, C, stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        tf = tb = 0.0
+        for _ in range(steps):
+            ev[0].record(stream)
+            U.ulysses_repack_fwd(plan, S, T, stream)
+            ev[1].record(stream)
+            U.ulysses_repack_bwd(plan, T, back, C, stream)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            tf += ev[0].elapsed_time(ev[1])
+            tb += ev[1].elapsed_time(ev[2])
+        ok = torch.equal(back, S)
+        nbytes = 2 * S.numel() * 2          # read + write per direction
+        return tf / steps, tb / steps, nbytes, ok, plan.plane_chunk
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    tf, tb, nbytes, ok, chunk = time_pair(N, args.steps, args.warmup)
+    clocks = sampler.stop()
+    sweep = []
+    for n in SWEEP_N:
+        f, b, nb, ok_n, ch = time_pair(n, max(3, args.steps // 2), 3)
+        sweep.append({"N": n, "fwd_gbs": round(nb / (f * 1e-3) / 1e9, 1), "bwd_gbs": round(nb / (b * 1e-3) / 1e9, 1),
+                      "planes_per_launch": ch, "round_trip_exact": ok_n})
+    if rank != 0:
+        return None
+    pk, pk_kind = peaks()
+    gbs_f, gbs_b = nbytes / (tf * 1e-3) / 1e9, nbytes / (tb * 1e-3) / 1e9
+    return {
+        "metric": "Ulysses layer µs; attn TFLOP/s and repack GB/s vs B200 peak",
+        "value": round((tf + tb) * 1000, 1), "unit": "us per repack fwd+bwd", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tf + tb, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic N(0,1) bf16, seeded",
+        "config": {"workload": WORKLOAD_TEXT["stress250k"], "name": "stress250k", "planes_per_launch": chunk,
+                   "l2": "inputs larger than L2 (14.3 GB per direction)"},
+        "repack_fwd_gbs": round(gbs_f, 1), "repack_bwd_gbs": round(gbs_b, 1), "round_trip_exact": ok,
+        "roofline": {"bound": "hbm", "kernel": "repack_kernel", "achieved": round(gbs_f, 1), "peak": pk["hbm_gbs"],
+                     "peak_kind": f"{pk_kind} copy", "unit": "GB/s", "frac": round(gbs_f / pk["hbm_gbs"], 3),
+                     "frac_spec_8TBs": round(gbs_f / SPEC_PEAKS["hbm_gbs"], 3),
+                     "traffic": recorded_traffic("repack_kernel", "stress250k")},
+        "sweep": sweep, "clocks": clocks,
+        "gpu_launches": 2 * C * args.steps,
+    }
+
+
 # ---------------------------------------------------------------------------- CPU oracle
 
 def _cores():
@@ -300,6 +370,13 @@ def oracle_sample(config, S_bits, rows_per_head=1024, heads=4, token_frac=16):
     P, N, H, C, seed, cu = WORKLOADS[config]
     Np = S_bits.shape[0]
     Hl = H // P
+    if config == "stress250k":   # repack forward + backward of all planes only
+        ns = max(P, (Np // token_frac) // P * P)
+        t0 = time.perf_counter()
+        Tsub = orc.repack_fwd(np.ascontiguousarray(S_bits[:ns]), P)
+        orc.repack_bwd(Tsub)
+        t = (time.perf_counter() - t0) * (Np / ns)
+        return t * 1e6, f"repack fwd+bwd of {ns}/{Np} tokens (x{Np / ns:.1f}), extrapolated linearly"
     # repack: a token slice (multiple of P rows), scaled by the slice fraction
     ns = max(P, (Np // token_frac) // P * P)
     t0 = time.perf_counter()
@@ -395,7 +472,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        if args.config == "stress250k":
+            line = run_repack_stress(args, rank, world, local_rank)
+        else:
+            line = run_ours(args, rank, world, local_rank)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

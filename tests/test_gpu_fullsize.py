@@ -1,0 +1,107 @@
+"""Full-size workloads, in the launch configuration the benchmark times.
+
+Repack: bit-exact against the oracle's index map (at 250k tokens one plane of
+896,000,000 bytes per rank at a time).  Attention: a seeded subset of 4096
+query rows per head against the fp64 oracle (rows 0, N-1 and every segment
+boundary always included), max-abs <= 2e-2 and mean-abs <= 2e-3; the fused
+layer equals the unfused layer bit for bit everywhere.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import ulysses_oracle as orc
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+ROWS_PER_HEAD = 4096
+
+# name: (P, N, H, C, seed, cu_seqlens)
+FULL = {
+    "dit19k": (4, 19_394, 56, 3, 1, None),
+    "clip38k-qkvg": (4, 38_912, 56, 4, 2, None),
+    "long104k": (8, 104_448, 56, 3, 3, None),
+    "long104k-varlen": (8, 104_448, 56, 3, 3, [0, 52_224, 83_456, 104_448]),
+}
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_layer(gpu, name):
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    P, N, H, C, seed, cu = FULL[name]
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu)
+    Np, Hl = plan.padded_tokens, H // P
+    S = inputs.qkv_seq(N, H, P, C, seed, gpu)
+    T = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    OSf = torch.empty_like(OS)
+    scale = 1.0 / math.sqrt(128)
+    # the benchmark's step, call by call
+    U.ulysses_repack_fwd(plan, S, T)
+    U.ulysses_attn_fwd(plan, T, OT, scale)
+    U.ulysses_repack_bwd(plan, OT, OS, 1)
+    U.ulysses_layer_fwd(plan, S, OSf, None, fused=1)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+
+    # step 1: bit-exact, plane by plane
+    for c in range(C):
+        s_c = inputs.host_bits(S[:, c:c + 1])
+        assert np.array_equal(inputs.host_bits(T[:, c:c + 1]), orc.repack_fwd(s_c, P)), f"plane {c}"
+        del s_c
+    # the fused layer never materialises T: it must still equal the unfused one
+    assert torch.equal(OS, OSf)
+
+    # step 2 on sampled rows (T is now known to equal the oracle's repack)
+    rows = orc.sample_rows(N, ROWS_PER_HEAD, seed, cu)
+    T_bits = inputs.host_bits(T[:, :3])
+    ref = orc.attention_heads(T_bits, N, scale, cu_seqlens=cu, rows=rows, workers=_cores())
+    del T_bits
+    idx = torch.from_numpy(rows).to(gpu)
+    got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert err.max() <= MAX_ABS, err.max()
+    assert err.mean() <= MEAN_ABS, err.mean()
+    # step 3: the layer output rows are the attention rows, heads regrouped
+    lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(lay, orc.output_repack_bwd(got))
+    # pad rows
+    if Np > N:
+        assert not OS[N:].any() and not OT[:, N:].any()
+
+
+def test_repack_stress_250k_qkvg(gpu):
+    """250,000 tokens, 56 heads, QKVG, SP 4: one 896,000,000-byte plane per rank per launch."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    P, N, H, C = 4, 250_000, 56, 4
+    plan = U.ulysses_plan(N, H, 128, P, C)
+    assert plan.window_bytes_per_plane == 896_000_000 and plan.plane_chunk == 1
+    S = inputs.qkv_seq(N, H, P, C, 4, gpu)
+    T = torch.empty((P, C, N, H // P, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, T)
+    back = torch.empty_like(S)
+    U.ulysses_repack_bwd(plan, T, back, C)
+    torch.cuda.synchronize()
+    assert torch.equal(back, S)          # mode 1 after mode 0 restores every bit
+    del back
+    for c in range(C):
+        s_c = inputs.host_bits(S[:, c:c + 1])
+        t_c = inputs.host_bits(T[:, c:c + 1])
+        assert np.array_equal(t_c, orc.repack_fwd(s_c, P)), f"plane {c}"
+        del s_c, t_c

@@ -181,6 +181,40 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
  */
 int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream);
 
+/*
+ * The fused layer (as ulysses_layer_fwd with fused = 1) for callers that
+ * cannot allocate device memory: code running inside an allocator or memory
+ * pool callback, a process whose device memory is reserved up front, or a
+ * runtime that forbids cudaMalloc after start-up.  ulysses_plan() allocates a
+ * device error word, so those callers cannot make a plan; this entry point
+ * takes the plan's arguments directly and allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library call).  The pages have no counterpart: it
+ * exists for this library's users only.
+ *
+ * The attention kernel's only scratch memory, its 4-byte device error word,
+ * lives in a file-scope device array of 256 bytes that every GPU loading the
+ * library holds until the process exits.  Each call clears the word on
+ * `stream` before launching.  All calls share that array, so calls that
+ * overlap on the GPU (other streams, other threads) race on it.  The first
+ * call on each device looks up the array's device address (and may trigger
+ * the library's lazy module load): make that first call before any stream
+ * capture.  A call never needs more than the 4 bytes, whatever N, H or P; a
+ * scratch requirement above the 256-byte maximum would be refused with
+ * ULYSSES_ERR_UNSUPPORTED.
+ *
+ * Arguments as ulysses_plan() (planes must be >= 3) and ulysses_layer_fwd():
+ * qkv_seq / out_seq are device buffers ([Np, C, H, D] by default strides,
+ * [Np, H, D] out).  host_status: NULL for a fully asynchronous call;
+ * otherwise the call synchronises `stream` after the launch and stores the
+ * kernel's error bits there (0 = none; ULYSSES_ERR_DEVICE is returned when
+ * they are non-zero).  Errors: ARG, DIVISIBILITY, ALIGN, UNSUPPORTED, CUDA,
+ * DEVICE.
+ */
+int ulysses_layer_fwd_fused_noalloc(const void* qkv_seq, void* out_seq, int64_t N, int32_t H, int32_t D,
+                                    int32_t P, int32_t planes, int64_t token_stride, int64_t plane_stride,
+                                    const int32_t* cu_seqlens_host, int32_t num_seqs, int32_t* host_status,
+                                    void* stream);
+
 /* Static description of a return code. */
 const char* ulysses_strerror(int code);
 

@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     ulysses_attn_fwd,
     ulysses_last_device_error,
     ulysses_layer_fwd,
+    ulysses_layer_fwd_fused_noalloc,
     ulysses_layer_fwd_host,
     ulysses_plan,
     ulysses_repack_bwd,

@@ -32,6 +32,7 @@ EXPORTS = (
     "ulysses_plan_window_bytes_per_plane", "ulysses_workspace_bytes", "ulysses_repack_fwd",
     "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
     "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
+    "ulysses_layer_fwd_fused_noalloc",
 )
 
 
@@ -87,6 +88,10 @@ def load() -> ctypes.CDLL:
         lib.ulysses_last_device_error.restype = ctypes.c_int
         lib.ulysses_strerror.argtypes = [ctypes.c_int]
         lib.ulysses_strerror.restype = ctypes.c_char_p
+        lib.ulysses_layer_fwd_fused_noalloc.argtypes = [vp, vp, i64, i32, i32, i32, i32, i64, i64,
+                                                        ctypes.POINTER(ctypes.c_int32), i32,
+                                                        ctypes.POINTER(ctypes.c_int32), vp]
+        lib.ulysses_layer_fwd_fused_noalloc.restype = ctypes.c_int
         lib.ulysses_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
         lib.ulysses_selftest_exp2_poly.restype = ctypes.c_int
         _handle = lib
@@ -218,3 +223,25 @@ def ulysses_selftest_exp2_poly(x, y, stream=None) -> None:
     """y = 2^x with the attention kernel's FMA-pipe exponential (float32 device tensors)."""
     _check(load().ulysses_selftest_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)),
            "ulysses_selftest_exp2_poly")
+
+
+def ulysses_layer_fwd_fused_noalloc(qkv_seq, out_seq, N: int, H: int, D: int, P: int, planes: int,
+                                    token_stride: int = 0, plane_stride: int = 0, cu_seqlens=None,
+                                    check: bool = False, stream=None) -> int:
+    """The fused layer without a plan and without any device allocation.
+
+    Returns the kernel's error bits when ``check`` is true (the call then
+    synchronises the stream), else 0.
+    """
+    if cu_seqlens is None:
+        arr, ns = None, 0
+    else:
+        vals = [int(x) for x in cu_seqlens]
+        arr = (ctypes.c_int32 * len(vals))(*vals)
+        ns = len(vals) - 1
+    status = ctypes.c_int32(0)
+    code = load().ulysses_layer_fwd_fused_noalloc(_ptr(qkv_seq), _ptr(out_seq), int(N), int(H), int(D), int(P),
+                                                  int(planes), int(token_stride), int(plane_stride), arr, ns,
+                                                  ctypes.byref(status) if check else None, _stream(stream))
+    _check(code, "ulysses_layer_fwd_fused_noalloc")
+    return status.value

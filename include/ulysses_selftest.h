@@ -23,6 +23,17 @@ extern "C" {
  */
 int ulysses_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
+/*
+ * Failure-path check of the kernels' bounded waits: one CTA waits on an
+ * mbarrier phase that nothing completes, first with the single-thread wait,
+ * then with the warp-collective wait, each limited to limit_us microseconds
+ * (1 .. 1,000,000).  Each wait gives up, sets bit 1 (wait timeout) of
+ * *dev_err, and the kernel also sets 0x100 / 0x200 for the two waits and
+ * returns; the context stays usable.  dev_err is a caller-owned device word.
+ * Returns 0, 1 for a bad argument, 6 for a CUDA launch error.
+ */
+int ulysses_selftest_wait_timeout(unsigned int* dev_err, int64_t limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,3 +36,34 @@ def test_fma_pipe_exp2_clamps_below_range(gpu):
     torch.cuda.synchronize()
     got = y.cpu().numpy().astype(np.float64)
     assert np.all(np.isfinite(got)) and np.all(got > 0) and np.all(got <= 2.0 ** -124)
+
+
+def test_bounded_wait_gives_up_and_reports(gpu):
+    """A wait on a phase nothing completes returns after its limit with the error bits set."""
+    import math
+    import time
+
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    lib = U.load()
+    err = torch.zeros(4, dtype=torch.int32, device=gpu)
+    t0 = time.time()
+    assert lib.ulysses_selftest_wait_timeout(err.data_ptr(), 20_000, torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    elapsed = time.time() - t0
+    word = int(err[0].item())
+    assert word & 1, word                      # kErrWaitTimeout
+    assert word & 0x100 and word & 0x200, hex(word)
+    assert elapsed < 5.0
+    # the context is still usable: a small layer still matches the fused path
+    from ulysses_sequence_attention_repack_b200 import inputs
+    plan = U.ulysses_plan(300, 4, 128, 2, 3)
+    S = inputs.qkv_seq(300, 4, 2, 3, 3, gpu)
+    a = torch.empty((300, 4, 128), dtype=torch.bfloat16, device=gpu)
+    b = torch.empty_like(a)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_layer_fwd(plan, S, a, ws, fused=0)
+    U.ulysses_layer_fwd(plan, S, b, None, fused=1)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and U.ulysses_last_device_error(plan) == 0
+    assert math.isfinite(float(a.float().abs().sum()))

@@ -32,7 +32,7 @@ EXPORTS = (
     "ulysses_plan_window_bytes_per_plane", "ulysses_workspace_bytes", "ulysses_repack_fwd",
     "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
     "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
-    "ulysses_layer_fwd_fused_noalloc",
+    "ulysses_layer_fwd_fused_noalloc", "ulysses_selftest_wait_timeout",
 )
 
 
@@ -92,6 +92,8 @@ def load() -> ctypes.CDLL:
                                                         ctypes.POINTER(ctypes.c_int32), i32,
                                                         ctypes.POINTER(ctypes.c_int32), vp]
         lib.ulysses_layer_fwd_fused_noalloc.restype = ctypes.c_int
+        lib.ulysses_selftest_wait_timeout.argtypes = [vp, i64, vp]
+        lib.ulysses_selftest_wait_timeout.restype = ctypes.c_int
         lib.ulysses_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
         lib.ulysses_selftest_exp2_poly.restype = ctypes.c_int
         _handle = lib

@@ -20,7 +20,35 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
   }
 }
 
+// One CTA waits on an mbarrier phase that nothing completes, once with the
+// single-thread wait and once with the warp-collective wait, each bounded by
+// limit_ns.  Both must give up, set kErrWaitTimeout in *err, and return.
+__global__ void wait_timeout_kernel(unsigned int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ulysses::mbar_init(ulysses::smem_u32(&bar), 1);
+    abort_flag = 0;
+    ulysses::fence_mbar_init();
+  }
+  __syncthreads();
+  ulysses::WaitGuard g{&abort_flag, err, limit_ns};
+  if (threadIdx.x == 0) {
+    if (!ulysses::mbar_wait(ulysses::smem_u32(&bar), 0, g)) atomicOr(err, 0x100u);
+    abort_flag = 0;   // re-arm so the warp-wide wait also runs its own limit
+  }
+  __syncwarp();
+  if (!ulysses::mbar_wait_warp(ulysses::smem_u32(&bar), 0, g) && threadIdx.x == 0) atomicOr(err, 0x200u);
+}
+
 }  // namespace
+
+extern "C" int ulysses_selftest_wait_timeout(unsigned int* dev_err, int64_t limit_us, void* stream) {
+  if (!dev_err || limit_us < 1 || limit_us > 1000000) return 1;
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev_err,
+                                                                      static_cast<uint64_t>(limit_us) * 1000u);
+  return cudaGetLastError() == cudaSuccess ? 0 : 6;
+}
 
 extern "C" int ulysses_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
   if (!x || !y || n < 0) return 1;

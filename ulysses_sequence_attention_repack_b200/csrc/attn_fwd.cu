@@ -9,18 +9,23 @@
 // the softmax is kept online (running max and sum), so the N x N score matrix
 // never leaves the SM.
 //
-// Design (one persistent CTA per SM, 10 warps):
+// Design (one persistent CTA per SM, 12 warps):
 //   warp 9      TMA producer: Q tiles (2 x 128 rows) and a 2-stage K ring and
 //               V ring, 128-byte swizzled, completion counted on mbarriers.
 //   warp 8      tcgen05 issuer (one lane): S_i = Q_i K^T into TMEM (fp32),
 //               then O_i += P_i V with P_i read from TMEM (bf16, aliased over
-//               S_i) and V from shared memory.  Two Q tiles ping-pong so the
-//               tensor core works on one tile while the other is in softmax.
+//               S_i) and V from shared memory, each group of MMAs one asm
+//               block with precomputed descriptors.  Two Q tiles ping-pong so
+//               the tensor core works on one tile while the other is in
+//               softmax (one issuer per tile was measured slower: the
+//               interleaving delays each tile's S).
 //   warps 0-7   two softmax warpgroups, one per Q tile; thread t of a group
 //               owns query row t, so row max and row sum need no shuffles.
+//               P is handed over in two halves (keys 0-63, then 64-127).
 //               The running max is only moved (and O rescaled in TMEM) when
 //               it grows by more than 8 in log2 units; the final 1/l uses the
-//               same stale max, so the result is unchanged.
+//               same stale max, so the result is unchanged.  The first thread
+//               of group 1 releases the K/V ring slots.
 // TMEM: S0 | S1 | O0 | O1, 128 fp32 columns each (all 512 columns).
 //
 // Every wait is bounded: on timeout the kernel sets an error bit, skips the
@@ -300,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(BAR(B_SFULL0));
         issue_s(1, ks);
         mma_commit(BAR(B_SFULL1));
-        mma_commit(BAR(B_KEMPTY0 + ks));
         ++kc;
         if (nkv == 1) mma_commit(BAR(B_QEMPTY));
         for (int t = 0; ok && t < nkv; ++t) {
@@ -325,14 +329,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               issue_s(1, ks);
               mma_commit(BAR(B_SFULL1));
-              mma_commit(BAR(B_KEMPTY0 + ks));
               ++kc;
               if (t + 1 == nkv - 1) mma_commit(BAR(B_QEMPTY));
             }
           }
           ++pc;
           if (!ok) break;
-          mma_commit(BAR(B_VEMPTY0 + vs));
           ++vc;
         }
       }
@@ -351,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + kColO0 + 128 * wg;
     const float sl2 = p.scale_log2;
     uint32_t sc = 0, uc = 0;
+    uint32_t kslot = 0, vslot = 0;   // K / V ring fills consumed (warpgroup 1 releases them)
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
       Unit w;
@@ -362,6 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < nkv; ++t) {
         if (!(ok = mbar_wait_warp(BAR(B_SFULL0 + wg), sc & 1, g))) break;
         ++sc;
+        if (wg == 1 && row == 0) {
+          // S1(t) complete => S0(t) complete (same issuer, issued earlier):
+          // K(t) is free.  S1(t) was issued after P1(t-1) V(t-1), the last
+          // use of V(t-1).  Releasing here saves two tcgen05.commit per step.
+          mbar_arrive(BAR(B_KEMPTY0 + kslot % kStages));
+          ++kslot;
+          if (t > 0) mbar_arrive(BAR(B_VEMPTY0 + vslot++ % kStages));
+        }
         tc_fence_after();
         uint32_t sraw[4][32];
 #pragma unroll
@@ -443,6 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // epilogue: O / l -> bf16 -> global
       if (!(ok = mbar_wait_warp(BAR(B_OFULL0 + wg), uc & 1, g))) break;
+      if (wg == 1 && row == 0) mbar_arrive(BAR(B_VEMPTY0 + vslot++ % kStages));   // last V of the unit
       tc_fence_after();
       uint32_t oraw[4][32];
 #pragma unroll

@@ -195,13 +195,17 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) ->
 
 def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
                     rows: np.ndarray | None = None, workers: int = 1,
-                    row_block: int = 256) -> np.ndarray:
+                    row_block: int = 256, causal: bool = False) -> np.ndarray:
     """Step two of the layer: attention on every head-sharded slab.
 
     T: head-sharded ``[P, C, Np, Hl, D]`` uint16; planes 0, 1, 2 are Q, K, V
     (a fourth plane, the gate, is ignored).  Query row n attends to the keys of
     its own segment (all keys ``< N`` without ``cu_seqlens``).  Rows ``n >= N``
     are padding and give zero.
+
+    With ``causal``, query row n attends only to keys m <= n of its segment
+    (the causal attention of the trainer's Ulysses flash wrapper in "Ulysses
+    context parallelism" of the prime-rl pull request).
 
     Returns fp64 ``[P, R, Hl, D]`` for the selected rows (all ``Np`` rows when
     ``rows`` is None).  Query rows are independent, so they are evaluated
@@ -226,6 +230,12 @@ def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
                 continue
             k = bf16_bits_to_f64(T[r, 1, a:b, j, :])
             v = bf16_bits_to_f64(T[r, 2, a:b, j, :])
+            if causal:
+                for i in sel:
+                    n = int(rows[i])
+                    q = bf16_bits_to_f64(T[r, 0, n:n + 1, j, :])
+                    out[r, i, j, :] = attention_rows(q, k[:n + 1 - a], v[:n + 1 - a], scale)[0]
+                continue
             for i0 in range(0, sel.size, row_block):
                 part = sel[i0:i0 + row_block]
                 q = bf16_bits_to_f64(T[r, 0, rows[part], j, :])
@@ -253,14 +263,14 @@ def output_repack_bwd(O_heads: np.ndarray) -> np.ndarray:
 
 
 def layer_fwd(S: np.ndarray, P: int, N: int, scale: float, cu_seqlens=None,
-              rows: np.ndarray | None = None, workers: int = 1) -> np.ndarray:
+              rows: np.ndarray | None = None, workers: int = 1, causal: bool = False) -> np.ndarray:
     """The whole layer: repack -> attention per slab -> inverse repack.
 
     S: sequence-sharded ``[Np, C, H, D]`` uint16.  Returns fp64 ``[R, H, D]``
     (sequence-sharded output rows, all ``Np`` rows when ``rows`` is None).
     """
     T = repack_fwd(S, P)
-    O = attention_heads(T, N, scale, cu_seqlens=cu_seqlens, rows=rows, workers=workers)
+    O = attention_heads(T, N, scale, cu_seqlens=cu_seqlens, rows=rows, workers=workers, causal=causal)
     return output_repack_bwd(O)
 
 
@@ -282,9 +292,16 @@ def sample_rows(N: int, count: int, seed: int, cu_seqlens=None) -> np.ndarray:
     return np.array(sorted(chosen | forced), dtype=np.int64)
 
 
-def attention_flops(N: int, H: int, D: int, cu_seqlens=None) -> float:
-    """Algorithmic attention FLOPs: 4 * L^2 * H * D summed over sequences."""
-    return float(sum(4 * (b - a) ** 2 * H * D for a, b in segments_from_cu_seqlens(cu_seqlens, N)))
+def attention_flops(N: int, H: int, D: int, cu_seqlens=None, causal: bool = False) -> float:
+    """Algorithmic attention FLOPs: 4 * L^2 * H * D summed over sequences.
+
+    Causal: each query row n of a segment starting at a uses n - a + 1 keys,
+    i.e. 4 * H * D * L (L + 1) / 2 per segment.
+    """
+    segs = segments_from_cu_seqlens(cu_seqlens, N)
+    if causal:
+        return float(sum(4 * H * D * (b - a) * (b - a + 1) // 2 for a, b in segs))
+    return float(sum(4 * (b - a) ** 2 * H * D for a, b in segs))
 
 
 def softmax_scale(D: int) -> float:

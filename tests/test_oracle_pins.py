@@ -275,3 +275,56 @@ def test_flop_count():
     assert orc.attention_flops(1024, 8, 128) == 4 * 1024 ** 2 * 8 * 128
     cu = [0, 52224, 83456, 104448]
     assert orc.attention_flops(104448, 56, 128, cu) == sum(4 * L ** 2 * 56 * 128 for L in (52224, 31232, 20992))
+
+
+# ---------------------------------------------------------------- causal variant
+
+def _plain_causal_mha(S, segs, scale):
+    Np, C, H, D = S.shape
+    out = np.zeros((Np, H, D))
+    for h in range(H):
+        for a, b in segs:
+            for n in range(a, b):
+                q = orc.bf16_bits_to_f64(S[n:n + 1, 0, h])
+                k = orc.bf16_bits_to_f64(S[a:n + 1, 1, h])
+                v = orc.bf16_bits_to_f64(S[a:n + 1, 2, h])
+                out[n, h] = _brute_force_softmax(q, k, v, scale)[0]
+    return out
+
+
+@pytest.mark.parametrize("P,N,H,cu", [(2, 12, 4, None), (4, 10, 8, None), (2, 14, 4, [0, 5, 6, 14])])
+def test_causal_layer_equals_plain_causal_attention(P, N, H, cu):
+    rng = np.random.default_rng(40 + N)
+    D = 8
+    Np = orc.padded_tokens(N, P)
+    S = _bf16_normal(rng, (Np, 3, H, D))
+    S[N:] = 0
+    got = orc.layer_fwd(S, P, N, 0.4, cu_seqlens=cu, causal=True)
+    segs = [(0, N)] if cu is None else list(zip(cu, cu[1:]))
+    want = _plain_causal_mha(S, segs, 0.4)
+    assert np.allclose(got[:N], want[:N], rtol=0, atol=1e-12)
+    assert np.all(got[N:] == 0)
+
+
+def test_causal_first_row_of_each_segment_is_its_value():
+    # the first query of a segment sees exactly one key: its own
+    rng = np.random.default_rng(41)
+    cu = [0, 4, 9]
+    S = _bf16_normal(rng, (9, 3, 2, 8))
+    got = orc.layer_fwd(S, 1, 9, 0.7, cu_seqlens=cu, causal=True)
+    for a in cu[:-1]:
+        assert np.array_equal(got[a], orc.bf16_bits_to_f64(S[a, 2]))
+
+
+def test_causal_last_row_equals_non_causal_last_row():
+    rng = np.random.default_rng(42)
+    S = _bf16_normal(rng, (8, 3, 2, 8))
+    full = orc.layer_fwd(S, 2, 8, 0.3)
+    causal = orc.layer_fwd(S, 2, 8, 0.3, causal=True)
+    assert np.allclose(full[7], causal[7], rtol=0, atol=1e-12)
+    assert not np.allclose(full[0], causal[0])
+
+
+def test_causal_flop_count():
+    assert orc.attention_flops(4, 1, 1, causal=True) == 4 * (1 + 2 + 3 + 4)
+    assert orc.attention_flops(6, 2, 8, [0, 2, 6], causal=True) == 4 * 2 * 8 * ((1 + 2) + (1 + 2 + 3 + 4))

@@ -36,7 +36,9 @@ WORKLOADS = {
     "long104k-varlen": (8, 104_448, 56, 3, 3, [0, 52_224, 83_456, 104_448]),
     "prof8k": (4, 8192, 56, 3, 1, None),   # small case for profiler captures (352 MB input > L2)
     "stress250k": (4, 250_000, 56, 4, 4, None),   # repack fwd + bwd only, plus an N sweep
+    "dit19k-causal": (4, 19_394, 56, 3, 1, None),
 }
+CAUSAL = {"dit19k-causal"}
 SWEEP_N = (4096, 8192, 16384, 32768, 65536, 131072, 250_000)
 WORKLOAD_TEXT = {
     "tiny": "Tiny Ulysses layer P=2 N=1024 H=8 D=128 packed QKV bf16",
@@ -47,6 +49,7 @@ WORKLOAD_TEXT = {
     "prof8k": "Profiling case P=4 N=8192 H=56 D=128 packed QKV bf16",
     "stress250k": "Repack stress P=4 N=250000 H=56 D=128 packed QKVG bf16, one 896,000,000-byte plane per rank "
                   "per launch; repack fwd+bwd; N sweep 4096..250000",
+    "dit19k-causal": "Video-DiT geometry with causal attention P=4 N=19394 H=56 D=128 packed QKV bf16",
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
@@ -61,8 +64,10 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def attn_flops(N, H, cu):
+def attn_flops(N, H, cu, causal=False):
     segs = [(0, N)] if cu is None else list(zip(cu, cu[1:]))
+    if causal:
+        return float(sum(4 * H * 128 * (b - a) * (b - a + 1) // 2 for a, b in segs))
     return float(sum(4 * (b - a) ** 2 * H * 128 for a, b in segs))
 
 
@@ -140,8 +145,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     P, N, H, C, seed, cu = WORKLOADS[args.config]
+    causal = args.config in CAUSAL
     Hl = H // P
-    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu)
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu, causal=causal)
     Np = plan.padded_tokens
     S = inputs.qkv_seq(N, H, P, C, seed, dev)
     T = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
@@ -233,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
         return None
 
     pk, pk_kind = peaks()
-    flops = attn_flops(N, H, cu)
+    flops = attn_flops(N, H, cu, causal)
     at_ms = statistics.mean(t_at)
     rf_ms, rb_ms = statistics.mean(t_rf), statistics.mean(t_rb)
     rf_bytes = 2 * C * Np * H * 128 * 2
@@ -258,7 +264,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16",
         "data": "synthetic N(0,1) bf16, seeded",
         "config": {"workload": WORKLOAD_TEXT[args.config], "name": args.config, "P": P, "N": N, "Np": Np,
-                   "H": H, "D": 128, "planes": C, "seed": seed, "cu_seqlens": cu,
+                   "H": H, "D": 128, "planes": C, "seed": seed, "cu_seqlens": cu, "causal": causal,
                    "step": "repack_fwd + attn_fwd + repack_bwd(output), one C-ABI call each",
                    "replicas": world, "l2": f"inputs larger than L2 ({S.numel() * 2 / 1e6:.0f} MB per step)"},
         "attn_us": round(at_ms * 1000, 2),

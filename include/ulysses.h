@@ -71,6 +71,10 @@ enum {
 #define ULYSSES_MAX_WINDOW_BYTES (1024LL * 1024LL * 1024LL)
 /* Most packed sequences one plan accepts (cu_seqlens has num_seqs + 1 entries). */
 #define ULYSSES_MAX_SEQS 64
+/* ulysses_plan_ex flag: causal attention (query n sees keys m <= n of its
+ * segment), as in the causal flash wrapper of the prime-rl Ulysses context
+ * parallelism pull request. */
+#define ULYSSES_PLAN_CAUSAL 1u
 
 typedef struct ulysses_plan_s ulysses_plan_t;
 
@@ -102,6 +106,12 @@ typedef struct ulysses_plan_s ulysses_plan_t;
 int ulysses_plan(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
                  int64_t token_stride, int64_t plane_stride, int64_t plane_chunk,
                  const int32_t* cu_seqlens_host, int32_t num_seqs);
+
+/* ulysses_plan with option flags (ULYSSES_PLAN_CAUSAL); ulysses_plan is
+ * ulysses_plan_ex with flags = 0.  Unknown flag bits -> ULYSSES_ERR_ARG. */
+int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
+                    int64_t token_stride, int64_t plane_stride, int64_t plane_chunk,
+                    const int32_t* cu_seqlens_host, int32_t num_seqs, uint32_t flags);
 
 void ulysses_plan_destroy(ulysses_plan_t* plan);
 
@@ -140,8 +150,9 @@ int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* 
 /*
  * Step 2: out_heads O_T [P, Np, Hl, D] = softmax(softmax_scale * Q K^T) V for
  * every rank r and local head j, with Q, K, V the planes 0, 1, 2 of
- * qkv_heads T [P, C, Np, Hl, D].  Non-causal; query row n attends to the keys
- * of its cu_seqlens segment (all keys < N without cu_seqlens).  fp32
+ * qkv_heads T [P, C, Np, Hl, D].  Non-causal unless the plan was made with
+ * ULYSSES_PLAN_CAUSAL; query row n attends to the keys of its cu_seqlens
+ * segment (all keys < N without cu_seqlens), only those m <= n when causal.  fp32
  * accumulation and softmax, bf16 probabilities for the second product, bf16
  * output; pad rows [N, Np) are written as zeros.  Errors: ARG, ALIGN, CUDA.
  */

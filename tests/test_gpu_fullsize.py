@@ -105,3 +105,30 @@ def test_repack_stress_250k_qkvg(gpu):
         t_c = inputs.host_bits(T[:, c:c + 1])
         assert np.array_equal(t_c, orc.repack_fwd(s_c, P)), f"plane {c}"
         del s_c, t_c
+
+
+def test_full_layer_causal_dit19k(gpu):
+    """Causal variant at the Video-DiT size: 512 seeded rows per head against fp64."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    P, N, H, C, seed = 4, 19_394, 56, 3, 1
+    plan = U.ulysses_plan(N, H, 128, P, C, causal=True)
+    Np, Hl = plan.padded_tokens, H // P
+    S = inputs.qkv_seq(N, H, P, C, seed, gpu)
+    T = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, T)
+    U.ulysses_attn_fwd(plan, T, OT, 1.0 / math.sqrt(128))
+    U.ulysses_layer_fwd(plan, S, OS, None, fused=1)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    rows = orc.sample_rows(N, 512, seed)
+    ref = orc.attention_heads(inputs.host_bits(T[:, :3]), N, 1.0 / math.sqrt(128), rows=rows, causal=True)
+    idx = torch.from_numpy(rows).to(gpu)
+    got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(lay, orc.output_repack_bwd(got))

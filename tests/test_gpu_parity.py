@@ -109,6 +109,47 @@ def test_repack_attention_layer_against_oracle(gpu, P, N, H, C, layout, cu, seed
     assert np.array_equal(_bits(OS), orc.repack_bwd(_bits(OT)[:, None])[:, 0])
 
 
+CAUSAL_CASES = [
+    pytest.param(2, 1024, 8, None, 13, id="causal-tiny"),
+    pytest.param(4, 1001, 8, None, 14, id="causal-ragged"),
+    pytest.param(1, 300, 2, None, 15, id="causal-P1"),
+    pytest.param(2, 1000, 4, [0, 300, 301, 777, 1000], 16, id="causal-varlen"),
+    pytest.param(2, 700, 4, [0, 256, 512, 700], 17, id="causal-varlen-aligned"),
+]
+
+
+@pytest.mark.parametrize("P,N,H,cu,seed", CAUSAL_CASES)
+def test_causal_attention_against_oracle(gpu, P, N, H, cu, seed):
+    torch = _torch()
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=True)
+    Np, Hl = plan.padded_tokens, H // P
+    S = inputs.qkv_seq(N, H, P, 3, seed, gpu)
+    T = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, T)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_attn_fwd(plan, T, OT, 1.0 / math.sqrt(128))
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_layer_fwd(plan, S, OS, ws, fused=0)
+    OSf = torch.empty_like(OS)
+    U.ulysses_layer_fwd(plan, S, OSf, None, fused=1)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    ref = orc.attention_heads(_bits(T), N, 1.0 / math.sqrt(128), cu_seqlens=cu, causal=True)
+    err = np.abs(_f32(OT) - ref)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    assert np.all(_f32(OT)[:, N:] == 0)
+    assert np.array_equal(_bits(OS), _bits(OSf))
+    assert np.array_equal(_bits(OS), orc.repack_bwd(_bits(OT)[:, None])[:, 0])
+    # the first row of every segment is exactly its own value row, rounded to bf16
+    segs = [(0, N)] if cu is None else list(zip(cu, cu[1:]))
+    for a, b in segs:
+        if b > a:
+            np.testing.assert_array_equal(_bits(OS[a]), _bits(S[a, 2]))
+
+
 def test_sharp_softmax_diagnostic(gpu):
     """Q scaled by 8: peaked rows exercise the running-max rescale path."""
     torch = _torch()

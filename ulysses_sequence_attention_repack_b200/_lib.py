@@ -24,11 +24,12 @@ ULYSSES_ERR_WORKSPACE = 5
 ULYSSES_ERR_CUDA = 6
 ULYSSES_ERR_DEVICE = 7
 ULYSSES_ERR_UNSUPPORTED = 8
+ULYSSES_PLAN_CAUSAL = 1
 MAX_SEQS = 64
 MAX_WINDOW_BYTES = 1024 ** 3
 
 EXPORTS = (
-    "ulysses_plan", "ulysses_plan_destroy", "ulysses_plan_padded_tokens", "ulysses_plan_plane_chunk",
+    "ulysses_plan", "ulysses_plan_ex", "ulysses_plan_destroy", "ulysses_plan_padded_tokens", "ulysses_plan_plane_chunk",
     "ulysses_plan_window_bytes_per_plane", "ulysses_workspace_bytes", "ulysses_repack_fwd",
     "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
     "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
@@ -64,6 +65,9 @@ def load() -> ctypes.CDLL:
         lib.ulysses_plan.argtypes = [ctypes.POINTER(vp), i64, i32, i32, i32, i32, i64, i64, i64,
                                      ctypes.POINTER(ctypes.c_int32), i32]
         lib.ulysses_plan.restype = ctypes.c_int
+        lib.ulysses_plan_ex.argtypes = [ctypes.POINTER(vp), i64, i32, i32, i32, i32, i64, i64, i64,
+                                        ctypes.POINTER(ctypes.c_int32), i32, ctypes.c_uint32]
+        lib.ulysses_plan_ex.restype = ctypes.c_int
         lib.ulysses_plan_destroy.argtypes = [vp]
         lib.ulysses_plan_destroy.restype = None
         lib.ulysses_plan_padded_tokens.argtypes = [vp]
@@ -130,9 +134,10 @@ def _stream(stream) -> int | None:
 class Plan:
     """Owner of a ulysses_plan_t*; destroyed with the object."""
 
-    def __init__(self, handle: int, N: int, H: int, D: int, P: int, planes: int, cu_seqlens):
+    def __init__(self, handle: int, N: int, H: int, D: int, P: int, planes: int, cu_seqlens, causal: bool = False):
         self._h = ctypes.c_void_p(handle)
         self.N, self.H, self.D, self.P, self.planes = N, H, D, P, planes
+        self.causal = bool(causal)
         self.cu_seqlens = None if cu_seqlens is None else [int(x) for x in cu_seqlens]
 
     @property
@@ -170,7 +175,8 @@ class Plan:
 
 
 def ulysses_plan(N: int, H: int, D: int, P: int, planes: int, token_stride: int = 0, plane_stride: int = 0,
-                 plane_chunk: int = 0, cu_seqlens=None) -> Plan:
+                 plane_chunk: int = 0, cu_seqlens=None, causal: bool = False) -> Plan:
+    """ulysses_plan (or ulysses_plan_ex with ULYSSES_PLAN_CAUSAL when causal)."""
     lib = load()
     h = ctypes.c_void_p()
     if cu_seqlens is None:
@@ -179,10 +185,14 @@ def ulysses_plan(N: int, H: int, D: int, P: int, planes: int, token_stride: int 
         vals = [int(x) for x in cu_seqlens]
         arr = (ctypes.c_int32 * len(vals))(*vals)
         ns = len(vals) - 1
-    code = lib.ulysses_plan(ctypes.byref(h), int(N), int(H), int(D), int(P), int(planes), int(token_stride),
-                            int(plane_stride), int(plane_chunk), arr, ns)
+    if causal:
+        code = lib.ulysses_plan_ex(ctypes.byref(h), int(N), int(H), int(D), int(P), int(planes), int(token_stride),
+                                   int(plane_stride), int(plane_chunk), arr, ns, ULYSSES_PLAN_CAUSAL)
+    else:
+        code = lib.ulysses_plan(ctypes.byref(h), int(N), int(H), int(D), int(P), int(planes), int(token_stride),
+                                int(plane_stride), int(plane_chunk), arr, ns)
     _check(code, "ulysses_plan")
-    return Plan(h.value, N, H, D, P, planes, cu_seqlens)
+    return Plan(h.value, N, H, D, P, planes, cu_seqlens, causal)
 
 
 def ulysses_repack_fwd(plan: Plan, src_seq, dst_heads, stream=None) -> None:

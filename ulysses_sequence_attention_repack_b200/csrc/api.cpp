@@ -119,8 +119,16 @@ extern "C" {
 int ulysses_plan(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
                  int64_t token_stride, int64_t plane_stride, int64_t plane_chunk, const int32_t* cu_seqlens_host,
                  int32_t num_seqs) {
+  return ulysses_plan_ex(out, N, H, D, P, planes, token_stride, plane_stride, plane_chunk, cu_seqlens_host, num_seqs,
+                         0u);
+}
+
+int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
+                    int64_t token_stride, int64_t plane_stride, int64_t plane_chunk, const int32_t* cu_seqlens_host,
+                    int32_t num_seqs, uint32_t flags) {
   if (!out) return ULYSSES_ERR_ARG;
   *out = nullptr;
+  if (flags & ~ULYSSES_PLAN_CAUSAL) return ULYSSES_ERR_ARG;
   if (D != kHeadDim) return ULYSSES_ERR_UNSUPPORTED;
   if (N < 1 || H < 1 || P < 1 || planes < 1 || planes > kMaxPlanes) return ULYSSES_ERR_ARG;
   if (H > kMaxHeads) return ULYSSES_ERR_UNSUPPORTED;
@@ -183,6 +191,7 @@ int ulysses_plan(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t 
   p->plane_stride = plane_stride;
   p->plane_chunk = static_cast<int32_t>(chunk);
   p->num_seqs = nseq;
+  p->causal = (flags & ULYSSES_PLAN_CAUSAL) ? 1 : 0;
   std::memcpy(p->segs, segs, sizeof(ulysses::Segment) * nseq);
   p->device = -1;
   p->dev_err = nullptr;

@@ -1,11 +1,13 @@
-// Non-causal softmax attention for the Ulysses layer on sm_100a.
+// Softmax attention for the Ulysses layer on sm_100a.
 //
 //   O[n, :] = sum_{m in K(n)} softmax_m(scale * <Q_n, K_m>) V_m
 //
 // (the FA4 backend call of flash_attn_cute.py in "hao-ai-lab FastVideo,
 // compare aryan/h3-nvfp4-stack-speedups...main": softmax_scale, non-causal,
 // varlen through cu_seqlens).  K(n) is the key range of the packed sequence
-// holding row n.  Computed flash-style: keys are visited in tiles of 128 and
+// holding row n; with the causal option (the trainer's causal Ulysses flash
+// wrapper in the prime-rl Ulysses context-parallelism pull request) only the
+// keys m <= n of that range.  Computed flash-style: keys are visited in tiles of 128 and
 // the softmax is kept online (running max and sum), so the N x N score matrix
 // never leaves the SM.
 //
@@ -115,6 +117,7 @@ struct AttnParams {
   int64_t o_stride_r, o_stride_n, o_stride_j;
   int32_t N, Np;
   int32_t Hl, P, fused;
+  int32_t causal;                  // query n sees keys m <= n only
   int32_t num_units, nseg;
   float scale_log2;
   SegDesc seg[ULYSSES_MAX_SEQS];   // longest first
@@ -159,6 +162,13 @@ __device__ __forceinline__ void exp_store_half(const float* s, int half, f2 scal
     pk[c] = pack_bf16x2(e.x, e.y);
   }
   tmem_st32(tS + 32 * half, pk);
+}
+
+// Number of 128-key tiles a unit visits: the whole segment, or (causal) the
+// keys up to the unit's last query row.
+__device__ __forceinline__ int unit_kv_tiles(const AttnParams& p, const SegDesc& sd, const Unit& w) {
+  const int hi = p.causal ? min(sd.kv_end, w.q0 + kUnitRows) : sd.kv_end;
+  return (hi - sd.start + BN - 1) / BN;
 }
 
 // waits that ignore the abort flag (used for draining in-flight work)
@@ -237,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_5d(sbase + kOffQ + (2 * i + h) * kHalfBytes, &tmap, BAR(B_QFULL0 + i), 64 * h, hc,
                         w.q0 + i * BM, 0, rc);
         }
-        const int nkv = (sd.kv_end - sd.start + BN - 1) / BN;
+        const int nkv = unit_kv_tiles(p, sd, w);
         for (int t = 0; t < nkv; ++t) {
           const int kv0 = sd.start + t * BN;
           {
@@ -295,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         Unit w;
         if (!decode_unit(p, u, w)) break;
         const SegDesc& sd = p.seg[w.seg];
-        const int nkv = (sd.kv_end - sd.start + BN - 1) / BN;
+        const int nkv = unit_kv_tiles(p, sd, w);
         if (!(ok = mbar_wait(BAR(B_QFULL0), uc & 1, g))) break;
         if (!(ok = mbar_wait(BAR(B_QFULL1), uc & 1, g))) break;
         uint32_t ks = kc % kStages;
@@ -359,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Unit w;
       if (!decode_unit(p, u, w)) break;
       const SegDesc& sd = p.seg[w.seg];
-      const int nkv = (sd.kv_end - sd.start + BN - 1) / BN;
+      const int nkv = unit_kv_tiles(p, sd, w);
       float m_used = -INFINITY;   // running max, log2 units (scaled)
       float l = 0.f;              // running sum of exp2(x - m_used)
       for (int t = 0; t < nkv; ++t) {
@@ -381,8 +391,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_regs_ready(sraw[c]);
         float* s = reinterpret_cast<float*>(&sraw[0][0]);
-        if (t == nkv - 1) {
-          const int valid = sd.kv_end - (sd.start + t * BN);   // 1..128
+        // keys past the segment end, and (causal) past this row, are masked
+        const int kv0 = sd.start + t * BN;
+        const int row_n = w.q0 + wg * BM + row;
+        const int valid = (p.causal ? min(sd.kv_end, row_n + 1) : sd.kv_end) - kv0;   // may be <= 0
+        const bool masked = __any_sync(0xffffffffu, valid < BN);
+        if (masked) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= valid) s[c] = -INFINITY;
@@ -429,8 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
         // P (bf16 pairs) over the first 64 columns of S, in two halves; the
         // first half is handed to the MMA warp before the second is computed.
-        // The masked last tile uses MUFU ex2 only, so masked keys give exact zeros.
-        const bool emu = t != nkv - 1;
+        // Masked tiles use MUFU ex2 only, so masked keys give exact zeros.
+        const bool emu = !masked;
         if (emu)
           exp_store_half<true>(s, 0, scale2, negm2, acc, tS);
         else
@@ -558,6 +572,7 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   p.Hl = a.Hl;
   p.P = a.P;
   p.fused = a.fused;
+  p.causal = pl->causal;
   p.scale_log2 = a.scale * 1.4426950408889634f;
 
   // Non-empty segments, longest first.  The segment that ends at N also

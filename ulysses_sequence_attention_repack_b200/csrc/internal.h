@@ -21,6 +21,7 @@ struct ulysses_plan_s {
   int64_t token_stride, plane_stride;   // elements, sequence-sharded input
   int32_t plane_chunk;
   int32_t num_seqs;
+  int32_t causal;                       // attention sees keys m <= n only
   ulysses::Segment segs[ULYSSES_MAX_SEQS];
   int32_t device;                       // device the plan's scratch lives on (-1: none)
   unsigned int* dev_err;                // device error word (16 bytes allocated)

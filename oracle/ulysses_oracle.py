@@ -307,3 +307,68 @@ def attention_flops(N: int, H: int, D: int, cu_seqlens=None, causal: bool = Fals
 def softmax_scale(D: int) -> float:
     """1/sqrt(D): the scale of the Ulysses layer (1/sqrt(128) for D = 128)."""
     return 1.0 / math.sqrt(D)
+
+
+# ---------------------------------------------------------------------------
+# QKV prologue (per-head RMSNorm + partial rotate-half RoPE), fused before the
+# repack.  Source: "hao-ai-lab FastVideo, compare aryan/h3-nvfp4-stack-speedups
+# ...main", fastvideo/models/dits/minimax_h3_fusions/mk/qkv_prologue.py (module
+# docstring and kernel): per 128-wide (token, head) row of Q and of K,
+#   y = x / sqrt(mean(x^2) + eps) * w        (eps = 1e-5, w the per-channel norm weight)
+#   y'[i] = y[i] cos[i] + rot(y)[i] sin[i]   for i < rotary_dim, where
+#   rot(y)[i] = -y[i + rotary_dim/2] (i < rotary_dim/2), y[i - rotary_dim/2] otherwise,
+#   channels i >= rotary_dim unchanged; V (and any further plane) copied verbatim.
+# cos / sin are per-token tables [S, rotary_dim].
+# ---------------------------------------------------------------------------
+
+PROLOGUE_EPS = 1e-5
+
+
+def rms_norm_rows(x: np.ndarray, w: np.ndarray, eps: float = PROLOGUE_EPS) -> np.ndarray:
+    """RMSNorm over the last axis in fp64: x / sqrt(mean(x^2) + eps) * w."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * np.asarray(w, dtype=np.float64)
+
+
+def rope_rotate_half(y: np.ndarray, cos: np.ndarray, sin: np.ndarray, rotary_dim: int) -> np.ndarray:
+    """Partial rotate-half RoPE on the first rotary_dim channels of the last axis.
+
+    y: [..., D]; cos, sin: broadcastable to [..., rotary_dim].
+    """
+    y = np.asarray(y, dtype=np.float64)
+    half = rotary_dim // 2
+    out = y.copy()
+    a, b = y[..., :half], y[..., half:rotary_dim]
+    c = np.asarray(cos, dtype=np.float64)
+    s = np.asarray(sin, dtype=np.float64)
+    out[..., :half] = a * c[..., :half] - b * s[..., :half]
+    out[..., half:rotary_dim] = b * c[..., half:rotary_dim] + a * s[..., half:rotary_dim]
+    return out
+
+
+def qkv_prologue(S: np.ndarray, wq: np.ndarray, wk: np.ndarray, cos: np.ndarray, sin: np.ndarray,
+                 rotary_dim: int, eps: float = PROLOGUE_EPS) -> np.ndarray:
+    """The prologue on the sequence-sharded pack, in fp64.
+
+    S: ``[Np, C, H, D]`` uint16 bf16 bits (planes Q, K, V[, G]); wq, wk: ``[D]``
+    bf16 bits; cos, sin: ``[Np, rotary_dim]`` bf16 bits.  Returns fp64
+    ``[Np, C, H, D]``: planes 0 and 1 normalised and rotated, the others the
+    exact input values.
+    """
+    x = bf16_bits_to_f64(S).reshape(S.shape)
+    c = bf16_bits_to_f64(cos).reshape(cos.shape)[:, None, :]       # [Np, 1, rd] broadcast over heads
+    s = bf16_bits_to_f64(sin).reshape(sin.shape)[:, None, :]
+    out = x.copy()
+    for plane, w in ((0, wq), (1, wk)):
+        y = rms_norm_rows(x[:, plane], bf16_bits_to_f64(w), eps)
+        out[:, plane] = rope_rotate_half(y, c, s, rotary_dim)
+    return out
+
+
+def prologue_repack_fwd(S: np.ndarray, P: int, wq, wk, cos, sin, rotary_dim: int,
+                        eps: float = PROLOGUE_EPS) -> np.ndarray:
+    """Prologue, then the mode-0 index map: fp64 ``[P, C, Np, Hl, D]``."""
+    y = qkv_prologue(S, wq, wk, cos, sin, rotary_dim, eps)
+    Np, C, H, D = y.shape
+    Nl, Hl = Np // P, H // P
+    return np.ascontiguousarray(y.reshape(P, Nl, C, P, Hl, D).transpose(3, 2, 0, 1, 4, 5)).reshape(P, C, Np, Hl, D)

@@ -328,3 +328,63 @@ def test_causal_last_row_equals_non_causal_last_row():
 def test_causal_flop_count():
     assert orc.attention_flops(4, 1, 1, causal=True) == 4 * (1 + 2 + 3 + 4)
     assert orc.attention_flops(6, 2, 8, [0, 2, 6], causal=True) == 4 * 2 * 8 * ((1 + 2) + (1 + 2 + 3 + 4))
+
+
+# ---------------------------------------------------------------- QKV prologue (RMSNorm + partial RoPE)
+
+def test_rms_norm_closed_forms():
+    # a constant row c: x / sqrt(c^2 + eps) -> c / sqrt(c^2 + eps) in every channel
+    x = np.full((1, 128), 3.0)
+    y = orc.rms_norm_rows(x, np.ones(128), 1e-5)
+    assert np.allclose(y, 3.0 / math.sqrt(9.0 + 1e-5), rtol=0, atol=1e-15)
+    # the weight scales channel by channel; the output's rms is 1 (up to eps) for unit weight
+    rng = np.random.default_rng(50)
+    x = rng.standard_normal((7, 128)) * 5
+    y = orc.rms_norm_rows(x, np.ones(128), 0.0)
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, rtol=0, atol=1e-13)
+    w = rng.standard_normal(128)
+    assert np.allclose(orc.rms_norm_rows(x, w, 0.0), y * w, rtol=0, atol=1e-13)
+
+
+def test_rope_identity_quarter_turn_and_pair_norms():
+    rng = np.random.default_rng(51)
+    y = rng.standard_normal((5, 128))
+    rd = 96
+    one, zero = np.ones((5, rd)), np.zeros((5, rd))
+    assert np.array_equal(orc.rope_rotate_half(y, one, zero, rd), y)
+    # cos 0, sin 1: a quarter turn of every (i, i + 48) pair
+    q = orc.rope_rotate_half(y, zero, one, rd)
+    assert np.array_equal(q[:, :48], -y[:, 48:96]) and np.array_equal(q[:, 48:96], y[:, :48])
+    assert np.array_equal(q[:, 96:], y[:, 96:])        # channels past rotary_dim untouched
+    # any angle (same angle for i and i + 48) keeps each pair's length
+    th = rng.uniform(-3, 3, (5, 48))
+    c = np.concatenate([np.cos(th), np.cos(th)], axis=1)
+    s = np.concatenate([np.sin(th), np.sin(th)], axis=1)
+    r = orc.rope_rotate_half(y, c, s, rd)
+    assert np.allclose(r[:, :48] ** 2 + r[:, 48:96] ** 2, y[:, :48] ** 2 + y[:, 48:96] ** 2, rtol=0, atol=1e-12)
+    # rotating by th then by -th restores the input
+    back = orc.rope_rotate_half(r, c, -s, rd)
+    assert np.allclose(back, y, rtol=0, atol=1e-12)
+
+
+def test_prologue_then_repack_commutes_and_copies_v():
+    rng = np.random.default_rng(52)
+    P, N, C, H, D, rd = 2, 6, 4, 4, 128, 96
+    S = _bf16_normal(rng, (N, C, H, D))
+    wq, wk = _bf16_normal(rng, (D,)), _bf16_normal(rng, (D,))
+    cos, sin = _bf16_normal(rng, (N, rd)), _bf16_normal(rng, (N, rd))
+    T = orc.prologue_repack_fwd(S, P, wq, wk, cos, sin, rd)
+    # equals repack of the prologue output (per-row ops commute with the index map)
+    y = orc.qkv_prologue(S, wq, wk, cos, sin, rd)
+    assert np.array_equal(orc.repack_fwd(orc.f64_to_bf16_bits(y), P), orc.f64_to_bf16_bits(T))
+    # planes 2 and 3 are the input, exactly
+    assert np.array_equal(T[:, 2:], orc.bf16_bits_to_f64(orc.repack_fwd(S, P)[:, 2:]).reshape(T[:, 2:].shape))
+    # head-by-head against a direct per-row formula for one element
+    n, h = 3, 2
+    x = orc.bf16_bits_to_f64(S[n, 1, h])
+    yk = x / math.sqrt(np.mean(x * x) + 1e-5) * orc.bf16_bits_to_f64(wk)
+    cc, ss = orc.bf16_bits_to_f64(cos[n]), orc.bf16_bits_to_f64(sin[n])
+    i = 10
+    want = yk[i] * cc[i] - yk[i + 48] * ss[i]
+    r, j = h // (H // P), h % (H // P)
+    assert abs(T[r, 1, n, j, i] - want) < 1e-12

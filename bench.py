@@ -199,6 +199,26 @@ def run_ours(args, rank, world, local_rank):
     if U.ulysses_last_device_error(plan) != 0:
         raise RuntimeError("a kernel reported a device error during the timed region")
 
+    # step 1 with the QKV prologue fused in (RMSNorm + partial RoPE on Q and K,
+    # rotary_dim 96 as in the pages), timed on the same input
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 500)
+    wq = torch.randn(128, generator=g, device=dev).to(torch.bfloat16)
+    wk = torch.randn(128, generator=g, device=dev).to(torch.bfloat16)
+    ang = torch.rand((Np, 48), generator=g, device=dev) * 6.2832
+    cos_t = torch.cat([torch.cos(ang), torch.cos(ang)], 1).to(torch.bfloat16).contiguous()
+    sin_t = torch.cat([torch.sin(ang), torch.sin(ang)], 1).to(torch.bfloat16).contiguous()
+    for _ in range(3):
+        U.ulysses_prologue_repack_fwd(plan, S, T, wq, wk, cos_t, sin_t, 96, 1e-5, stream)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    npro = max(3, args.steps)
+    p0.record(stream)
+    for _ in range(npro):
+        U.ulysses_prologue_repack_fwd(plan, S, T, wq, wk, cos_t, sin_t, 96, 1e-5, stream)
+    p1.record(stream)
+    torch.cuda.synchronize()
+    prologue_ms = p0.elapsed_time(p1) / npro
+
     # fused variant (attention reads the sequence-sharded input directly)
     for _ in range(3):
         U.ulysses_layer_fwd(plan, S, OS, None, fused=1, stream=stream)
@@ -280,6 +300,8 @@ def run_ours(args, rank, world, local_rank):
                                                                        pk["bf16_tflops"]), 3),
                       "spec_2250": round(attn_tflops / SPEC_PEAKS["bf16_tflops"], 3)},
         "fused_layer_us": round(fused_ms * 1000, 2),
+        "prologue_repack_fwd_us": round(prologue_ms * 1000, 2),
+        "prologue_repack_fwd_gbs": round(rf_bytes / (prologue_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": round(attn_tflops, 1),
                      "peak": pk["bf16_tflops"], "peak_kind": f"{pk_kind} bf16 burst", "unit": "TFLOP/s",
                      "frac": round(attn_tflops / pk["bf16_tflops"], 3), "traffic": traffic,

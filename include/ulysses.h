@@ -138,6 +138,29 @@ size_t ulysses_workspace_bytes(const ulysses_plan_t* plan);
 int ulysses_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads, void* stream);
 
 /*
+ * Step 1 with the QKV prologue fused in: the mode-0 repack of
+ * ulysses_repack_fwd, where planes 0 (Q) and 1 (K) first get per-head RMSNorm
+ * and partial rotate-half RoPE, as mk/qkv_prologue.py does on the FastVideo
+ * layer page ("per-head QK RMSNorm + partial RoPE + stacked QKV output"):
+ *   y = x / sqrt(mean(x^2) + eps) * w                     (w: norm_q_weight / norm_k_weight)
+ *   y[i] = y[i] cos[n,i] - y[i + rd/2] sin[n,i]          for i <  rd/2
+ *   y[i] = y[i] cos[n,i] + y[i - rd/2] sin[n,i]          for rd/2 <= i < rd
+ * channels >= rd unchanged; planes >= 2 copied verbatim.  fp32 arithmetic,
+ * one bf16 rounding per output element.  It moves the same bytes as the plain
+ * repack (the prologue's own read and write of Q and K disappear).
+ *   norm_q_weight, norm_k_weight: device bf16 [D]
+ *   cos_table, sin_table:         device bf16 [Np, rotary_dim] (row n = token n;
+ *                                 may be NULL when rotary_dim = 0)
+ *   rotary_dim:                   0 .. D, a multiple of 16 (96 in the pages)
+ *   eps:                          > 0 (1e-5 in the pages)
+ * Errors: ARG (C < 2, bad eps/rotary_dim, overlap), ALIGN (any pointer not
+ * 16-byte aligned), UNSUPPORTED (rotary_dim % 16 != 0), CUDA.
+ */
+int ulysses_prologue_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads,
+                                const void* norm_q_weight, const void* norm_k_weight, const void* cos_table,
+                                const void* sin_table, int32_t rotary_dim, float eps, void* stream);
+
+/*
  * Step 3, Ulysses mode 1 (the inverse map): src_heads [P, planes, Np, Hl, D]
  * -> dst_seq.  With planes == C, dst_seq uses the plan's input strides (a full
  * round trip restores the input bit for bit).  With planes < C, dst_seq is a

@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     ulysses_layer_fwd_fused_noalloc,
     ulysses_layer_fwd_host,
     ulysses_plan,
+    ulysses_prologue_repack_fwd,
     ulysses_repack_bwd,
     ulysses_repack_fwd,
     ulysses_selftest_exp2_poly,

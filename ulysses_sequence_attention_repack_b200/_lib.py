@@ -33,7 +33,7 @@ EXPORTS = (
     "ulysses_plan_window_bytes_per_plane", "ulysses_workspace_bytes", "ulysses_repack_fwd",
     "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
     "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
-    "ulysses_layer_fwd_fused_noalloc", "ulysses_selftest_wait_timeout",
+    "ulysses_layer_fwd_fused_noalloc", "ulysses_selftest_wait_timeout", "ulysses_prologue_repack_fwd",
 )
 
 
@@ -80,6 +80,8 @@ def load() -> ctypes.CDLL:
         lib.ulysses_workspace_bytes.restype = sz
         lib.ulysses_repack_fwd.argtypes = [vp, vp, vp, vp]
         lib.ulysses_repack_fwd.restype = ctypes.c_int
+        lib.ulysses_prologue_repack_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp]
+        lib.ulysses_prologue_repack_fwd.restype = ctypes.c_int
         lib.ulysses_repack_bwd.argtypes = [vp, vp, vp, i32, vp]
         lib.ulysses_repack_bwd.restype = ctypes.c_int
         lib.ulysses_attn_fwd.argtypes = [vp, vp, vp, ctypes.c_float, vp]
@@ -198,6 +200,13 @@ def ulysses_plan(N: int, H: int, D: int, P: int, planes: int, token_stride: int 
 def ulysses_repack_fwd(plan: Plan, src_seq, dst_heads, stream=None) -> None:
     _check(load().ulysses_repack_fwd(plan.handle, _ptr(src_seq), _ptr(dst_heads), _stream(stream)),
            "ulysses_repack_fwd")
+
+
+def ulysses_prologue_repack_fwd(plan: Plan, src_seq, dst_heads, norm_q_weight, norm_k_weight, cos, sin,
+                                rotary_dim: int, eps: float = 1e-5, stream=None) -> None:
+    _check(load().ulysses_prologue_repack_fwd(plan.handle, _ptr(src_seq), _ptr(dst_heads), _ptr(norm_q_weight),
+                                              _ptr(norm_k_weight), _ptr(cos), _ptr(sin), int(rotary_dim),
+                                              float(eps), _stream(stream)), "ulysses_prologue_repack_fwd")
 
 
 def ulysses_repack_bwd(plan: Plan, src_heads, dst_seq, planes: int, stream=None) -> None:

@@ -265,6 +265,34 @@ int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* 
   return repack_bwd_impl(plan, src_heads, dst_seq, planes, static_cast<cudaStream_t>(stream));
 }
 
+int ulysses_prologue_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads,
+                                const void* norm_q_weight, const void* norm_k_weight, const void* cos_table,
+                                const void* sin_table, int32_t rotary_dim, float eps, void* stream) {
+  if (!plan || !src_seq || !dst_heads || !norm_q_weight || !norm_k_weight) return ULYSSES_ERR_ARG;
+  if (plan->C < 2 || !(eps > 0.f) || !std::isfinite(eps)) return ULYSSES_ERR_ARG;
+  if (rotary_dim < 0 || rotary_dim > plan->D) return ULYSSES_ERR_ARG;
+  if (rotary_dim % 16) return ULYSSES_ERR_UNSUPPORTED;
+  if (rotary_dim > 0 && (!cos_table || !sin_table)) return ULYSSES_ERR_ARG;
+  const void* ptrs[] = {src_seq, dst_heads, norm_q_weight, norm_k_weight};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return ULYSSES_ERR_ALIGN;
+  if (rotary_dim > 0 && (!aligned16(cos_table) || !aligned16(sin_table))) return ULYSSES_ERR_ALIGN;
+  if (overlap(src_seq, seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride), dst_heads,
+              heads_bytes(plan, plan->C)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int32_t c0 = 0; c0 < plan->C; c0 += plan->plane_chunk) {
+    const int32_t cc = std::min(plan->plane_chunk, plan->C - c0);
+    s = status_of(ulysses::launch_prologue_repack(src_seq, dst_heads, norm_q_weight, norm_k_weight, cos_table,
+                                                  sin_table, rotary_dim, eps, plan->Np, plan->H, plan->P, plan->C,
+                                                  c0, cc, plan->token_stride, plan->plane_stride, st));
+    if (s != ULYSSES_OK) return s;
+  }
+  return ULYSSES_OK;
+}
+
 int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, float softmax_scale,
                      void* stream) {
   if (!plan || !qkv_heads || !out_heads) return ULYSSES_ERR_ARG;

@@ -36,6 +36,13 @@ namespace ulysses {
 cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
                           int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream);
 
+// Prologue (per-head RMSNorm + partial RoPE on planes 0 and 1) fused with one
+// mode-0 repack launch over planes [c0, c0 + cc).
+cudaError_t launch_prologue_repack(const void* src, void* dst, const void* wq, const void* wk, const void* cos,
+                                   const void* sin, int32_t rd, float eps, int64_t Np, int32_t H, int32_t P,
+                                   int32_t Ctot, int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
+                                   cudaStream_t stream);
+
 // Attention launch description (filled by api.cpp).
 struct AttnLaunch {
   const void* base;        // Q/K/V source buffer

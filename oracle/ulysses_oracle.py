@@ -372,3 +372,74 @@ def prologue_repack_fwd(S: np.ndarray, P: int, wq, wk, cos, sin, rotary_dim: int
     Np, C, H, D = y.shape
     Nl, Hl = Np // P, H // P
     return np.ascontiguousarray(y.reshape(P, Nl, C, P, Hl, D).transpose(3, 2, 0, 1, 4, 5)).reshape(P, C, Np, Hl, D)
+
+
+# ---------------------------------------------------------------------------
+# Attention backward (the gradient the Ulysses transport carries back under
+# the forward's plan: _FusedUlyssesA2A.backward runs the inverse map on the
+# incoming gradient).  Written from the definition O = softmax(s Q K^T) V:
+#   P = softmax(s Q K^T), dV = P^T dO, dP = dO V^T,
+#   dS = P o (dP - rowsum(dP o P)),  dQ = s dS K,  dK = s dS^T Q.
+# rowsum(dP o P) equals rowsum(dO o O) (both are sum_m P_nm (dO_n . V_m)).
+# ---------------------------------------------------------------------------
+
+def attention_rows_bwd(q, k, v, do, scale: float, causal_offset: int | None = None):
+    """fp64 gradients of O = softmax(scale q k^T) v for query rows q [R, D].
+
+    With causal_offset = a, query row i (global index a + i... relative to the
+    key block start) sees keys 0..i only.  Returns (dq [R, D], dk [M, D], dv [M, D]).
+    """
+    q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
+    z = scale * (q @ k.T)
+    if causal_offset is not None:
+        R, M = z.shape
+        mask = np.arange(M)[None, :] > (np.arange(R)[:, None] + causal_offset)
+        z = np.where(mask, -np.inf, z)
+    z = z - z.max(axis=1, keepdims=True)
+    p = np.exp(z)
+    p /= p.sum(axis=1, keepdims=True)
+    dv = p.T @ do
+    dp = do @ v.T
+    ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+def attention_heads_bwd(T: np.ndarray, dO: np.ndarray, N: int, scale: float, cu_seqlens=None,
+                        causal: bool = False) -> np.ndarray:
+    """Gradients of step two for every head-sharded slab.
+
+    T: head-sharded ``[P, C, Np, Hl, D]`` uint16 (Q, K, V planes); dO: fp64 or
+    uint16 ``[P, Np, Hl, D]``.  Returns fp64 ``[P, 3, Np, Hl, D]`` (dQ, dK, dV);
+    pad rows and the gate plane get no gradient (zeros).
+    """
+    P, C, Np, Hl, D = T.shape
+    g = dO if dO.dtype != np.uint16 else bf16_bits_to_f64(dO)
+    out = np.zeros((P, 3, Np, Hl, D), dtype=np.float64)
+    for r in range(P):
+        for j in range(Hl):
+            for a, b in segments_from_cu_seqlens(cu_seqlens, N):
+                if b <= a:
+                    continue
+                q = bf16_bits_to_f64(T[r, 0, a:b, j])
+                k = bf16_bits_to_f64(T[r, 1, a:b, j])
+                v = bf16_bits_to_f64(T[r, 2, a:b, j])
+                dq, dk, dv = attention_rows_bwd(q, k, v, g[r, a:b, j], scale, 0 if causal else None)
+                out[r, 0, a:b, j], out[r, 1, a:b, j], out[r, 2, a:b, j] = dq, dk, dv
+    return out
+
+
+def layer_bwd(S: np.ndarray, dOut: np.ndarray, P: int, N: int, scale: float, cu_seqlens=None,
+              causal: bool = False) -> np.ndarray:
+    """Backward of the whole layer: dOut ``[Np, H, D]`` -> d(S) ``[Np, 3, H, D]`` fp64.
+
+    Mode 0 on the output gradient, attention backward per slab, mode 1 on the
+    three input gradients (the transport's backward runs the inverse map).
+    """
+    T = repack_fwd(S, P)
+    Np, H, D = dOut.shape
+    g = dOut if dOut.dtype != np.uint16 else bf16_bits_to_f64(dOut)
+    dO_T = np.ascontiguousarray(g.reshape(P, Np // P, 1, P, H // P, D).transpose(3, 2, 0, 1, 4, 5)).reshape(
+        P, Np, H // P, D)
+    dT = attention_heads_bwd(T, dO_T, N, scale, cu_seqlens, causal)
+    return np.ascontiguousarray(dT.reshape(P, 3, P, Np // P, H // P, D).transpose(2, 3, 1, 0, 4, 5)).reshape(
+        Np, 3, H, D)

@@ -388,3 +388,65 @@ def test_prologue_then_repack_commutes_and_copies_v():
     want = yk[i] * cc[i] - yk[i + 48] * ss[i]
     r, j = h // (H // P), h % (H // P)
     assert abs(T[r, 1, n, j, i] - want) < 1e-12
+
+
+# ---------------------------------------------------------------- attention backward
+
+def _loss(q, k, v, g, scale, causal):
+    z = scale * (q @ k.T)
+    if causal:
+        z = np.where(np.arange(k.shape[0])[None, :] > np.arange(q.shape[0])[:, None], -np.inf, z)
+    z = z - z.max(axis=1, keepdims=True)
+    p = np.exp(z)
+    p /= p.sum(axis=1, keepdims=True)
+    return float(np.sum((p @ v) * g))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_backward_matches_finite_differences(causal):
+    # central differences of L = sum(O * G) pin every gradient independently of the formulas
+    rng = np.random.default_rng(60 + causal)
+    R, D = 5, 6
+    q, k, v, g = (rng.standard_normal((R, D)) for _ in range(4))
+    dq, dk, dv = orc.attention_rows_bwd(q, k, v, g, 0.7, 0 if causal else None)
+    h = 1e-6
+    for X, dX in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            old = X[idx]
+            X[idx] = old + h
+            lp = _loss(q, k, v, g, 0.7, causal)
+            X[idx] = old - h
+            lm = _loss(q, k, v, g, 0.7, causal)
+            X[idx] = old
+            num[idx] = (lp - lm) / (2 * h)
+        assert np.allclose(dX, num, rtol=1e-6, atol=1e-8), np.abs(dX - num).max()
+
+
+def test_backward_row_term_identity():
+    # rowsum(dP o P) == rowsum(dO o O)
+    rng = np.random.default_rng(62)
+    q, k, v, g = (rng.standard_normal((7, 8)) for _ in range(4))
+    z = 0.5 * q @ k.T
+    p = np.exp(z - z.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    assert np.allclose(((g @ v.T) * p).sum(1), (g * (p @ v)).sum(1), rtol=0, atol=1e-12)
+
+
+def test_layer_backward_is_transposed_repack_of_head_gradients():
+    # sum over all gradients of the layer equals the per-head plain MHA gradients, regrouped
+    rng = np.random.default_rng(63)
+    P, N, H, D = 2, 6, 4, 8
+    S = _bf16_normal(rng, (N, 3, H, D))
+    G = rng.standard_normal((N, H, D))
+    dS = orc.layer_bwd(S, G, P, N, 0.4)
+    for h in range(H):
+        q, k, v = (orc.bf16_bits_to_f64(S[:, c, h]) for c in range(3))
+        dq, dk, dv = orc.attention_rows_bwd(q, k, v, G[:, h], 0.4)
+        assert np.allclose(dS[:, 0, h], dq, atol=1e-12) and np.allclose(dS[:, 1, h], dk, atol=1e-12)
+        assert np.allclose(dS[:, 2, h], dv, atol=1e-12)
+    # varlen: cross-segment gradients vanish
+    dS2 = orc.layer_bwd(S, G, P, N, 0.4, cu_seqlens=[0, 3, 6])
+    q, k, v = (orc.bf16_bits_to_f64(S[:3, c, 0]) for c in range(3))
+    dq, dk, dv = orc.attention_rows_bwd(q, k, v, G[:3, 0], 0.4)
+    assert np.allclose(dS2[:3, 1, 0], dk, atol=1e-12)

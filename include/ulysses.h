@@ -182,6 +182,55 @@ int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* 
 int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, float softmax_scale,
                      void* stream);
 
+/* ---------------------------------------------------------------- training
+ * The gradient of the layer.  The FastVideo transport carries gradients back
+ * through the inverse map under the forward's plan (_FusedUlyssesA2A.backward
+ * in ulysses_a2a.py); attention's own gradient is that of
+ * O = softmax(s Q K^T) V:  dV = P^T dO,  dS = P o (dO V^T - rowsum(dO o O)),
+ * dQ = s dS K,  dK = s dS^T Q.
+ */
+
+/* Bytes of the log-sum-exp buffer: P*Hl rows of lse_row_stride floats
+ * (Np rounded up to 4, plus 128). */
+size_t ulysses_lse_bytes(const ulysses_plan_t* plan);
+
+/*
+ * ulysses_attn_fwd that also writes, per (rank, local head, query row n),
+ * lse[(r*Hl + j) * stride + n] = m + log2(l): the row's log-sum-exp of
+ * s*log2(e)*Q K^T in base 2 (device fp32, ulysses_lse_bytes()).  Errors: as
+ * ulysses_attn_fwd.
+ */
+int ulysses_attn_fwd_lse(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, void* lse,
+                         float softmax_scale, void* stream);
+
+/* Workspace of ulysses_attn_bwd (the row terms rowsum(dO o O)). */
+size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan);
+
+/*
+ * dqkv_heads [P, 3, Np, Hl, D] = (dQ, dK, dV) for the attention step, given
+ * qkv_heads T [P, C, Np, Hl, D], its output out_heads O_T [P, Np, Hl, D], the
+ * output gradient dout_heads [P, Np, Hl, D] and the forward's lse.  Honors the
+ * plan's segments and causal flag; pad rows get zero gradients.  fp32
+ * accumulation, bf16 output.  Two passes over the keys and the queries; no
+ * atomics, deterministic.  Errors: ARG, ALIGN, WORKSPACE, CUDA.
+ */
+int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads,
+                     const void* dout_heads, const void* lse, void* dqkv_heads, void* workspace,
+                     size_t workspace_bytes, float softmax_scale, void* stream);
+
+/* Workspace of ulysses_layer_bwd: dO_T, (dQ, dK, dV) head-sharded and the row terms. */
+size_t ulysses_layer_bwd_workspace_bytes(const ulysses_plan_t* plan);
+
+/*
+ * Backward of the unfused layer (softmax_scale 1/sqrt(D)): mode 0 on
+ * dout_seq [Np, H, D], ulysses_attn_bwd with the forward's saved qkv_heads,
+ * out_heads and lse, then mode 1 on (dQ, dK, dV) into planes 0..2 of dqkv_seq
+ * (the plan's input layout; planes >= 3 are not written -- attention does not
+ * use the gate).  Errors: ARG, ALIGN, WORKSPACE, CUDA.
+ */
+int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads, const void* lse,
+                      const void* dout_seq, void* dqkv_seq, void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * The whole layer with softmax_scale = 1/sqrt(D):  out_seq O_S [Np, H, D]
  * from qkv_seq (sequence-sharded, plan strides).

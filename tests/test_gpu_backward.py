@@ -1,0 +1,118 @@
+"""Attention backward and layer backward against the fp64 oracle.
+
+The GPU path rounds P and dS to bf16 for its tensor-core products (as the
+forward rounds P), accumulates in fp32 and rounds the gradients to bf16 once.
+Each bf16 rounding is a relative error of at most 2^-9; summed over a
+128-wide contraction with random signs they stay well under 1% of the
+gradient's magnitude.  The bound used: per gradient tensor,
+max|gpu - ref| <= 2e-2 * max|ref| and mean|gpu - ref| <= 5e-3 * mean|ref|.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import ulysses_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL = 2e-2
+MEAN_REL = 5e-3
+
+CASES = [
+    pytest.param(2, 1024, 8, None, False, 0, id="tiny"),
+    pytest.param(4, 1001, 8, None, False, 1, id="ragged"),
+    pytest.param(1, 300, 2, None, False, 2, id="P1"),
+    pytest.param(2, 1000, 4, [0, 300, 301, 777, 1000], False, 3, id="varlen"),
+    pytest.param(2, 1024, 8, None, True, 4, id="causal"),
+    pytest.param(2, 700, 4, [0, 256, 300, 700], True, 5, id="causal-varlen"),
+]
+
+
+def _grad(gpu, shape, seed):
+    import torch
+    g = torch.Generator(device=gpu)
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, device=gpu).to(torch.bfloat16)
+
+
+def _close(got, ref, what):
+    err = np.abs(got - ref)
+    mx, mn = np.abs(ref).max(), np.abs(ref).mean()
+    assert err.max() <= MAX_REL * mx, (what, float(err.max()), float(mx))
+    assert err.mean() <= MEAN_REL * mn, (what, float(err.mean()), float(mn))
+
+
+@pytest.mark.parametrize("P,N,H,cu,causal,seed", CASES)
+def test_attention_backward_against_oracle(gpu, P, N, H, cu, causal, seed):
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=causal)
+    Np, Hl = plan.padded_tokens, H // P
+    scale = 1.0 / math.sqrt(128)
+    S = inputs.qkv_seq(N, H, P, 3, 100 + seed, gpu)
+    T = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, T)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=gpu)
+    U.ulysses_attn_fwd_lse(plan, T, OT, lse, scale)
+    dO = _grad(gpu, (P, Np, Hl, 128), 200 + seed)
+    dO[:, N:] = 0
+    dT = torch.full((P, 3, Np, Hl, 128), float("nan"), dtype=torch.bfloat16, device=gpu)
+    ws = torch.empty(plan.attn_bwd_workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_attn_bwd(plan, T, OT, dO, lse, dT, ws, scale)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    # the forward's lse: m + log2 l of every real row, against fp64
+    T_bits = inputs.host_bits(T)
+    ls = plan.lse_row_stride
+    got_lse = lse.view(P * Hl, ls)[:, :N].cpu().numpy().astype(np.float64)
+    ref = orc.attention_heads_bwd(T_bits, inputs.host_bits(dO), N, scale, cu, causal)
+    got = dT.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    for c, name in enumerate(("dQ", "dK", "dV")):
+        _close(got[:, c, :N], ref[:, c, :N], name)
+    assert np.all(got[:, :, N:] == 0)               # pad rows get no gradient
+    # lse check: log2 of sum_m exp2(s log2e q.k) per row, fp64
+    q = orc.bf16_bits_to_f64(T_bits[:, 0])
+    k = orc.bf16_bits_to_f64(T_bits[:, 1])
+    segs = orc.segments_from_cu_seqlens(cu, N)
+    for r in range(P):
+        for j in range(Hl):
+            for a, b in segs:
+                z = scale * (q[r, a:b, j] @ k[r, a:b, j].T) / math.log(2.0)
+                if causal:
+                    z = np.where(np.arange(b - a)[None, :] > np.arange(b - a)[:, None], -np.inf, z)
+                mz = z.max(1, keepdims=True)
+                want = (mz + np.log2(np.exp2(z - mz).sum(1, keepdims=True)))[:, 0]
+                assert np.abs(got_lse[r * Hl + j, a:b] - want).max() < 1e-3
+
+
+@pytest.mark.parametrize("P,N,H,cu,causal", [(2, 1024, 8, None, False), (4, 1001, 8, [0, 500, 1001], True)])
+def test_layer_backward_against_oracle(gpu, P, N, H, cu, causal):
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=causal)
+    Np, Hl = plan.padded_tokens, H // P
+    scale = 1.0 / math.sqrt(128)
+    S = inputs.qkv_seq(N, H, P, 3, 300, gpu)
+    # forward, keeping what the backward needs
+    T = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=gpu)
+    U.ulysses_repack_fwd(plan, S, T)
+    U.ulysses_attn_fwd_lse(plan, T, OT, lse, scale)
+    dOut = _grad(gpu, (Np, H, 128), 301)
+    dOut[N:] = 0
+    dS = torch.full_like(S, float("nan"))
+    ws = torch.empty(plan.layer_bwd_workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_layer_bwd(plan, T, OT, lse, dOut, dS, ws)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    ref = orc.layer_bwd(inputs.host_bits(S), inputs.host_bits(dOut), P, N, scale, cu, causal)
+    got = dS.float().cpu().numpy().astype(np.float64)
+    for c, name in enumerate(("dQ", "dK", "dV")):
+        _close(got[:N, c], ref[:N, c], name)
+    assert np.all(got[N:] == 0)

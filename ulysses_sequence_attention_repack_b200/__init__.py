@@ -13,8 +13,11 @@ from ._lib import (  # noqa: F401
     library_path,
     load,
     strerror,
+    ulysses_attn_bwd,
     ulysses_attn_fwd,
+    ulysses_attn_fwd_lse,
     ulysses_last_device_error,
+    ulysses_layer_bwd,
     ulysses_layer_fwd,
     ulysses_layer_fwd_fused_noalloc,
     ulysses_layer_fwd_host,

@@ -34,6 +34,8 @@ EXPORTS = (
     "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
     "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
     "ulysses_layer_fwd_fused_noalloc", "ulysses_selftest_wait_timeout", "ulysses_prologue_repack_fwd",
+    "ulysses_lse_bytes", "ulysses_attn_fwd_lse", "ulysses_attn_bwd_workspace_bytes", "ulysses_attn_bwd",
+    "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd",
 )
 
 
@@ -82,6 +84,18 @@ def load() -> ctypes.CDLL:
         lib.ulysses_repack_fwd.restype = ctypes.c_int
         lib.ulysses_prologue_repack_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp]
         lib.ulysses_prologue_repack_fwd.restype = ctypes.c_int
+        lib.ulysses_lse_bytes.argtypes = [vp]
+        lib.ulysses_lse_bytes.restype = sz
+        lib.ulysses_attn_fwd_lse.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp]
+        lib.ulysses_attn_fwd_lse.restype = ctypes.c_int
+        lib.ulysses_attn_bwd_workspace_bytes.argtypes = [vp]
+        lib.ulysses_attn_bwd_workspace_bytes.restype = sz
+        lib.ulysses_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, ctypes.c_float, vp]
+        lib.ulysses_attn_bwd.restype = ctypes.c_int
+        lib.ulysses_layer_bwd_workspace_bytes.argtypes = [vp]
+        lib.ulysses_layer_bwd_workspace_bytes.restype = sz
+        lib.ulysses_layer_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.ulysses_layer_bwd.restype = ctypes.c_int
         lib.ulysses_repack_bwd.argtypes = [vp, vp, vp, i32, vp]
         lib.ulysses_repack_bwd.restype = ctypes.c_int
         lib.ulysses_attn_fwd.argtypes = [vp, vp, vp, ctypes.c_float, vp]
@@ -164,6 +178,23 @@ class Plan:
     def workspace_bytes(self) -> int:
         return load().ulysses_workspace_bytes(self.handle)
 
+    @property
+    def lse_bytes(self) -> int:
+        return load().ulysses_lse_bytes(self.handle)
+
+    @property
+    def lse_row_stride(self) -> int:
+        """Floats between the lse rows of consecutive (rank, local head) pairs."""
+        return self.lse_bytes // 4 // self.H
+
+    @property
+    def attn_bwd_workspace_bytes(self) -> int:
+        return load().ulysses_attn_bwd_workspace_bytes(self.handle)
+
+    @property
+    def layer_bwd_workspace_bytes(self) -> int:
+        return load().ulysses_layer_bwd_workspace_bytes(self.handle)
+
     def destroy(self) -> None:
         if self._h:
             load().ulysses_plan_destroy(self._h)
@@ -207,6 +238,29 @@ def ulysses_prologue_repack_fwd(plan: Plan, src_seq, dst_heads, norm_q_weight, n
     _check(load().ulysses_prologue_repack_fwd(plan.handle, _ptr(src_seq), _ptr(dst_heads), _ptr(norm_q_weight),
                                               _ptr(norm_k_weight), _ptr(cos), _ptr(sin), int(rotary_dim),
                                               float(eps), _stream(stream)), "ulysses_prologue_repack_fwd")
+
+
+def ulysses_attn_fwd_lse(plan: Plan, qkv_heads, out_heads, lse, softmax_scale: float, stream=None) -> None:
+    _check(load().ulysses_attn_fwd_lse(plan.handle, _ptr(qkv_heads), _ptr(out_heads), _ptr(lse),
+                                       float(softmax_scale), _stream(stream)), "ulysses_attn_fwd_lse")
+
+
+def ulysses_attn_bwd(plan: Plan, qkv_heads, out_heads, dout_heads, lse, dqkv_heads, workspace,
+                     softmax_scale: float, workspace_bytes: int | None = None, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(load().ulysses_attn_bwd(plan.handle, _ptr(qkv_heads), _ptr(out_heads), _ptr(dout_heads), _ptr(lse),
+                                   _ptr(dqkv_heads), _ptr(workspace), int(workspace_bytes), float(softmax_scale),
+                                   _stream(stream)), "ulysses_attn_bwd")
+
+
+def ulysses_layer_bwd(plan: Plan, qkv_heads, out_heads, lse, dout_seq, dqkv_seq, workspace,
+                      workspace_bytes: int | None = None, stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(load().ulysses_layer_bwd(plan.handle, _ptr(qkv_heads), _ptr(out_heads), _ptr(lse), _ptr(dout_seq),
+                                    _ptr(dqkv_seq), _ptr(workspace), int(workspace_bytes), _stream(stream)),
+           "ulysses_layer_bwd")
 
 
 def ulysses_repack_bwd(plan: Plan, src_heads, dst_seq, planes: int, stream=None) -> None:

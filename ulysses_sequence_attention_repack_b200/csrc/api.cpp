@@ -86,7 +86,12 @@ int repack_bwd_impl(const ulysses_plan_t* p, const void* src, void* dst, int32_t
   return ULYSSES_OK;
 }
 
-int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, float scale, cudaStream_t st) {
+inline int64_t lse_bytes(const ulysses_plan_t* p) {
+  return static_cast<int64_t>(p->P) * p->Hl * ulysses::lse_row_stride(p->Np) * 4;
+}
+
+int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, float scale, cudaStream_t st,
+              float* lse = nullptr) {
   ulysses::AttnLaunch a;
   a.base = base;
   a.fused = fused;
@@ -109,6 +114,8 @@ int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, f
   a.o_stride_j = p->D;
   a.scale = scale;
   a.plan = p;
+  a.lse = lse;
+  a.lse_stride = ulysses::lse_row_stride(p->Np);
   return status_of(ulysses::launch_attn(a, st));
 }
 
@@ -302,6 +309,107 @@ int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* ou
   int s = device_ready(plan);
   if (s != ULYSSES_OK) return s;
   return attn_impl(plan, qkv_heads, 0, out_heads, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+size_t ulysses_lse_bytes(const ulysses_plan_t* plan) { return plan ? static_cast<size_t>(lse_bytes(plan)) : 0; }
+
+int ulysses_attn_fwd_lse(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, void* lse,
+                         float softmax_scale, void* stream) {
+  if (!plan || !qkv_heads || !out_heads || !lse) return ULYSSES_ERR_ARG;
+  if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
+  if (!aligned16(qkv_heads) || !aligned16(out_heads) || !aligned16(lse)) return ULYSSES_ERR_ALIGN;
+  if (overlap(qkv_heads, heads_bytes(plan, plan->C), out_heads, heads_bytes(plan, 1)) ||
+      overlap(lse, lse_bytes(plan), qkv_heads, heads_bytes(plan, plan->C)) ||
+      overlap(lse, lse_bytes(plan), out_heads, heads_bytes(plan, 1)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  return attn_impl(plan, qkv_heads, 0, out_heads, softmax_scale, static_cast<cudaStream_t>(stream),
+                   static_cast<float*>(lse));
+}
+
+size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan) {
+  return plan ? static_cast<size_t>(lse_bytes(plan)) : 0;
+}
+
+int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads,
+                     const void* dout_heads, const void* lse, void* dqkv_heads, void* workspace,
+                     size_t workspace_bytes, float softmax_scale, void* stream) {
+  if (!plan || !qkv_heads || !out_heads || !dout_heads || !lse || !dqkv_heads) return ULYSSES_ERR_ARG;
+  if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
+  if (!workspace || workspace_bytes < ulysses_attn_bwd_workspace_bytes(plan)) return ULYSSES_ERR_WORKSPACE;
+  const void* ptrs[] = {qkv_heads, out_heads, dout_heads, lse, dqkv_heads, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return ULYSSES_ERR_ALIGN;
+  const int64_t dq = heads_bytes(plan, 3), ws = lse_bytes(plan);
+  if (overlap(dqkv_heads, dq, qkv_heads, heads_bytes(plan, plan->C)) || overlap(dqkv_heads, dq, out_heads, heads_bytes(plan, 1)) ||
+      overlap(dqkv_heads, dq, dout_heads, heads_bytes(plan, 1)) || overlap(dqkv_heads, dq, lse, ws) ||
+      overlap(workspace, ws, dqkv_heads, dq) || overlap(workspace, ws, lse, ws))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  ulysses::AttnBwdLaunch a;
+  a.qkv = qkv_heads;
+  a.out = out_heads;
+  a.dout = dout_heads;
+  a.lse = static_cast<const float*>(lse);
+  a.delta = static_cast<float*>(workspace);
+  a.dqkv = dqkv_heads;
+  a.scale = softmax_scale;
+  a.plan = plan;
+  return status_of(ulysses::launch_attn_bwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t ulysses_layer_bwd_workspace_bytes(const ulysses_plan_t* plan) {
+  if (!plan) return 0;
+  return static_cast<size_t>(align_up(heads_bytes(plan, 1), 256) + align_up(heads_bytes(plan, 3), 256) +
+                             align_up(lse_bytes(plan), 256));
+}
+
+int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads, const void* lse,
+                      const void* dout_seq, void* dqkv_seq, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!plan || !qkv_heads || !out_heads || !lse || !dout_seq || !dqkv_seq) return ULYSSES_ERR_ARG;
+  if (plan->C < 3) return ULYSSES_ERR_ARG;
+  if (!workspace || workspace_bytes < ulysses_layer_bwd_workspace_bytes(plan)) return ULYSSES_ERR_WORKSPACE;
+  const void* ptrs[] = {qkv_heads, out_heads, lse, dout_seq, dqkv_seq, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return ULYSSES_ERR_ALIGN;
+  const int64_t ws = static_cast<int64_t>(ulysses_layer_bwd_workspace_bytes(plan));
+  const int64_t dseq = seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride);
+  if (overlap(workspace, ws, qkv_heads, heads_bytes(plan, plan->C)) || overlap(workspace, ws, out_heads, heads_bytes(plan, 1)) ||
+      overlap(workspace, ws, lse, lse_bytes(plan)) || overlap(workspace, ws, dout_seq, out_seq_bytes(plan)) ||
+      overlap(workspace, ws, dqkv_seq, dseq) || overlap(dqkv_seq, dseq, dout_seq, out_seq_bytes(plan)) ||
+      overlap(dqkv_seq, dseq, qkv_heads, heads_bytes(plan, plan->C)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* dOT = static_cast<uint8_t*>(workspace);
+  uint8_t* dT = dOT + align_up(heads_bytes(plan, 1), 256);
+  float* delta = reinterpret_cast<float*>(dT + align_up(heads_bytes(plan, 3), 256));
+  // mode 0 on the output gradient (one dense plane [Np, H, D])
+  const int64_t row = static_cast<int64_t>(plan->H) * plan->D;
+  s = status_of(ulysses::launch_repack(0, dout_seq, dOT, plan->Np, plan->H, plan->P, 1, 0, 1, row, row, st));
+  if (s != ULYSSES_OK) return s;
+  ulysses::AttnBwdLaunch a;
+  a.qkv = qkv_heads;
+  a.out = out_heads;
+  a.dout = dOT;
+  a.lse = static_cast<const float*>(lse);
+  a.delta = delta;
+  a.dqkv = dT;
+  a.scale = 1.0f / std::sqrt(static_cast<float>(plan->D));
+  a.plan = plan;
+  s = status_of(ulysses::launch_attn_bwd(a, st));
+  if (s != ULYSSES_OK) return s;
+  // mode 1 on dQ, dK, dV into planes 0..2 of the plan's input layout
+  for (int32_t c0 = 0; c0 < 3; c0 += plan->plane_chunk) {
+    const int32_t cc = std::min(plan->plane_chunk, 3 - c0);
+    s = status_of(ulysses::launch_repack(1, dT, dqkv_seq, plan->Np, plan->H, plan->P, 3, c0, cc, plan->token_stride,
+                                         plan->plane_stride, st));
+    if (s != ULYSSES_OK) return s;
+  }
+  return ULYSSES_OK;
 }
 
 int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,

@@ -113,6 +113,8 @@ struct SegDesc {
 
 struct AttnParams {
   __nv_bfloat16* out;
+  float* lse;                      // optional: log2-domain log-sum-exp per row (m + log2 l)
+  int64_t lse_stride;              // floats between (rank, head) rows of lse
   unsigned int* err;
   int64_t o_stride_r, o_stride_n, o_stride_j;
   int32_t N, Np;
@@ -479,6 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(BAR(B_OEMPTY0 + wg));
       const int n = w.q0 + wg * BM + row;
+      if (p.lse && n < sd.q_end && n < p.Np)
+        p.lse[(static_cast<int64_t>(w.r) * p.Hl + w.j) * p.lse_stride + n] = m_used + log2f(l);
       if (n < sd.q_end && n < p.Np) {
         uint4* dst = reinterpret_cast<uint4*>(p.out + w.r * p.o_stride_r + static_cast<int64_t>(n) * p.o_stride_n +
                                               w.j * p.o_stride_j);
@@ -563,6 +567,8 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
   p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
+  p.lse_stride = a.lse_stride;
   p.err = pl->dev_err;
   p.o_stride_r = a.o_stride_r;
   p.o_stride_n = a.o_stride_n;

@@ -54,8 +54,30 @@ struct AttnLaunch {
   int64_t o_stride_r, o_stride_n, o_stride_j;   // elements
   float scale;
   const ulysses_plan_t* plan;
+  float* lse = nullptr;          // optional log2-domain LSE output [P*Hl][lse_stride]
+  int64_t lse_stride = 0;
 };
 
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream);
+
+// Row stride (floats) of the LSE / D buffers of one (rank, local head): Np
+// rounded up to 4 plus 144, so the 132-float bulk copy the backward makes for
+// any 128-row block starting below Np (from the block start rounded down to
+// a multiple of 4, keeping the copy 16-byte aligned) stays inside the buffer.
+inline int64_t lse_row_stride(int64_t Np) { return (Np + 3) / 4 * 4 + 144; }
+
+// Attention backward launch description (filled by api.cpp).
+struct AttnBwdLaunch {
+  const void* qkv;      // head-sharded T [P, C, Np, Hl, D]
+  const void* out;      // O_T [P, Np, Hl, D]
+  const void* dout;     // dO_T [P, Np, Hl, D]
+  const float* lse;     // [P*Hl][lse_stride] from the forward
+  float* delta;         // workspace [P*Hl][lse_stride]: rowsum(dO o O)
+  void* dqkv;           // [P, 3, Np, Hl, D]
+  float scale;
+  const ulysses_plan_t* plan;
+};
+
+cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream);
 
 }  // namespace ulysses

@@ -219,6 +219,26 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     prologue_ms = p0.elapsed_time(p1) / npro
 
+    # training direction: forward with lse, then the attention backward
+    # (algorithmic FLOPs 2.5x the forward's: dV, dP, dQ, dK plus S recomputed)
+    lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=dev)
+    dO = torch.randn(OT.shape, generator=g, device=dev).to(torch.bfloat16)
+    dT = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
+    bws = torch.empty(plan.attn_bwd_workspace_bytes, dtype=torch.uint8, device=dev)
+    U.ulysses_attn_fwd_lse(plan, T, OT, lse, scale, stream)
+    for _ in range(2):
+        U.ulysses_attn_bwd(plan, T, OT, dO, lse, dT, bws, scale, stream=stream)
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nbw = max(3, args.steps // 3)
+    b0.record(stream)
+    for _ in range(nbw):
+        U.ulysses_attn_bwd(plan, T, OT, dO, lse, dT, bws, scale, stream=stream)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    bwd_ms = b0.elapsed_time(b1) / nbw
+    if U.ulysses_last_device_error(plan) != 0:
+        raise RuntimeError("a kernel reported a device error in the backward")
+
     # fused variant (attention reads the sequence-sharded input directly)
     for _ in range(3):
         U.ulysses_layer_fwd(plan, S, OS, None, fused=1, stream=stream)
@@ -300,6 +320,8 @@ def run_ours(args, rank, world, local_rank):
                                                                        pk["bf16_tflops"]), 3),
                       "spec_2250": round(attn_tflops / SPEC_PEAKS["bf16_tflops"], 3)},
         "fused_layer_us": round(fused_ms * 1000, 2),
+        "attn_bwd_us": round(bwd_ms * 1000, 2),
+        "attn_bwd_tflops": round(2.5 * flops / (bwd_ms * 1e-3) / 1e12, 1),
         "prologue_repack_fwd_us": round(prologue_ms * 1000, 2),
         "prologue_repack_fwd_gbs": round(rf_bytes / (prologue_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": round(attn_tflops, 1),

@@ -17,11 +17,11 @@
 //           P^T and dS^T (bf16, aliased over them), then
 //           dV += P^T dO and dK += dS^T Q with A read from TMEM;
 //   pass B (unit = 128 queries, loop over key blocks): S = Q K^T and
-//           dP = dO V^T, then dS, then dQ += dS K.
+//           dP = dO V^T, then dS (bf16, over dP), then dQ += dS K.
 // Both reuse the forward's machinery: TMA-fed 128B-swizzled tiles, grouped
-// tcgen05 MMAs issued by one thread, one thread per TMEM lane for the
-// elementwise step, bounded mbarrier waits.  Warps: 0-3 elementwise and
-// epilogue, 4 MMA issuer, 5 TMA producer.
+// tcgen05 MMAs issued by one thread, bounded mbarrier waits.  Warps: 0-7
+// elementwise and epilogue (two warpgroups, each one thread per TMEM lane and
+// 64 of the 128 columns), 8 MMA issuer, 9 TMA producer.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -36,9 +36,10 @@
 namespace ulysses {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kMmaWarp = 4;
-constexpr int kTmaWarp = 5;
+constexpr int kEwWarps = 8;                           // two warpgroups, 64 columns each
+constexpr int kThreads = 32 * (kEwWarps + 2);
+constexpr int kMmaWarp = kEwWarps;
+constexpr int kTmaWarp = kEwWarps + 1;
 constexpr int BT = 128;                               // rows per tile (keys or queries)
 constexpr int HD = 128;
 constexpr uint32_t kHalfBytes = BT * 64 * 2;          // 16 KB swizzled box
@@ -57,8 +58,8 @@ constexpr uint32_t kRowStageBytes = 2 * kRowFloats * 4;                // 1056
 constexpr uint32_t kOffRow = kOffX + kStages * 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffRow + kStages * kRowStageBytes;
 enum {
-  B_FFULL = 0, B_FEMPTY, B_XFULL0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_SFULL, B_PFULL, B_OFULL, B_OEMPTY, B_DONE,
-  B_COUNT
+  B_FFULL = 0, B_FEMPTY, B_XFULL0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_SFULL, B_DPFULL, B_PFULL, B_DSFULL, B_OFULL,
+  B_OEMPTY, B_DONE, B_COUNT
 };
 constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;
 constexpr uint32_t kOffAbort = kOffSlot + 4;
@@ -167,6 +168,59 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const int4* __restrict__
   }
 }
 
+// Elementwise step of one streamed block for one thread: its TMEM lane (a key
+// in pass A, a query in pass B) against the 64 columns of its warpgroup.
+//   P  = exp2(s log2e S - lse)             (0 where the pair is masked)
+// kMask: the block straddles a segment end or the causal diagonal.
+template <bool kPassA, bool kMask>
+__device__ __forceinline__ void p_block(const uint32_t (&sv)[2][32], float (&pr)[64], float sl2,
+                                        const float* lse_s, float lse_row, int col0, int my, int end, int causal) {
+  if (kPassA) {
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+      const f2 x = ffma2(f2{__uint_as_float(sv[e >> 5][e & 31]), __uint_as_float(sv[e >> 5][(e & 31) + 1])},
+                         f2{sl2, sl2}, f2{-lse_s[e], -lse_s[e + 1]});
+      pr[e] = ex2_approx(x.x);
+      pr[e + 1] = ex2_approx(x.y);
+    }
+  } else {
+    const f2 nl{-lse_row, -lse_row};
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+      const f2 x = ffma2(f2{__uint_as_float(sv[e >> 5][e & 31]), __uint_as_float(sv[e >> 5][(e & 31) + 1])},
+                         f2{sl2, sl2}, nl);
+      pr[e] = ex2_approx(x.x);
+      pr[e + 1] = ex2_approx(x.y);
+    }
+  }
+  if (kMask) {
+    const bool row_ok = my < end;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+      const int other = col0 + e;                      // query (pass A) or key (pass B) index
+      const bool valid = row_ok && other < end && (!causal || (kPassA ? other >= my : other <= my));
+      pr[e] = valid ? pr[e] : 0.f;
+    }
+  }
+}
+
+//   dS = P o (dP - D), packed to bf16 pairs (pk[h][k] holds columns 32h + 2k, 2k + 1)
+template <bool kPassA, bool kMask>
+__device__ __forceinline__ void ds_block(const uint32_t (&dv)[2][32], const float (&pr)[64], const float* dlt_s,
+                                         float d_row, uint32_t (&pk)[2][16]) {
+#pragma unroll
+  for (int e = 0; e < 64; e += 2) {
+    const f2 nd = kPassA ? f2{-dlt_s[e], -dlt_s[e + 1]} : f2{-d_row, -d_row};
+    const f2 t = fadd2(f2{__uint_as_float(dv[e >> 5][e & 31]), __uint_as_float(dv[e >> 5][(e & 31) + 1])}, nd);
+    f2 d = fmul2(f2{pr[e], pr[e + 1]}, t);
+    if (kMask) {   // D past the segment end may be anything: masked entries stay exactly 0
+      d.x = pr[e] == 0.f ? 0.f : d.x;
+      d.y = pr[e + 1] == 0.f ? 0.f : d.y;
+    }
+    pk[e >> 5][(e & 31) >> 1] = pack_bf16x2(d.x, d.y);
+  }
+}
+
 template <bool kPassA>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
@@ -191,9 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR(B_XEMPTY0 + s), 1);
     }
     mbar_init(BAR(B_SFULL), 1);
-    mbar_init(BAR(B_PFULL), BT);
+    mbar_init(BAR(B_DPFULL), 1);
+    mbar_init(BAR(B_PFULL), kEwWarps);      // one elected arrival per elementwise warp
+    mbar_init(BAR(B_DSFULL), kEwWarps);
     mbar_init(BAR(B_OFULL), 1);
-    mbar_init(BAR(B_OEMPTY), BT);
+    mbar_init(BAR(B_OEMPTY), kEwWarps);
     mbar_init(BAR(B_DONE), 1);
     fence_mbar_init();
   }
@@ -209,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
@@ -266,10 +323,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ tcgen05 issuer
+    // Per block i (pass A):  [P^T(i) ready] dV += P^T dO, S(i+1), [dS^T(i) ready] dK += dS^T Q, dP(i+1)
+    //           (pass B):  [S(i) read]      S(i+1),          [dS(i) ready]   dQ += dS K,   dP(i+1)
+    // so the next block's S is computed while the elementwise warps form dS.
+    // The bf16 operands P^T / dS come in two halves of 32 TMEM columns, one per
+    // elementwise warpgroup, at column offsets 0 and 64 of their region.
     if (lane == 0) {
       uint32_t xc = 0, uc = 0, pc = 0;
       bool ok = true;
       const uint64_t dF0 = desc_sw128(sbase + kOffF0, 16, 1024), dF1 = desc_sw128(sbase + kOffF1, 16, 1024);
+      auto xdesc = [&](uint32_t s, int t, uint32_t lbo) {
+        return desc_sw128(sbase + kOffX + s * 2 * kTileBytes + t * kTileBytes, lbo, 1024);
+      };
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
         UnitB w;
         if (!decode_b(p, u, w)) break;
@@ -277,43 +342,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         int first, count;
         stream_range<kPassA>(p, sd, w, first, count);
         if (!(ok = mbar_wait(BAR(B_FFULL), uc & 1, g))) break;
+        // the accumulators are free once the previous unit's epilogue has read them
+        if (uc > 0 && !(ok = mbar_wait(BAR(B_OEMPTY), (uc - 1) & 1, g))) break;
         tc_fence_after();
-        for (int i = 0; ok && i < count; ++i) {
+        if (count > 0) {
           const uint32_t s = xc % kStages;
-          const uint32_t x0 = sbase + kOffX + s * 2 * kTileBytes, x1 = x0 + kTileBytes;
           if (!(ok = mbar_wait(BAR(B_XFULL0 + s), (xc / kStages) & 1, g))) break;
           tc_fence_after();
           // pass A: S^T = K Q^T, dP^T = V dO^T;  pass B: S = Q K^T, dP = dO V^T
-          mma_ss_k128(tmem + kColA0, dF0, desc_sw128(x0, 16, 1024), kIdescSS, 0);
-          mma_ss_k128(tmem + kColA1, dF1, desc_sw128(x1, 16, 1024), kIdescSS, 0);
+          mma_ss_k128(tmem + kColA0, dF0, xdesc(s, 0, 16), kIdescSS, 0);
           mma_commit(BAR(B_SFULL));
-          if (i == 0 && uc > 0 && !(ok = mbar_wait(BAR(B_OEMPTY), (uc - 1) & 1, g))) break;
+          mma_ss_k128(tmem + kColA1, dF1, xdesc(s, 1, 16), kIdescSS, 0);
+          mma_commit(BAR(B_DPFULL));
+        }
+        for (int i = 0; ok && i < count; ++i) {
+          const uint32_t xi = xc + i, s = xi % kStages, sn = (xi + 1) % kStages;
+          const bool more = i + 1 < count;
           if (!(ok = mbar_wait(BAR(B_PFULL), pc & 1, g))) break;
-          ++pc;
           tc_fence_after();
-          if (kPassA) {
-            // dV += P^T dO, dK += dS^T Q (B operands read MN-major from the stage)
-            mma_ts_k128(tmem + kColAcc0, tmem + kColA0, desc_sw128(x1, kHalfBytes, 1024), kIdescTS, i > 0);
-            mma_ts_k128(tmem + kColAcc1, tmem + kColA1, desc_sw128(x0, kHalfBytes, 1024), kIdescTS, i > 0);
-          } else {
-            // dQ += dS K
-            mma_ts_k128(tmem + kColAcc0, tmem + kColA0, desc_sw128(x0, kHalfBytes, 1024), kIdescTS, i > 0);
+          if (kPassA) {   // dV += P^T dO (B: dO read MN-major from the stage)
+            mma_ts_k64(tmem + kColAcc0, tmem + kColA0, xdesc(s, 1, kHalfBytes), kIdescTS, i > 0);
+            mma_ts_k64(tmem + kColAcc0, tmem + kColA0 + 64, xdesc(s, 1, kHalfBytes) + 512, kIdescTS, 1);
           }
+          if (more) {     // S of the next block over A0 (in order after the MMAs that read it)
+            if (!(ok = mbar_wait(BAR(B_XFULL0 + sn), ((xi + 1) / kStages) & 1, g))) break;
+            tc_fence_after();
+            mma_ss_k128(tmem + kColA0, dF0, xdesc(sn, 0, 16), kIdescSS, 0);
+            mma_commit(BAR(B_SFULL));
+          }
+          if (!(ok = mbar_wait(BAR(B_DSFULL), pc & 1, g))) break;
+          tc_fence_after();
+          ++pc;
+          // pass A: dK += dS^T Q (B: Q MN-major);  pass B: dQ += dS K (B: K MN-major)
+          const uint32_t acc = kPassA ? kColAcc1 : kColAcc0;
+          mma_ts_k64(tmem + acc, tmem + kColA1, xdesc(s, 0, kHalfBytes), kIdescTS, i > 0);
+          mma_ts_k64(tmem + acc, tmem + kColA1 + 64, xdesc(s, 0, kHalfBytes) + 512, kIdescTS, 1);
           mma_commit(BAR(B_XEMPTY0 + s));
-          ++xc;
+          if (more) {     // dP of the next block over A1
+            mma_ss_k128(tmem + kColA1, dF1, xdesc(sn, 1, 16), kIdescSS, 0);
+            mma_commit(BAR(B_DPFULL));
+          }
         }
         if (!ok) break;
+        xc += count;
         mma_commit(BAR(B_OFULL));
         mma_commit(BAR(B_FEMPTY));
       }
       mma_commit(BAR(B_DONE));
       drain_wait_b(BAR(B_DONE), 0);
     }
-  } else if (warp < 4) {
+  } else if (warp < kEwWarps) {
     // ------------------------------------------------------------ elementwise + epilogue
-    const int row = threadIdx.x;                       // TMEM lane == row of the unit's tile
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tA0 = tmem + lane_base + kColA0, tA1 = tmem + lane_base + kColA1;
+    // Warp w owns TMEM lanes 32 (w % 4) .. +31 (one row of the unit's tile per
+    // thread) and, with its warpgroup w / 4, 64 of the 128 columns.
+    const int wg = warp >> 2;
+    const int row = 32 * (warp & 3) + lane;
+    const int c0 = 64 * wg;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const uint32_t tA0 = tmem + lane_base + kColA0 + c0, tA1 = tmem + lane_base + kColA1 + c0;
     const float sl2 = p.scale_log2;
     const float* srow = reinterpret_cast<const float*>(smem + kOffRow);
     uint32_t sc = 0, uc = 0, xc = 0;
@@ -322,6 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       UnitB w;
       if (!decode_b(p, u, w)) break;
       const SegB& sd = p.seg[w.seg];
+      const int end = sd.end;
       int first, count;
       stream_range<kPassA>(p, sd, w, first, count);
       const int my = w.row0 + row;                     // key (pass A) or query (pass B) index
@@ -337,79 +424,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int r0 = sd.start + (first + i) * BT;    // first streamed index of this block
         const uint32_t s = xc % kStages;
+        // pass A reads the block's lse / D rows, which arrive with the stage
+        if (kPassA && !(ok = mbar_wait_warp(BAR(B_XFULL0 + s), (xc / kStages) & 1, g))) break;
         ++xc;
-        // pass A: lse / D of the 128 streamed queries (the copy starts at r0 rounded down to 4)
-        const float* lse_s = srow + s * (kRowStageBytes / 4) + (r0 & 3);
+        // lse / D of the warpgroup's 64 streamed queries (the copy starts at r0 rounded down to 4)
+        const float* lse_s = srow + s * (kRowStageBytes / 4) + (r0 & 3) + c0;
         const float* dlt_s = lse_s + kRowFloats;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32], dv[32];
-          tmem_ld32(tA0 + 32 * c, sv);
-          tmem_ld32(tA1 + 32 * c, dv);
+        // the whole 128 x 128 block is inside the segment and off the causal diagonal
+        const bool full = w.row0 + BT <= end && r0 + BT <= end &&
+                          (!p.causal || (kPassA ? r0 > w.row0 : r0 < w.row0));
+        // phase 1 (S ready): P in fp32, kept for phase 2; pass A stores P^T (bf16) for dV += P^T dO
+        float pr[64];
+        {
+          uint32_t sv[2][32];
+          tmem_ld32(tA0, sv[0]);
+          tmem_ld32(tA0 + 32, sv[1]);
           tmem_wait_ld();
-          tmem_regs_ready(sv);
-          tmem_regs_ready(dv);
-          uint32_t pk_p[16], pk_ds[16];
+          tmem_regs_ready(sv[0]);
+          tmem_regs_ready(sv[1]);
+          if (full)
+            p_block<kPassA, false>(sv, pr, sl2, lse_s, lse_row, r0 + c0, my, end, p.causal);
+          else
+            p_block<kPassA, true>(sv, pr, sl2, lse_s, lse_row, r0 + c0, my, end, p.causal);
+        }
+        if (kPassA) {
+          uint32_t pk[2][16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2], ds[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int col = 32 * c + e + h;
-              const int other = r0 + col;              // query (pass A) or key (pass B) index
-              float lse_q, d_q;
-              bool valid;
-              if (kPassA) {
-                lse_q = lse_s[col];
-                d_q = dlt_s[col];
-                valid = other < sd.end && my < sd.end && (!p.causal || other >= my);
-              } else {
-                lse_q = lse_row;
-                d_q = d_row;
-                valid = other < sd.end && my < sd.end && (!p.causal || other <= my);
-              }
-              const float x = fmaf(__uint_as_float(sv[e + h]), sl2, -lse_q);
-              const float pe = ex2_approx(x);
-              pv[h] = valid ? pe : 0.f;
-              ds[h] = valid ? pe * (__uint_as_float(dv[e + h]) - d_q) : 0.f;
-            }
-            pk_p[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-            pk_ds[e >> 1] = pack_bf16x2(ds[0], ds[1]);
-          }
-          if (kPassA) {
-            tmem_st16(tA0 + 16 * c, pk_p);    // P^T over the first 64 columns of A0
-            tmem_st16(tA1 + 16 * c, pk_ds);   // dS^T over the first 64 columns of A1
-          } else {
-            tmem_st16(tA0 + 16 * c, pk_ds);   // dS over the first 64 columns of A0
-          }
+          for (int e = 0; e < 32; ++e) pk[e >> 4][e & 15] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+          tmem_st16(tA0, pk[0]);                       // P^T over columns c0 .. c0 + 31 of A0
+          tmem_st16(tA0 + 16, pk[1]);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_PFULL));     // pass B: S has been read
+        // phase 2 (dP ready): dS = P o (dP - D) over columns c0 .. c0 + 31 of A1
+        if (!(ok = mbar_wait_warp(BAR(B_DPFULL), (sc - 1) & 1, g))) break;
+        tc_fence_after();
+        {
+          uint32_t dv[2][32];
+          tmem_ld32(tA1, dv[0]);
+          tmem_ld32(tA1 + 32, dv[1]);
+          tmem_wait_ld();
+          tmem_regs_ready(dv[0]);
+          tmem_regs_ready(dv[1]);
+          uint32_t pk[2][16];
+          if (full)
+            ds_block<kPassA, false>(dv, pr, dlt_s, d_row, pk);
+          else
+            ds_block<kPassA, true>(dv, pr, dlt_s, d_row, pk);
+          tmem_st16(tA1, pk[0]);
+          tmem_st16(tA1 + 16, pk[1]);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(B_PFULL));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_DSFULL));
       }
       if (!ok) break;
-      // epilogue: accumulators -> bf16 rows of dQ / dK / dV (pad rows: zeros)
+      // epilogue: this warpgroup's 64 accumulator columns -> bf16 rows of dQ / dK / dV (pad rows: zeros)
       if (!(ok = mbar_wait_warp(BAR(B_OFULL), uc & 1, g))) break;
       tc_fence_after();
-      const bool live = count > 0 && my < sd.end;
+      const bool live = count > 0 && my < end;
       const bool write = my < sd.tile_end && my < p.Np;
       const int nacc = kPassA ? 2 : 1;
       for (int a = 0; a < nacc; ++a) {
         // pass A: acc0 = dV (plane 2), acc1 = dK (plane 1, times scale); pass B: acc0 = dQ (plane 0)
         const int plane = kPassA ? (a == 0 ? 2 : 1) : 0;
         const float f = (kPassA && a == 0) ? 1.0f : p.scale;
-        uint32_t ov[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + (a == 0 ? kColAcc0 : kColAcc1) + 32 * c, ov[c]);
+        uint32_t ov[2][32];
+        const uint32_t tacc = tmem + lane_base + (a == 0 ? kColAcc0 : kColAcc1) + c0;
+        tmem_ld32(tacc, ov[0]);
+        tmem_ld32(tacc + 32, ov[1]);
         tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_regs_ready(ov[c]);
+        tmem_regs_ready(ov[0]);
+        tmem_regs_ready(ov[1]);
         if (write) {
           uint4* dst = reinterpret_cast<uint4*>(
-              p.dqkv + ((((static_cast<int64_t>(w.r) * 3 + plane) * p.Np + my) * p.Hl + w.j) * HD));
+              p.dqkv + ((((static_cast<int64_t>(w.r) * 3 + plane) * p.Np + my) * p.Hl + w.j) * HD + c0));
           const float* o = reinterpret_cast<const float*>(&ov[0][0]);
 #pragma unroll
-          for (int v = 0; v < 16; ++v) {
+          for (int v = 0; v < 8; ++v) {
             uint4 q = make_uint4(0u, 0u, 0u, 0u);
             if (live) {
               q.x = pack_bf16x2(o[8 * v + 0] * f, o[8 * v + 1] * f);
@@ -422,7 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(BAR(B_OEMPTY));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_OEMPTY));
     }
   }
 

@@ -404,6 +404,42 @@ def attention_rows_bwd(q, k, v, do, scale: float, causal_offset: int | None = No
     return scale * (ds @ k), scale * (ds.T @ q), dv
 
 
+def attention_bwd_sampled(q, k, v, do, scale: float, q_rows, k_rows, causal: bool = False, block: int = 512):
+    """dQ at query rows ``q_rows`` and dK, dV at key rows ``k_rows`` of one
+    (head, segment) block, fp64, from the same definition as
+    ``attention_rows_bwd``: every query row's softmax row, dP row and
+    rowsum(dP o P) are formed in full.  Query rows are visited ``block`` at a
+    time only to bound memory (each row's terms are independent of the
+    others).  Causal: query n sees keys m <= n (indices within the segment).
+    Returns (dq [len(q_rows), D], dk [len(k_rows), D], dv [len(k_rows), D]).
+    """
+    q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
+    R, M = q.shape[0], k.shape[0]
+    qr = np.asarray(q_rows, dtype=np.int64)
+    kr = np.asarray(k_rows, dtype=np.int64)
+
+    def row_terms(idx):
+        z = scale * (q[idx] @ k.T)
+        if causal:
+            z = np.where(np.arange(M)[None, :] > idx[:, None], -np.inf, z)
+        z = z - z.max(axis=1, keepdims=True)
+        p = np.exp(z)
+        p /= p.sum(axis=1, keepdims=True)
+        dp = do[idx] @ v.T
+        return p, p * (dp - (dp * p).sum(axis=1, keepdims=True))
+
+    _, ds = row_terms(qr)
+    dq = scale * (ds @ k)
+    dk = np.zeros((kr.size, q.shape[1]))
+    dv = np.zeros((kr.size, v.shape[1]))
+    for i0 in range(0, R if kr.size else 0, block):
+        idx = np.arange(i0, min(R, i0 + block))
+        p, ds = row_terms(idx)
+        dk += scale * (ds[:, kr].T @ q[idx])
+        dv += p[:, kr].T @ do[idx]
+    return dq, dk, dv
+
+
 def attention_heads_bwd(T: np.ndarray, dO: np.ndarray, N: int, scale: float, cu_seqlens=None,
                         causal: bool = False) -> np.ndarray:
     """Gradients of step two for every head-sharded slab.

@@ -116,3 +116,64 @@ def test_layer_backward_against_oracle(gpu, P, N, H, cu, causal):
     for c, name in enumerate(("dQ", "dK", "dV")):
         _close(got[:N, c], ref[:N, c], name)
     assert np.all(got[N:] == 0)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_backward_dit19k(gpu, causal):
+    """Video-DiT size (P=4, N=19,394, H=56), as the benchmark times it.
+
+    Every head: sum_k dK[k] = 0 (each row of dS sums to zero) and
+    sum_k dV[k] = sum_q dO[q] (each row of P sums to one).  Sampled rows against
+    fp64: dQ at 256 queries of every head, dK / dV at 256 keys of two heads.
+    """
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    P, N, H = 4, 19_394, 56
+    plan = U.ulysses_plan(N, H, 128, P, 3, causal=causal)
+    Np, Hl = plan.padded_tokens, H // P
+    scale = 1.0 / math.sqrt(128)
+    S = inputs.qkv_seq(N, H, P, 3, 1, gpu)
+    T = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, T)
+    del S
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=gpu)
+    U.ulysses_attn_fwd_lse(plan, T, OT, lse, scale)
+    dO = _grad(gpu, (P, Np, Hl, 128), 210 + causal)
+    dO[:, N:] = 0
+    dT = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    ws = torch.empty(plan.attn_bwd_workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_attn_bwd(plan, T, OT, dO, lse, dT, ws, scale)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    assert not dT[:, :, N:].any()
+    # invariants on every head, fp64 sums of the bf16 gradients
+    dK = dT[:, 1, :N].double()
+    dV = dT[:, 2, :N].double()
+    g = dO[:, :N].double()
+    assert (dK.sum(1).abs() <= 1e-3 * dK.abs().sum(1) + 1e-6).all()
+    assert ((dV.sum(1) - g.sum(1)).abs() <= 1e-3 * g.abs().sum(1) + 1e-6).all()
+    del dK, dV, g
+    # sampled rows
+    rng = np.random.default_rng(7 + causal)
+    qr = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 254, replace=False)]))
+    kr = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 254, replace=False)]))
+    iq, ik = torch.from_numpy(qr).to(gpu), torch.from_numpy(kr).to(gpu)
+    got_q = dT[:, 0].index_select(1, iq).double().cpu().numpy()          # [P, R, Hl, D]
+    got_k = dT[:, 1].index_select(1, ik).double().cpu().numpy()
+    got_v = dT[:, 2].index_select(1, ik).double().cpu().numpy()
+    T_bits = inputs.host_bits(T)
+    dO_bits = inputs.host_bits(dO)
+    full_heads = {(0, 0), (P - 1, Hl - 1)}
+    for r in range(P):
+        for j in range(Hl):
+            q, k, v = (orc.bf16_bits_to_f64(T_bits[r, c, :N, j]) for c in range(3))
+            g_h = orc.bf16_bits_to_f64(dO_bits[r, :N, j])
+            sel = kr if (r, j) in full_heads else kr[:0]
+            dq, dk, dv = orc.attention_bwd_sampled(q, k, v, g_h, scale, qr, sel, causal)
+            _close(got_q[r, :, j], dq, f"dQ {r},{j}")
+            if sel.size:
+                _close(got_k[r, :, j], dk, f"dK {r},{j}")
+                _close(got_v[r, :, j], dv, f"dV {r},{j}")

@@ -450,3 +450,17 @@ def test_layer_backward_is_transposed_repack_of_head_gradients():
     q, k, v = (orc.bf16_bits_to_f64(S[:3, c, 0]) for c in range(3))
     dq, dk, dv = orc.attention_rows_bwd(q, k, v, G[:3, 0], 0.4)
     assert np.allclose(dS2[:3, 1, 0], dk, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_backward_equals_full_rows(causal):
+    # the row-sampled backward reduces to the full one (pinned above by finite differences)
+    rng = np.random.default_rng(64 + causal)
+    R, D = 37, 8
+    q, k, v, g = (rng.standard_normal((R, D)) for _ in range(4))
+    dq, dk, dv = orc.attention_rows_bwd(q, k, v, g, 0.6, 0 if causal else None)
+    qr, kr = np.array([0, 5, 36, 17]), np.array([36, 0, 11])
+    sq, sk, sv = orc.attention_bwd_sampled(q, k, v, g, 0.6, qr, kr, causal, block=5)
+    assert np.allclose(sq, dq[qr], rtol=0, atol=1e-12)
+    assert np.allclose(sk, dk[kr], rtol=0, atol=1e-12)
+    assert np.allclose(sv, dv[kr], rtol=0, atol=1e-12)

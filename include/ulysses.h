@@ -203,7 +203,8 @@ size_t ulysses_lse_bytes(const ulysses_plan_t* plan);
 int ulysses_attn_fwd_lse(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, void* lse,
                          float softmax_scale, void* stream);
 
-/* Workspace of ulysses_attn_bwd (the row terms rowsum(dO o O)). */
+/* Workspace of ulysses_attn_bwd: the row terms -rowsum(dO o O) and a negated
+ * copy of lse, each ulysses_lse_bytes() long. */
 size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan);
 
 /*

@@ -329,7 +329,7 @@ int ulysses_attn_fwd_lse(const ulysses_plan_t* plan, const void* qkv_heads, void
 }
 
 size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan) {
-  return plan ? static_cast<size_t>(lse_bytes(plan)) : 0;
+  return plan ? static_cast<size_t>(2 * lse_bytes(plan)) : 0;
 }
 
 int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads,
@@ -341,10 +341,12 @@ int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const vo
   const void* ptrs[] = {qkv_heads, out_heads, dout_heads, lse, dqkv_heads, workspace};
   for (const void* q : ptrs)
     if (!aligned16(q)) return ULYSSES_ERR_ALIGN;
-  const int64_t dq = heads_bytes(plan, 3), ws = lse_bytes(plan);
+  const int64_t dq = heads_bytes(plan, 3), lb = lse_bytes(plan), ws = 2 * lb;
   if (overlap(dqkv_heads, dq, qkv_heads, heads_bytes(plan, plan->C)) || overlap(dqkv_heads, dq, out_heads, heads_bytes(plan, 1)) ||
-      overlap(dqkv_heads, dq, dout_heads, heads_bytes(plan, 1)) || overlap(dqkv_heads, dq, lse, ws) ||
-      overlap(workspace, ws, dqkv_heads, dq) || overlap(workspace, ws, lse, ws))
+      overlap(dqkv_heads, dq, dout_heads, heads_bytes(plan, 1)) || overlap(dqkv_heads, dq, lse, lb) ||
+      overlap(workspace, ws, dqkv_heads, dq) || overlap(workspace, ws, lse, lb) ||
+      overlap(workspace, ws, qkv_heads, heads_bytes(plan, plan->C)) || overlap(workspace, ws, out_heads, heads_bytes(plan, 1)) ||
+      overlap(workspace, ws, dout_heads, heads_bytes(plan, 1)))
     return ULYSSES_ERR_ARG;
   int s = device_ready(plan);
   if (s != ULYSSES_OK) return s;
@@ -363,7 +365,7 @@ int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const vo
 size_t ulysses_layer_bwd_workspace_bytes(const ulysses_plan_t* plan) {
   if (!plan) return 0;
   return static_cast<size_t>(align_up(heads_bytes(plan, 1), 256) + align_up(heads_bytes(plan, 3), 256) +
-                             align_up(lse_bytes(plan), 256));
+                             align_up(2 * lse_bytes(plan), 256));
 }
 
 int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads, const void* lse,

@@ -37,7 +37,7 @@ namespace ulysses {
 namespace {
 
 constexpr int kEwWarps = 8;                           // two warpgroups, 64 columns each
-constexpr int kThreads = 32 * (kEwWarps + 2);
+constexpr int kThreads = 32 * (kEwWarps + 2);         // + the MMA and TMA warps
 constexpr int kMmaWarp = kEwWarps;
 constexpr int kTmaWarp = kEwWarps + 1;
 constexpr int BT = 128;                               // rows per tile (keys or queries)
@@ -51,15 +51,19 @@ constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 constexpr uint32_t kOffF0 = 0;                                // fixed tile 0
 constexpr uint32_t kOffF1 = kTileBytes;                       // fixed tile 1
 constexpr uint32_t kOffX = 2 * kTileBytes;                    // [stage][X0, X1]
-// pass A: per stage, 132 lse floats then 132 D floats, copied from the block
-// start rounded down to a multiple of 4 (16-byte aligned bulk copies)
+// pass A: per stage, 132 floats of -lse then 132 of -D, copied from the
+// block start rounded down to a multiple of 4 (16-byte aligned bulk copies)
 constexpr uint32_t kRowFloats = 132;
 constexpr uint32_t kRowStageBytes = 2 * kRowFloats * 4;                // 1056
 constexpr uint32_t kOffRow = kOffX + kStages * 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffRow + kStages * kRowStageBytes;
+// Streamed tiles: X0 (pass A: Q, pass B: K) and X1 (dO / V) arrive on their
+// own barriers, so the MMA that needs X0 first does not wait for X1.  Pass A
+// frees both with one commit after dK; pass B frees V as soon as dP is done
+// (an elementwise thread arrives) and K with a commit after dQ.
 enum {
-  B_FFULL = 0, B_FEMPTY, B_XFULL0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_SFULL, B_DPFULL, B_PFULL, B_DSFULL, B_OFULL,
-  B_OEMPTY, B_DONE, B_COUNT
+  B_FFULL = 0, B_FEMPTY, B_X0FULL0, B_X0FULL1, B_X1FULL0, B_X1FULL1, B_X0EMPTY0, B_X0EMPTY1, B_X1EMPTY0,
+  B_X1EMPTY1, B_SFULL, B_DPFULL, B_PFULL, B_DSFULL, B_OFULL, B_OEMPTY, B_DONE, B_COUNT
 };
 constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;
 constexpr uint32_t kOffAbort = kOffSlot + 4;
@@ -79,9 +83,9 @@ struct SegB {
 
 struct BwdParams {
   __nv_bfloat16* dqkv;     // [P, 3, Np, Hl, D]
-  const float* lse;        // [P*Hl][ls]
-  const float* delta;      // [P*Hl][ls]
-  int64_t ls;              // row stride of lse / delta
+  const float* nlse;       // [P*Hl][ls]: -lse
+  const float* nd;         // [P*Hl][ls]: -rowsum(dO o O)
+  int64_t ls;              // row stride of both
   unsigned int* err;
   int32_t N, Np, Hl, P, causal;
   int32_t num_units, nseg;
@@ -132,10 +136,13 @@ __device__ __forceinline__ bool drain_wait_b(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-// D[(r*Hl + j) * ls + n] = sum_d dO[r, n, j, d] * O[r, n, j, d] for n < Np.
-// One half-warp per row: 16 lanes x 8 channels.
+// nd[(r*Hl + j) * ls + n] = -sum_d dO[r, n, j, d] * O[r, n, j, d] and
+// nlse[...] = -lse[...] for n < Np: the row terms the elementwise step
+// subtracts, stored negated so that it adds them.  One half-warp per row:
+// 16 lanes x 8 channels.
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const int4* __restrict__ out, const int4* __restrict__ dout,
-                                                        float* __restrict__ delta, int64_t rows, int32_t Np,
+                                                        const float* __restrict__ lse, float* __restrict__ nd,
+                                                        float* __restrict__ nlse, int64_t rows, int32_t Np,
                                                         int32_t Hl, int64_t ls) {
   const int64_t hw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
   const int64_t nhw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
@@ -163,7 +170,9 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const int4* __restrict__
       const int64_t j = row % Hl;
       const int64_t rn = row / Hl;
       const int64_t n = rn % Np, r = rn / Np;
-      delta[(r * Hl + j) * ls + n] = acc;
+      const int64_t o = (r * Hl + j) * ls + n;
+      nd[o] = -acc;
+      nlse[o] = -lse[o];
     }
   }
 }
@@ -171,24 +180,31 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const int4* __restrict__
 // Elementwise step of one streamed block for one thread: its TMEM lane (a key
 // in pass A, a query in pass B) against the 64 columns of its warpgroup.
 //   P  = exp2(s log2e S - lse)             (0 where the pair is masked)
-// kMask: the block straddles a segment end or the causal diagonal.
+// Pass A takes -lse per column from shared memory (nl_s), pass B one value
+// per row (nl_row).  kMask: the block straddles a segment end or the causal
+// diagonal, or (pass A) its rows are not 16-byte aligned in shared memory;
+// otherwise the columns are read four at a time.
 template <bool kPassA, bool kMask>
 __device__ __forceinline__ void p_block(const uint32_t (&sv)[2][32], float (&pr)[64], float sl2,
-                                        const float* lse_s, float lse_row, int col0, int my, int end, int causal) {
-  if (kPassA) {
+                                        const float* nl_s, uint32_t nl_sa, float nl_row, int col0, int my, int end,
+                                        int causal) {
+  auto sval = [&](int e) { return __uint_as_float(sv[e >> 5][e & 31]); };
+  if (kPassA && !kMask) {
 #pragma unroll
-    for (int e = 0; e < 64; e += 2) {
-      const f2 x = ffma2(f2{__uint_as_float(sv[e >> 5][e & 31]), __uint_as_float(sv[e >> 5][(e & 31) + 1])},
-                         f2{sl2, sl2}, f2{-lse_s[e], -lse_s[e + 1]});
-      pr[e] = ex2_approx(x.x);
-      pr[e + 1] = ex2_approx(x.y);
+    for (int e = 0; e < 64; e += 4) {
+      const float4 l = lds128(nl_sa + 4 * e);
+      const f2 x0 = ffma2(f2{sval(e), sval(e + 1)}, f2{sl2, sl2}, f2{l.x, l.y});
+      const f2 x1 = ffma2(f2{sval(e + 2), sval(e + 3)}, f2{sl2, sl2}, f2{l.z, l.w});
+      pr[e] = ex2_approx(x0.x);
+      pr[e + 1] = ex2_approx(x0.y);
+      pr[e + 2] = ex2_approx(x1.x);
+      pr[e + 3] = ex2_approx(x1.y);
     }
   } else {
-    const f2 nl{-lse_row, -lse_row};
 #pragma unroll
     for (int e = 0; e < 64; e += 2) {
-      const f2 x = ffma2(f2{__uint_as_float(sv[e >> 5][e & 31]), __uint_as_float(sv[e >> 5][(e & 31) + 1])},
-                         f2{sl2, sl2}, nl);
+      const f2 nl = kPassA ? f2{nl_s[e], nl_s[e + 1]} : f2{nl_row, nl_row};
+      const f2 x = ffma2(f2{sval(e), sval(e + 1)}, f2{sl2, sl2}, nl);
       pr[e] = ex2_approx(x.x);
       pr[e + 1] = ex2_approx(x.y);
     }
@@ -204,20 +220,34 @@ __device__ __forceinline__ void p_block(const uint32_t (&sv)[2][32], float (&pr)
   }
 }
 
-//   dS = P o (dP - D), packed to bf16 pairs (pk[h][k] holds columns 32h + 2k, 2k + 1)
+//   dS = P o (dP - D) over 32 columns, packed to bf16 pairs (pk[k] holds
+// columns 2k, 2k + 1); -D per column (pass A, nd_s) or per row (pass B, nd_row)
 template <bool kPassA, bool kMask>
-__device__ __forceinline__ void ds_block(const uint32_t (&dv)[2][32], const float (&pr)[64], const float* dlt_s,
-                                         float d_row, uint32_t (&pk)[2][16]) {
+__device__ __forceinline__ void ds_half(const uint32_t (&dv)[32], const float* pr, const float* nd_s, uint32_t nd_sa,
+                                        float nd_row, uint32_t (&pk)[16]) {
 #pragma unroll
-  for (int e = 0; e < 64; e += 2) {
-    const f2 nd = kPassA ? f2{-dlt_s[e], -dlt_s[e + 1]} : f2{-d_row, -d_row};
-    const f2 t = fadd2(f2{__uint_as_float(dv[e >> 5][e & 31]), __uint_as_float(dv[e >> 5][(e & 31) + 1])}, nd);
-    f2 d = fmul2(f2{pr[e], pr[e + 1]}, t);
-    if (kMask) {   // D past the segment end may be anything: masked entries stay exactly 0
-      d.x = pr[e] == 0.f ? 0.f : d.x;
-      d.y = pr[e + 1] == 0.f ? 0.f : d.y;
+  for (int e = 0; e < 32; e += 4) {
+    f2 n0, n1;
+    if (kPassA && !kMask) {
+      const float4 d = lds128(nd_sa + 4 * e);
+      n0 = f2{d.x, d.y};
+      n1 = f2{d.z, d.w};
+    } else if (kPassA) {
+      n0 = f2{nd_s[e], nd_s[e + 1]};
+      n1 = f2{nd_s[e + 2], nd_s[e + 3]};
+    } else {
+      n0 = n1 = f2{nd_row, nd_row};
     }
-    pk[e >> 5][(e & 31) >> 1] = pack_bf16x2(d.x, d.y);
+    f2 d0 = fmul2(f2{pr[e], pr[e + 1]}, fadd2(f2{__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])}, n0));
+    f2 d1 = fmul2(f2{pr[e + 2], pr[e + 3]}, fadd2(f2{__uint_as_float(dv[e + 2]), __uint_as_float(dv[e + 3])}, n1));
+    if (kMask) {   // D past the segment end may be anything: masked entries stay exactly 0
+      d0.x = pr[e] == 0.f ? 0.f : d0.x;
+      d0.y = pr[e + 1] == 0.f ? 0.f : d0.y;
+      d1.x = pr[e + 2] == 0.f ? 0.f : d1.x;
+      d1.y = pr[e + 3] == 0.f ? 0.f : d1.y;
+    }
+    pk[e >> 1] = pack_bf16x2(d0.x, d0.y);
+    pk[(e >> 1) + 1] = pack_bf16x2(d1.x, d1.y);
   }
 }
 
@@ -241,8 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(BAR(B_FFULL), 1);
     mbar_init(BAR(B_FEMPTY), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(BAR(B_XFULL0 + s), 1);
-      mbar_init(BAR(B_XEMPTY0 + s), 1);
+      mbar_init(BAR(B_X0FULL0 + s), 1);
+      mbar_init(BAR(B_X1FULL0 + s), 1);
+      mbar_init(BAR(B_X0EMPTY0 + s), 1);
+      mbar_init(BAR(B_X1EMPTY0 + s), 1);
     }
     mbar_init(BAR(B_SFULL), 1);
     mbar_init(BAR(B_DPFULL), 1);
@@ -267,10 +299,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
 
-  if (warp == kTmaWarp) {
+  if (warp >= kEwWarps) {
+   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t xc = 0, uc = 0;
+      uint32_t xc = 0, uc = 0, x0c = 0, x1c = 0;   // blocks, units, copies issued per tile barrier
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
         UnitB w;
@@ -295,33 +328,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < count; ++i) {
           const int r0 = sd.start + (first + i) * BT;
           const uint32_t s = xc % kStages, ph = (xc / kStages) & 1;
-          if (xc >= kStages && !(ok = mbar_wait(BAR(B_XEMPTY0 + s), ph ^ 1, g))) break;
           const uint32_t x0 = sbase + kOffX + s * 2 * kTileBytes, x1 = x0 + kTileBytes;
-          if (kPassA) {   // streamed: Q and dO of a query block, its lse and D
-            mbar_arrive_expect_tx(BAR(B_XFULL0 + s), 2 * kTileBytes + kRowStageBytes);
-            for (int h = 0; h < 2; ++h) {
-              tma_load_5d(x0 + h * kHalfBytes, &tm_qkv, BAR(B_XFULL0 + s), 64 * h, w.j, r0, 0, w.r);
-              tma_load_5d(x1 + h * kHalfBytes, &tm_do, BAR(B_XFULL0 + s), 64 * h, w.j, r0, 0, w.r);
-            }
+          if (kPassA) {   // streamed: Q with its -lse / -D rows, then dO, of a query block
+            if (xc >= kStages && !(ok = mbar_wait(BAR(B_X0EMPTY0 + s), ph ^ 1, g))) break;
+            mbar_arrive_expect_tx(BAR(B_X0FULL0 + s), kTileBytes + kRowStageBytes);
+            for (int h = 0; h < 2; ++h)
+              tma_load_5d(x0 + h * kHalfBytes, &tm_qkv, BAR(B_X0FULL0 + s), 64 * h, w.j, r0, 0, w.r);
             const int64_t roff = (static_cast<int64_t>(w.r) * p.Hl + w.j) * p.ls + (r0 & ~3);
-            bulk_load(sbase + kOffRow + s * kRowStageBytes, p.lse + roff, kRowFloats * 4, BAR(B_XFULL0 + s));
-            bulk_load(sbase + kOffRow + s * kRowStageBytes + kRowFloats * 4, p.delta + roff, kRowFloats * 4,
-                      BAR(B_XFULL0 + s));
-          } else {        // streamed: K and V of a key block
-            mbar_arrive_expect_tx(BAR(B_XFULL0 + s), 2 * kTileBytes);
-            for (int h = 0; h < 2; ++h) {
-              tma_load_5d(x0 + h * kHalfBytes, &tm_qkv, BAR(B_XFULL0 + s), 64 * h, w.j, r0, 1, w.r);
-              tma_load_5d(x1 + h * kHalfBytes, &tm_qkv, BAR(B_XFULL0 + s), 64 * h, w.j, r0, 2, w.r);
-            }
+            bulk_load(sbase + kOffRow + s * kRowStageBytes, p.nlse + roff, kRowFloats * 4, BAR(B_X0FULL0 + s));
+            bulk_load(sbase + kOffRow + s * kRowStageBytes + kRowFloats * 4, p.nd + roff, kRowFloats * 4,
+                      BAR(B_X0FULL0 + s));
+            ++x0c;
+            mbar_arrive_expect_tx(BAR(B_X1FULL0 + s), kTileBytes);
+            for (int h = 0; h < 2; ++h)
+              tma_load_5d(x1 + h * kHalfBytes, &tm_do, BAR(B_X1FULL0 + s), 64 * h, w.j, r0, 0, w.r);
+            ++x1c;
+          } else {        // streamed: V as soon as its slot is free (after dP), then K (after dQ)
+            if (xc >= kStages && !(ok = mbar_wait(BAR(B_X1EMPTY0 + s), ph ^ 1, g))) break;
+            mbar_arrive_expect_tx(BAR(B_X1FULL0 + s), kTileBytes);
+            for (int h = 0; h < 2; ++h)
+              tma_load_5d(x1 + h * kHalfBytes, &tm_qkv, BAR(B_X1FULL0 + s), 64 * h, w.j, r0, 2, w.r);
+            ++x1c;
+            if (xc >= kStages && !(ok = mbar_wait(BAR(B_X0EMPTY0 + s), ph ^ 1, g))) break;
+            mbar_arrive_expect_tx(BAR(B_X0FULL0 + s), kTileBytes);
+            for (int h = 0; h < 2; ++h)
+              tma_load_5d(x0 + h * kHalfBytes, &tm_qkv, BAR(B_X0FULL0 + s), 64 * h, w.j, r0, 1, w.r);
+            ++x0c;
           }
           ++xc;
         }
       }
+      // no copy may be in flight when the CTA exits
       if (uc > 0) drain_wait_b(BAR(B_FFULL), (uc - 1) & 1);
-      for (uint32_t n = (xc > kStages ? xc - kStages : 0); n < xc; ++n)
-        drain_wait_b(BAR(B_XFULL0 + n % kStages), (n / kStages) & 1);
+      for (uint32_t n = (x0c > kStages ? x0c - kStages : 0); n < x0c; ++n)
+        drain_wait_b(BAR(B_X0FULL0 + n % kStages), (n / kStages) & 1);
+      for (uint32_t n = (x1c > kStages ? x1c - kStages : 0); n < x1c; ++n)
+        drain_wait_b(BAR(B_X1FULL0 + n % kStages), (n / kStages) & 1);
     }
-  } else if (warp == kMmaWarp) {
+   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ tcgen05 issuer
     // Per block i (pass A):  [P^T(i) ready] dV += P^T dO, S(i+1), [dS^T(i) ready] dK += dS^T Q, dP(i+1)
     //           (pass B):  [S(i) read]      S(i+1),          [dS(i) ready]   dQ += dS K,   dP(i+1)
@@ -346,12 +390,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (uc > 0 && !(ok = mbar_wait(BAR(B_OEMPTY), (uc - 1) & 1, g))) break;
         tc_fence_after();
         if (count > 0) {
-          const uint32_t s = xc % kStages;
-          if (!(ok = mbar_wait(BAR(B_XFULL0 + s), (xc / kStages) & 1, g))) break;
+          const uint32_t s = xc % kStages, ph = (xc / kStages) & 1;
+          if (!(ok = mbar_wait(BAR(B_X0FULL0 + s), ph, g))) break;
           tc_fence_after();
           // pass A: S^T = K Q^T, dP^T = V dO^T;  pass B: S = Q K^T, dP = dO V^T
           mma_ss_k128(tmem + kColA0, dF0, xdesc(s, 0, 16), kIdescSS, 0);
           mma_commit(BAR(B_SFULL));
+          if (!(ok = mbar_wait(BAR(B_X1FULL0 + s), ph, g))) break;
+          tc_fence_after();
           mma_ss_k128(tmem + kColA1, dF1, xdesc(s, 1, 16), kIdescSS, 0);
           mma_commit(BAR(B_DPFULL));
         }
@@ -365,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts_k64(tmem + kColAcc0, tmem + kColA0 + 64, xdesc(s, 1, kHalfBytes) + 512, kIdescTS, 1);
           }
           if (more) {     // S of the next block over A0 (in order after the MMAs that read it)
-            if (!(ok = mbar_wait(BAR(B_XFULL0 + sn), ((xi + 1) / kStages) & 1, g))) break;
+            if (!(ok = mbar_wait(BAR(B_X0FULL0 + sn), ((xi + 1) / kStages) & 1, g))) break;
             tc_fence_after();
             mma_ss_k128(tmem + kColA0, dF0, xdesc(sn, 0, 16), kIdescSS, 0);
             mma_commit(BAR(B_SFULL));
@@ -377,8 +423,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t acc = kPassA ? kColAcc1 : kColAcc0;
           mma_ts_k64(tmem + acc, tmem + kColA1, xdesc(s, 0, kHalfBytes), kIdescTS, i > 0);
           mma_ts_k64(tmem + acc, tmem + kColA1 + 64, xdesc(s, 0, kHalfBytes) + 512, kIdescTS, 1);
-          mma_commit(BAR(B_XEMPTY0 + s));
+          mma_commit(BAR(B_X0EMPTY0 + s));
           if (more) {     // dP of the next block over A1
+            if (!(ok = mbar_wait(BAR(B_X1FULL0 + sn), ((xi + 1) / kStages) & 1, g))) break;
+            tc_fence_after();
             mma_ss_k128(tmem + kColA1, dF1, xdesc(sn, 1, 16), kIdescSS, 0);
             mma_commit(BAR(B_DPFULL));
           }
@@ -391,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(BAR(B_DONE));
       drain_wait_b(BAR(B_DONE), 0);
     }
-  } else if (warp < kEwWarps) {
+   }
+  } else {
     // ------------------------------------------------------------ elementwise + epilogue
     // Warp w owns TMEM lanes 32 (w % 4) .. +31 (one row of the unit's tile per
     // thread) and, with its warpgroup w / 4, 64 of the 128 columns.
@@ -412,11 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int first, count;
       stream_range<kPassA>(p, sd, w, first, count);
       const int my = w.row0 + row;                     // key (pass A) or query (pass B) index
-      float lse_row = 0.f, d_row = 0.f;
+      float nl_row = 0.f, nd_row = 0.f;               // pass B: -lse and -D of this thread's query
       if (!kPassA && my < p.Np) {
         const int64_t off = (static_cast<int64_t>(w.r) * p.Hl + w.j) * p.ls + my;
-        lse_row = p.lse[off];
-        d_row = p.delta[off];
+        nl_row = p.nlse[off];
+        nd_row = p.nd[off];
       }
       for (int i = 0; i < count; ++i) {
         if (!(ok = mbar_wait_warp(BAR(B_SFULL), sc & 1, g))) break;
@@ -425,14 +474,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r0 = sd.start + (first + i) * BT;    // first streamed index of this block
         const uint32_t s = xc % kStages;
         // pass A reads the block's lse / D rows, which arrive with the stage
-        if (kPassA && !(ok = mbar_wait_warp(BAR(B_XFULL0 + s), (xc / kStages) & 1, g))) break;
+        const uint32_t ph = (xc / kStages) & 1;
+        if (kPassA && !(ok = mbar_wait_warp(BAR(B_X0FULL0 + s), ph, g))) break;
         ++xc;
         // lse / D of the warpgroup's 64 streamed queries (the copy starts at r0 rounded down to 4)
-        const float* lse_s = srow + s * (kRowStageBytes / 4) + (r0 & 3) + c0;
-        const float* dlt_s = lse_s + kRowFloats;
+        const float* nl_s = srow + s * (kRowStageBytes / 4) + (r0 & 3) + c0;
+        const float* nd_s = nl_s + kRowFloats;
+        const uint32_t nl_sa = sbase + kOffRow + s * kRowStageBytes + 4 * ((r0 & 3) + c0);   // same, shared window
+        const uint32_t nd_sa = nl_sa + 4 * kRowFloats;
         // the whole 128 x 128 block is inside the segment and off the causal diagonal
+        // (pass A also needs its shared-memory rows 16-byte aligned: blocks start at
+        // the segment start plus multiples of 128)
         const bool full = w.row0 + BT <= end && r0 + BT <= end &&
-                          (!p.causal || (kPassA ? r0 > w.row0 : r0 < w.row0));
+                          (!p.causal || (kPassA ? r0 > w.row0 : r0 < w.row0)) && (!kPassA || (r0 & 3) == 0);
         // phase 1 (S ready): P in fp32, kept for phase 2; pass A stores P^T (bf16) for dV += P^T dO
         float pr[64];
         {
@@ -443,9 +497,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_regs_ready(sv[0]);
           tmem_regs_ready(sv[1]);
           if (full)
-            p_block<kPassA, false>(sv, pr, sl2, lse_s, lse_row, r0 + c0, my, end, p.causal);
+            p_block<kPassA, false>(sv, pr, sl2, nl_s, nl_sa, nl_row, r0 + c0, my, end, p.causal);
           else
-            p_block<kPassA, true>(sv, pr, sl2, lse_s, lse_row, r0 + c0, my, end, p.causal);
+            p_block<kPassA, true>(sv, pr, sl2, nl_s, nl_sa, nl_row, r0 + c0, my, end, p.causal);
         }
         if (kPassA) {
           uint32_t pk[2][16];
@@ -461,20 +515,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // phase 2 (dP ready): dS = P o (dP - D) over columns c0 .. c0 + 31 of A1
         if (!(ok = mbar_wait_warp(BAR(B_DPFULL), (sc - 1) & 1, g))) break;
         tc_fence_after();
-        {
-          uint32_t dv[2][32];
-          tmem_ld32(tA1, dv[0]);
-          tmem_ld32(tA1 + 32, dv[1]);
+        if (!kPassA && threadIdx.x == 0) mbar_arrive(BAR(B_X1EMPTY0 + s));   // dP done: V's slot is free
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {    // two halves of 32 columns: dS of half 0 lands before half 1 is read
+          uint32_t dv[32];
+          tmem_ld32(tA1 + 32 * h, dv);
           tmem_wait_ld();
-          tmem_regs_ready(dv[0]);
-          tmem_regs_ready(dv[1]);
-          uint32_t pk[2][16];
+          tmem_regs_ready(dv);
+          uint32_t pk[16];
           if (full)
-            ds_block<kPassA, false>(dv, pr, dlt_s, d_row, pk);
+            ds_half<kPassA, false>(dv, pr + 32 * h, nd_s + 32 * h, nd_sa + 128 * h, nd_row, pk);
           else
-            ds_block<kPassA, true>(dv, pr, dlt_s, d_row, pk);
-          tmem_st16(tA1, pk[0]);
-          tmem_st16(tA1 + 16, pk[1]);
+            ds_half<kPassA, true>(dv, pr + 32 * h, nd_s + 32 * h, nd_sa + 128 * h, nd_row, pk);
+          tmem_st16(tA1 + 16 * h, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -595,8 +648,8 @@ cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
     const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
     if (grid > 0)
       bwd_delta_kernel<<<grid, 256, 0, stream>>>(static_cast<const int4*>(a.out), static_cast<const int4*>(a.dout),
-                                                 a.delta, rows, static_cast<int32_t>(Np), static_cast<int32_t>(Hl),
-                                                 ls);
+                                                 a.lse, a.delta, a.delta + P * Hl * ls, rows,
+                                                 static_cast<int32_t>(Np), static_cast<int32_t>(Hl), ls);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -607,8 +660,8 @@ cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   p.dqkv = static_cast<__nv_bfloat16*>(a.dqkv);
-  p.lse = a.lse;
-  p.delta = a.delta;
+  p.nd = a.delta;
+  p.nlse = a.delta + P * Hl * ls;
   p.ls = ls;
   p.err = pl->dev_err;
   p.N = static_cast<int32_t>(pl->N);

@@ -72,7 +72,7 @@ struct AttnBwdLaunch {
   const void* out;      // O_T [P, Np, Hl, D]
   const void* dout;     // dO_T [P, Np, Hl, D]
   const float* lse;     // [P*Hl][lse_stride] from the forward
-  float* delta;         // workspace [P*Hl][lse_stride]: rowsum(dO o O)
+  float* delta;         // workspace: -rowsum(dO o O), then -lse, each [P*Hl][lse_stride]
   void* dqkv;           // [P, 3, Np, Hl, D]
   float scale;
   const ulysses_plan_t* plan;

@@ -355,6 +355,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// 16-byte shared-memory load at a shared-window address (volatile: stays after
+// the barrier wait that publishes the data).
+__device__ __forceinline__ float4 lds128(uint32_t saddr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(saddr));
+  return v;
+}
+
 // Paired fp32 arithmetic (one instruction for two lanes of a register pair).
 struct f2 {
   float x, y;

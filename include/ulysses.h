@@ -247,11 +247,27 @@ int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out
                       size_t workspace_bytes, int32_t fused, void* stream);
 
 /*
- * ulysses_layer_fwd from HOST buffers: copies host_qkv_seq (pinned host
- * memory, the plan's input layout) into dev_qkv_seq, runs the layer into
- * dev_out_seq, and copies O_S back to host_out_seq, all on `stream`
- * (asynchronous: synchronise before reading host_out_seq).  Device buffers
- * and workspace are the caller's.  Errors: as ulysses_layer_fwd.
+ * ulysses_layer_fwd from HOST buffers: host_qkv_seq (the plan's input
+ * layout) is copied into dev_qkv_seq, the layer runs into dev_out_seq, and
+ * O_S [Np, H, D] is copied back to host_out_seq.  Device buffers and the
+ * workspace are the caller's; the host buffers should be pinned (pageable
+ * memory works but serialises the copies with the host).
+ *
+ * The work is streamed by virtual rank, which is exact because rank r's share
+ * of the layer (its heads [r*Hl, (r+1)*Hl) of every token, mode 0 into its
+ * head slab, attention, mode 1 back into its head columns of O_S) touches no
+ * other rank's data: the host->device copy of rank r+1's head columns
+ * overlaps rank r's kernels on `stream`, which overlap the device->host copy
+ * of rank r-1's output columns.  The copies run on two streams owned by the
+ * plan (created with 2P+2 events by the plan's first call of this function,
+ * destroyed with the plan) and are ordered against `stream` by events: they
+ * start after the work already queued on `stream`, and `stream` completes
+ * only after the last output copy, so synchronising `stream` is enough
+ * before reading host_out_seq.  Concurrent calls with one plan are
+ * serialised on the host while they enqueue.  The result equals
+ * ulysses_layer_fwd's bit for bit.  Errors: as ulysses_layer_fwd; CUDA if a
+ * stream, event or copy could not be created or queued (the device buffers
+ * may then hold partial results).
  */
 int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
                            void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,

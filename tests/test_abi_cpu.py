@@ -109,6 +109,14 @@ def test_launch_argument_checks_before_any_device_work():
     assert lib.ulysses_layer_fwd(h, 0x10000, 0x90000000, None, 0, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
     assert lib.ulysses_layer_fwd(h, 0x10000, 0x90000000, 0xA0000000, 16, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
     assert lib.ulysses_layer_fwd(h, 0x10000, 0x90000000, None, 0, 2, None) == _lib.ULYSSES_ERR_ARG
+    # host-buffer layer: same checks, made before any stream or copy is created
+    hl = lib.ulysses_layer_fwd_host
+    assert hl(h, None, 0x20000000, 0x10000, 0x90000000, None, 0, 1, None) == _lib.ULYSSES_ERR_ARG
+    assert hl(h, 0x30000000, 0x20000000, 0x10000, 0x90000000, None, 0, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
+    assert hl(h, 0x30000000, 0x20000000, 0x10008, 0x90000000, None, 0, 1, None) == _lib.ULYSSES_ERR_ALIGN
+    assert hl(h, 0x30000000, 0x30000000, 0x10000, 0x90000000, None, 0, 1, None) == _lib.ULYSSES_ERR_ARG
+    assert hl(h, 0x30000000, 0x20000000, 0x10000, 0x10000, None, 0, 1, None) == _lib.ULYSSES_ERR_ARG
+    assert hl(h, 0x30000000, 0x20000000, 0x10000, 0x90000000, None, 0, 3, None) == _lib.ULYSSES_ERR_ARG
     # a gate-less plan cannot run attention
     p2 = U.ulysses_plan(1024, 8, 128, 2, 2)
     assert lib.ulysses_attn_fwd(p2.handle, 0x10000, 0x90000000, 0.1, None) == _lib.ULYSSES_ERR_ARG

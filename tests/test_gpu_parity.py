@@ -184,3 +184,52 @@ def test_uniform_keys_give_mean_of_v(gpu):
     want = np.broadcast_to(v.mean(axis=0, keepdims=True), v.shape)
     err = np.abs(_f32(OS) - want)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+
+
+HOST_CASES = [
+    pytest.param(2, 1024, 8, 3, "token", None, False, 30, id="tiny"),
+    pytest.param(4, 1001, 8, 3, "token", None, False, 31, id="ragged-P4"),
+    pytest.param(4, 777, 8, 4, "token", None, False, 32, id="qkvg-P4"),
+    pytest.param(2, 640, 4, 3, "plane", None, False, 33, id="plane-major"),
+    pytest.param(8, 2048, 16, 3, "token", [0, 1024, 1536, 2048], False, 34, id="varlen-P8"),
+    pytest.param(4, 1001, 8, 3, "token", None, True, 35, id="causal-P4"),
+]
+
+
+@pytest.mark.parametrize("P,N,H,C,layout,cu,causal,seed", HOST_CASES)
+def test_host_layer_streams_ranks_exactly(gpu, P, N, H, C, layout, cu, causal, seed):
+    """ulysses_layer_fwd_host (copies and kernels streamed rank by rank) equals
+    the device layer bit for bit, fused and unfused, on two calls in a row
+    with a non-default stream that is the only thing synchronised."""
+    torch = _torch()
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    ts, ps = _strides(layout, N, P, C, H)
+    plan = U.ulysses_plan(N, H, 128, P, C, ts, ps, 0, cu, causal=causal)
+    Np = plan.padded_tokens
+    S = inputs.qkv_seq(N, H, P, C, seed, gpu, layout=layout)
+    want = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_layer_fwd(plan, S, want, ws, fused=0)
+    torch.cuda.synchronize()
+    want_bits = _bits(want)
+    host_in = S.cpu().pin_memory()
+    dev_in = torch.empty_like(S)
+    dev_out = torch.empty_like(want)
+    stream = torch.cuda.Stream(device=gpu)
+    for fused in (0, 1, 0):
+        host_out = torch.full(want.shape, float("nan"), dtype=torch.bfloat16).pin_memory()
+        dev_in.zero_()
+        dev_out.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            U.ulysses_layer_fwd_host(plan, host_in, host_out, dev_in, dev_out, ws if fused == 0 else None,
+                                     fused=fused, stream=stream)
+        stream.synchronize()
+        assert U.ulysses_last_device_error(plan, stream) == 0
+        assert np.array_equal(host_out.view(torch.int16).numpy().view("uint16"), want_bits), fused
+        assert torch.equal(dev_in, S)
+    ref = orc.layer_fwd(_seq_as_token_major(_bits(S), layout), P, N, 1.0 / math.sqrt(128), cu_seqlens=cu,
+                        causal=causal)
+    err = np.abs(_f32(want) - ref)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "internal.h"
@@ -119,6 +120,144 @@ int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, f
   return status_of(ulysses::launch_attn(a, st));
 }
 
+// ---------------------------------------------------------------- host-buffer layer, pipelined by rank
+//
+// Virtual rank r owns heads [r*Hl, (r+1)*Hl) after the all-to-all, and its
+// share of the layer (mode 0 into its head slab, attention on it, mode 1 back
+// into its head columns of O_S) reads and writes nothing of the other ranks.
+// The host path therefore streams the layer rank by rank: the copy of rank
+// r+1's head columns to the device overlaps rank r's kernels, which overlap
+// the copy of rank r-1's output columns back to the host.
+
+}  // namespace
+
+namespace ulysses {
+
+// Two copy streams (host->device, device->host) and the events that order
+// them against the caller's stream: start, one input and one output event per
+// rank, done.  Owned by the plan, created by its first host-buffer call.
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t* in = nullptr;
+  cudaEvent_t* out = nullptr;
+  int32_t n = 0;
+};
+
+}  // namespace ulysses
+
+namespace {
+
+std::mutex g_pipe_mutex;   // guards pipe creation and the enqueue of one host-buffer call
+
+void destroy_pipe(ulysses::HostPipe* h) {
+  if (!h) return;
+  if (h->h2d) cudaStreamDestroy(h->h2d);
+  if (h->d2h) cudaStreamDestroy(h->d2h);
+  if (h->start) cudaEventDestroy(h->start);
+  if (h->done) cudaEventDestroy(h->done);
+  for (int32_t i = 0; i < h->n; ++i) {
+    if (h->in && h->in[i]) cudaEventDestroy(h->in[i]);
+    if (h->out && h->out[i]) cudaEventDestroy(h->out[i]);
+  }
+  delete[] h->in;
+  delete[] h->out;
+  delete h;
+  cudaGetLastError();
+}
+
+// The plan's pipe, created on first use (call with g_pipe_mutex held, on the plan's device).
+ulysses::HostPipe* plan_pipe(const ulysses_plan_t* p) {
+  if (p->pipe) return p->pipe;
+  ulysses::HostPipe* h = new (std::nothrow) ulysses::HostPipe;
+  if (!h) return nullptr;
+  h->in = new (std::nothrow) cudaEvent_t[p->P]();
+  h->out = new (std::nothrow) cudaEvent_t[p->P]();
+  bool ok = h->in && h->out;
+  if (ok) h->n = p->P;
+  ok = ok && cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking) == cudaSuccess;
+  ok = ok && cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking) == cudaSuccess;
+  ok = ok && cudaEventCreateWithFlags(&h->start, cudaEventDisableTiming) == cudaSuccess;
+  ok = ok && cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming) == cudaSuccess;
+  for (int32_t i = 0; ok && i < p->P; ++i) {
+    ok = cudaEventCreateWithFlags(&h->in[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&h->out[i], cudaEventDisableTiming) == cudaSuccess;
+  }
+  if (!ok) {
+    destroy_pipe(h);
+    return nullptr;
+  }
+  const_cast<ulysses_plan_t*>(p)->pipe = h;   // a cache: the plan's geometry stays immutable
+  return h;
+}
+
+// Copy rank r's head columns of the sequence-sharded input (every token and
+// plane) between host and device; both sides use the plan's strides.
+cudaError_t copy_rank_input(const ulysses_plan_t* p, int32_t r, const uint8_t* host, uint8_t* dev, cudaStream_t s) {
+  const size_t width = static_cast<size_t>(p->Hl) * p->D * 2;
+  const size_t off = static_cast<size_t>(r) * width;
+  const size_t tok = static_cast<size_t>(p->token_stride) * 2, pl = static_cast<size_t>(p->plane_stride) * 2;
+  if (p->C == 1 || p->token_stride == static_cast<int64_t>(p->C) * p->plane_stride)   // rows (n, c) at pitch pl
+    return cudaMemcpy2DAsync(dev + off, pl, host + off, pl, width, static_cast<size_t>(p->Np) * p->C,
+                             cudaMemcpyHostToDevice, s);
+  if (p->plane_stride == p->Np * p->token_stride)   // rows (c, n) at pitch tok
+    return cudaMemcpy2DAsync(dev + off, tok, host + off, tok, width, static_cast<size_t>(p->Np) * p->C,
+                             cudaMemcpyHostToDevice, s);
+  for (int32_t c = 0; c < p->C; ++c) {
+    const size_t o = off + static_cast<size_t>(c) * pl;
+    cudaError_t e = cudaMemcpy2DAsync(dev + o, tok, host + o, tok, width, static_cast<size_t>(p->Np),
+                                      cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// Rank r's share of the layer on `st`: its heads of every token in S, its
+// head columns of O_S.  The kernels see the rank's slabs as a one-rank
+// problem (P = 1, H = Hl) at offset pointers.
+int rank_layer_impl(const ulysses_plan_t* p, int32_t r, const uint8_t* S, uint8_t* OS, uint8_t* T, uint8_t* OT,
+                    int32_t fused, float scale, cudaStream_t st) {
+  const int64_t head_cols = static_cast<int64_t>(p->Hl) * p->D;      // elements of one rank's heads in a row
+  const int64_t row = static_cast<int64_t>(p->H) * p->D;
+  const uint8_t* Sr = S + r * head_cols * 2;
+  uint8_t* OSr = OS + r * head_cols * 2;
+  ulysses::AttnLaunch a;
+  a.fused = fused;
+  a.Np = p->Np;
+  a.N = p->N;
+  a.H = p->Hl;
+  a.P = 1;
+  a.Hl = p->Hl;
+  a.C = p->C;
+  a.tok_stride = p->token_stride;
+  a.plane_stride = p->plane_stride;
+  a.o_stride_j = p->D;
+  a.scale = scale;
+  a.plan = p;
+  if (fused) {
+    a.base = Sr;
+    a.out = OSr;
+    a.o_stride_r = head_cols;
+    a.o_stride_n = row;
+    return status_of(ulysses::launch_attn(a, st));
+  }
+  uint8_t* Tr = T + r * static_cast<int64_t>(p->C) * p->Np * head_cols * 2;
+  uint8_t* OTr = OT + r * p->Np * head_cols * 2;
+  for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
+    const int32_t cc = std::min(p->plane_chunk, p->C - c0);
+    int s = status_of(ulysses::launch_repack(0, Sr, Tr, p->Np, p->Hl, 1, p->C, c0, cc, p->token_stride,
+                                             p->plane_stride, st));
+    if (s != ULYSSES_OK) return s;
+  }
+  a.base = Tr;
+  a.out = OTr;
+  a.o_stride_r = p->Np * head_cols;
+  a.o_stride_n = head_cols;
+  int s = status_of(ulysses::launch_attn(a, st));
+  if (s != ULYSSES_OK) return s;
+  return status_of(ulysses::launch_repack(1, OTr, OSr, p->Np, p->Hl, 1, 1, 0, 1, row, row, st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -202,6 +341,7 @@ int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32
   std::memcpy(p->segs, segs, sizeof(ulysses::Segment) * nseq);
   p->device = -1;
   p->dev_err = nullptr;
+  p->pipe = nullptr;
 
   // device error word (16 bytes) on the current device; absent without a GPU
   int dev = -1;
@@ -227,6 +367,7 @@ void ulysses_plan_destroy(ulysses_plan_t* plan) {
     int cur = -1;
     cudaGetDevice(&cur);
     if (cur != plan->device) cudaSetDevice(plan->device);
+    destroy_pipe(plan->pipe);
     cudaFree(plan->dev_err);
     if (cur >= 0 && cur != plan->device) cudaSetDevice(cur);
     cudaGetLastError();
@@ -447,17 +588,53 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
                            void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
                            int32_t fused, void* stream) {
   if (!plan || !host_qkv_seq || !host_out_seq || !dev_qkv_seq || !dev_out_seq) return ULYSSES_ERR_ARG;
+  if (plan->C < 3 || (fused != 0 && fused != 1)) return ULYSSES_ERR_ARG;
+  if (!aligned16(dev_qkv_seq) || !aligned16(dev_out_seq)) return ULYSSES_ERR_ALIGN;
+  const int64_t in_bytes = seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride);
+  if (overlap(dev_qkv_seq, in_bytes, dev_out_seq, out_seq_bytes(plan)) ||
+      overlap(host_qkv_seq, in_bytes, host_out_seq, out_seq_bytes(plan)))
+    return ULYSSES_ERR_ARG;
+  uint8_t* T = nullptr;
+  uint8_t* OT = nullptr;
+  if (!fused) {
+    if (!workspace || workspace_bytes < ulysses_workspace_bytes(plan)) return ULYSSES_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ULYSSES_ERR_ALIGN;
+    const int64_t ws = static_cast<int64_t>(ulysses_workspace_bytes(plan));
+    if (overlap(workspace, ws, dev_qkv_seq, in_bytes) || overlap(workspace, ws, dev_out_seq, out_seq_bytes(plan)))
+      return ULYSSES_ERR_ARG;
+    T = static_cast<uint8_t*>(workspace);
+    OT = T + align_up(heads_bytes(plan, plan->C), 256);
+  }
   int s = device_ready(plan);
   if (s != ULYSSES_OK) return s;
+  const float scale = 1.0f / std::sqrt(static_cast<float>(plan->D));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t in_bytes = seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride);
-  if (cudaMemcpyAsync(dev_qkv_seq, host_qkv_seq, static_cast<size_t>(in_bytes), cudaMemcpyHostToDevice, st) !=
-      cudaSuccess)
+  const uint8_t* hin = static_cast<const uint8_t*>(host_qkv_seq);
+  uint8_t* hout = static_cast<uint8_t*>(host_out_seq);
+  uint8_t* din = static_cast<uint8_t*>(dev_qkv_seq);
+  uint8_t* dout = static_cast<uint8_t*>(dev_out_seq);
+  const size_t width = static_cast<size_t>(plan->Hl) * plan->D * 2, pitch = static_cast<size_t>(plan->H) * plan->D * 2;
+
+  std::lock_guard<std::mutex> lock(g_pipe_mutex);
+  ulysses::HostPipe* h = plan_pipe(plan);
+  if (!h) return ULYSSES_ERR_CUDA;
+  // the copies start after everything already queued on the caller's stream
+  if (cudaEventRecord(h->start, st) != cudaSuccess || cudaStreamWaitEvent(h->h2d, h->start, 0) != cudaSuccess)
     return status_of(cudaErrorUnknown);
-  s = ulysses_layer_fwd(plan, dev_qkv_seq, dev_out_seq, workspace, workspace_bytes, fused, stream);
-  if (s != ULYSSES_OK) return s;
-  if (cudaMemcpyAsync(host_out_seq, dev_out_seq, static_cast<size_t>(out_seq_bytes(plan)), cudaMemcpyDeviceToHost,
-                      st) != cudaSuccess)
+  for (int32_t r = 0; r < plan->P; ++r) {
+    if (copy_rank_input(plan, r, hin, din, h->h2d) != cudaSuccess || cudaEventRecord(h->in[r], h->h2d) != cudaSuccess)
+      return status_of(cudaErrorUnknown);
+  }
+  for (int32_t r = 0; r < plan->P; ++r) {
+    if (cudaStreamWaitEvent(st, h->in[r], 0) != cudaSuccess) return status_of(cudaErrorUnknown);
+    if ((s = rank_layer_impl(plan, r, din, dout, T, OT, fused, scale, st)) != ULYSSES_OK) return s;
+    if (cudaEventRecord(h->out[r], st) != cudaSuccess || cudaStreamWaitEvent(h->d2h, h->out[r], 0) != cudaSuccess ||
+        cudaMemcpy2DAsync(hout + r * width, pitch, dout + r * width, pitch, width, static_cast<size_t>(plan->Np),
+                          cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess)
+      return status_of(cudaErrorUnknown);
+  }
+  // the caller's stream completes only after the last output copy
+  if (cudaEventRecord(h->done, h->d2h) != cudaSuccess || cudaStreamWaitEvent(st, h->done, 0) != cudaSuccess)
     return status_of(cudaErrorUnknown);
   return ULYSSES_OK;
 }

@@ -13,6 +13,8 @@ struct Segment {
   int32_t start, end;   // key / query range [start, end) of one packed sequence
 };
 
+struct HostPipe;   // copy streams and events of the host-buffer layer (api.cpp)
+
 }  // namespace ulysses
 
 struct ulysses_plan_s {
@@ -25,6 +27,7 @@ struct ulysses_plan_s {
   ulysses::Segment segs[ULYSSES_MAX_SEQS];
   int32_t device;                       // device the plan's scratch lives on (-1: none)
   unsigned int* dev_err;                // device error word (16 bytes allocated)
+  ulysses::HostPipe* pipe;              // created by the first ulysses_layer_fwd_host call
 };
 
 namespace ulysses {

@@ -253,21 +253,25 @@ int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out
  * workspace are the caller's; the host buffers should be pinned (pageable
  * memory works but serialises the copies with the host).
  *
- * The work is streamed by virtual rank, which is exact because rank r's share
- * of the layer (its heads [r*Hl, (r+1)*Hl) of every token, mode 0 into its
- * head slab, attention, mode 1 back into its head columns of O_S) touches no
- * other rank's data: the host->device copy of rank r+1's head columns
- * overlaps rank r's kernels on `stream`, which overlap the device->host copy
- * of rank r-1's output columns.  The copies run on two streams owned by the
- * plan (created with 2P+2 events by the plan's first call of this function,
+ * The work is streamed by groups of heads inside each virtual rank, which is
+ * exact because a head's share of the layer (mode 0 into a head slab,
+ * attention, mode 1 back into that head's columns of O_S) touches no other
+ * head's data: the host->device copy of group g+1's head columns overlaps
+ * group g's kernels on `stream`, which overlap the device->host copy of group
+ * g-1's output columns.  A group is the smallest divisor of H/P heads whose
+ * attention launch still fills every SM about three times over (at most one
+ * rank).  With fused = 0 the workspace holds the groups' head slabs one after
+ * another (its size is ulysses_workspace_bytes() as for the device layer; its
+ * layout is internal).  The copies run on two streams owned by the plan
+ * (created with their events by the plan's first call of this function,
  * destroyed with the plan) and are ordered against `stream` by events: they
  * start after the work already queued on `stream`, and `stream` completes
- * only after the last output copy, so synchronising `stream` is enough
- * before reading host_out_seq.  Concurrent calls with one plan are
- * serialised on the host while they enqueue.  The result equals
- * ulysses_layer_fwd's bit for bit.  Errors: as ulysses_layer_fwd; CUDA if a
- * stream, event or copy could not be created or queued (the device buffers
- * may then hold partial results).
+ * only after the last output copy, so synchronising `stream` is enough before
+ * reading host_out_seq.  Concurrent calls with one plan are serialised on the
+ * host while they enqueue.  The result equals ulysses_layer_fwd's bit for
+ * bit.  Errors: as ulysses_layer_fwd; CUDA if a stream, event or copy could
+ * not be created or queued (the device buffers may then hold partial
+ * results).
  */
 int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
                            void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,

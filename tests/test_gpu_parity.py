@@ -193,6 +193,8 @@ HOST_CASES = [
     pytest.param(2, 640, 4, 3, "plane", None, False, 33, id="plane-major"),
     pytest.param(8, 2048, 16, 3, "token", [0, 1024, 1536, 2048], False, 34, id="varlen-P8"),
     pytest.param(4, 1001, 8, 3, "token", None, True, 35, id="causal-P4"),
+    # 223 work units per head: the pipeline splits each rank's 4 heads into 2 groups
+    pytest.param(2, 57_001, 8, 3, "token", None, False, 36, id="head-groups"),
 ]
 
 
@@ -229,7 +231,8 @@ def test_host_layer_streams_ranks_exactly(gpu, P, N, H, C, layout, cu, causal, s
         assert U.ulysses_last_device_error(plan, stream) == 0
         assert np.array_equal(host_out.view(torch.int16).numpy().view("uint16"), want_bits), fused
         assert torch.equal(dev_in, S)
-    ref = orc.layer_fwd(_seq_as_token_major(_bits(S), layout), P, N, 1.0 / math.sqrt(128), cu_seqlens=cu,
-                        causal=causal)
-    err = np.abs(_f32(want) - ref)
-    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+    if N <= 4096:   # the device layer at larger N is checked against the oracle in the full-size tests
+        ref = orc.layer_fwd(_seq_as_token_major(_bits(S), layout), P, N, 1.0 / math.sqrt(128), cu_seqlens=cu,
+                            causal=causal)
+        err = np.abs(_f32(want) - ref)
+        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS

@@ -120,14 +120,15 @@ int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, f
   return status_of(ulysses::launch_attn(a, st));
 }
 
-// ---------------------------------------------------------------- host-buffer layer, pipelined by rank
+// ---------------------------------------------------------------- host-buffer layer, pipelined by head group
 //
-// Virtual rank r owns heads [r*Hl, (r+1)*Hl) after the all-to-all, and its
-// share of the layer (mode 0 into its head slab, attention on it, mode 1 back
-// into its head columns of O_S) reads and writes nothing of the other ranks.
-// The host path therefore streams the layer rank by rank: the copy of rank
-// r+1's head columns to the device overlaps rank r's kernels, which overlap
-// the copy of rank r-1's output columns back to the host.
+// Virtual rank r owns heads [r*Hl, (r+1)*Hl) after the all-to-all, and each
+// head's share of the layer (mode 0 into a head slab, attention on it, mode 1
+// back into that head's columns of O_S) reads and writes nothing of the other
+// heads.  The host path therefore streams the layer by groups of heads inside
+// each rank: the copy of group g+1's head columns to the device overlaps
+// group g's kernels, which overlap the copy of group g-1's output columns
+// back to the host.
 
 }  // namespace
 
@@ -135,13 +136,14 @@ namespace ulysses {
 
 // Two copy streams (host->device, device->host) and the events that order
 // them against the caller's stream: start, one input and one output event per
-// rank, done.  Owned by the plan, created by its first host-buffer call.
+// head group, done.  Owned by the plan, created by its first host-buffer call.
 struct HostPipe {
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t start = nullptr, done = nullptr;
   cudaEvent_t* in = nullptr;
   cudaEvent_t* out = nullptr;
-  int32_t n = 0;
+  int32_t n = 0;            // events per array (= head groups)
+  int32_t group_heads = 0;  // heads per group (divides Hl)
 };
 
 }  // namespace ulysses
@@ -166,20 +168,41 @@ void destroy_pipe(ulysses::HostPipe* h) {
   cudaGetLastError();
 }
 
+// Heads per group: the smallest divisor of Hl whose attention launch still
+// fills every SM about three times over (256-row work units per head, as the
+// attention kernel tiles them), so the groups stay efficient while the
+// pipeline's fill and drain (one group's copy in, one group's kernels and
+// copy out) stay short.
+int32_t host_group_heads(const ulysses_plan_t* p, int sms) {
+  int64_t units_per_head = 0;
+  for (int32_t s = 0; s < p->num_seqs; ++s) {
+    const int64_t q_end = (p->segs[s].end == p->N) ? p->Np : p->segs[s].end;
+    if (p->segs[s].end > p->segs[s].start) units_per_head += (q_end - p->segs[s].start + 255) / 256;
+  }
+  for (int32_t d = 1; d < p->Hl; ++d)
+    if (p->Hl % d == 0 && d * units_per_head >= 3 * static_cast<int64_t>(sms)) return d;
+  return p->Hl;
+}
+
 // The plan's pipe, created on first use (call with g_pipe_mutex held, on the plan's device).
 ulysses::HostPipe* plan_pipe(const ulysses_plan_t* p) {
   if (p->pipe) return p->pipe;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   ulysses::HostPipe* h = new (std::nothrow) ulysses::HostPipe;
   if (!h) return nullptr;
-  h->in = new (std::nothrow) cudaEvent_t[p->P]();
-  h->out = new (std::nothrow) cudaEvent_t[p->P]();
+  h->group_heads = host_group_heads(p, sms);
+  const int32_t groups = p->H / h->group_heads;
+  h->in = new (std::nothrow) cudaEvent_t[groups]();
+  h->out = new (std::nothrow) cudaEvent_t[groups]();
   bool ok = h->in && h->out;
-  if (ok) h->n = p->P;
+  if (ok) h->n = groups;
   ok = ok && cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking) == cudaSuccess;
   ok = ok && cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking) == cudaSuccess;
   ok = ok && cudaEventCreateWithFlags(&h->start, cudaEventDisableTiming) == cudaSuccess;
   ok = ok && cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming) == cudaSuccess;
-  for (int32_t i = 0; ok && i < p->P; ++i) {
+  for (int32_t i = 0; ok && i < groups; ++i) {
     ok = cudaEventCreateWithFlags(&h->in[i], cudaEventDisableTiming) == cudaSuccess &&
          cudaEventCreateWithFlags(&h->out[i], cudaEventDisableTiming) == cudaSuccess;
   }
@@ -191,11 +214,12 @@ ulysses::HostPipe* plan_pipe(const ulysses_plan_t* p) {
   return h;
 }
 
-// Copy rank r's head columns of the sequence-sharded input (every token and
-// plane) between host and device; both sides use the plan's strides.
-cudaError_t copy_rank_input(const ulysses_plan_t* p, int32_t r, const uint8_t* host, uint8_t* dev, cudaStream_t s) {
-  const size_t width = static_cast<size_t>(p->Hl) * p->D * 2;
-  const size_t off = static_cast<size_t>(r) * width;
+// Copy the columns of heads [h0, h0 + hg) of the sequence-sharded input
+// (every token and plane) from host to device; both sides use the plan's strides.
+cudaError_t copy_heads_in(const ulysses_plan_t* p, int32_t h0, int32_t hg, const uint8_t* host, uint8_t* dev,
+                          cudaStream_t s) {
+  const size_t width = static_cast<size_t>(hg) * p->D * 2;
+  const size_t off = static_cast<size_t>(h0) * p->D * 2;
   const size_t tok = static_cast<size_t>(p->token_stride) * 2, pl = static_cast<size_t>(p->plane_stride) * 2;
   if (p->C == 1 || p->token_stride == static_cast<int64_t>(p->C) * p->plane_stride)   // rows (n, c) at pitch pl
     return cudaMemcpy2DAsync(dev + off, pl, host + off, pl, width, static_cast<size_t>(p->Np) * p->C,
@@ -212,22 +236,23 @@ cudaError_t copy_rank_input(const ulysses_plan_t* p, int32_t r, const uint8_t* h
   return cudaSuccess;
 }
 
-// Rank r's share of the layer on `st`: its heads of every token in S, its
-// head columns of O_S.  The kernels see the rank's slabs as a one-rank
-// problem (P = 1, H = Hl) at offset pointers.
-int rank_layer_impl(const ulysses_plan_t* p, int32_t r, const uint8_t* S, uint8_t* OS, uint8_t* T, uint8_t* OT,
-                    int32_t fused, float scale, cudaStream_t st) {
-  const int64_t head_cols = static_cast<int64_t>(p->Hl) * p->D;      // elements of one rank's heads in a row
+// The layer for heads [h0, h0 + hg) (inside one rank) on `st`: their columns
+// of S in, their columns of O_S out.  The kernels see the group as a one-rank
+// problem (P = 1, H = hg) at offset pointers; with fused = 0 its head slab and
+// attention output live in the caller's workspace at Tg / OTg.
+int group_layer_impl(const ulysses_plan_t* p, int32_t h0, int32_t hg, const uint8_t* S, uint8_t* OS, uint8_t* Tg,
+                     uint8_t* OTg, int32_t fused, float scale, cudaStream_t st) {
+  const int64_t cols = static_cast<int64_t>(hg) * p->D;   // elements of the group's heads in a row
   const int64_t row = static_cast<int64_t>(p->H) * p->D;
-  const uint8_t* Sr = S + r * head_cols * 2;
-  uint8_t* OSr = OS + r * head_cols * 2;
+  const uint8_t* Sg = S + static_cast<int64_t>(h0) * p->D * 2;
+  uint8_t* OSg = OS + static_cast<int64_t>(h0) * p->D * 2;
   ulysses::AttnLaunch a;
   a.fused = fused;
   a.Np = p->Np;
   a.N = p->N;
-  a.H = p->Hl;
+  a.H = hg;
   a.P = 1;
-  a.Hl = p->Hl;
+  a.Hl = hg;
   a.C = p->C;
   a.tok_stride = p->token_stride;
   a.plane_stride = p->plane_stride;
@@ -235,27 +260,25 @@ int rank_layer_impl(const ulysses_plan_t* p, int32_t r, const uint8_t* S, uint8_
   a.scale = scale;
   a.plan = p;
   if (fused) {
-    a.base = Sr;
-    a.out = OSr;
-    a.o_stride_r = head_cols;
+    a.base = Sg;
+    a.out = OSg;
+    a.o_stride_r = cols;
     a.o_stride_n = row;
     return status_of(ulysses::launch_attn(a, st));
   }
-  uint8_t* Tr = T + r * static_cast<int64_t>(p->C) * p->Np * head_cols * 2;
-  uint8_t* OTr = OT + r * p->Np * head_cols * 2;
   for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
     const int32_t cc = std::min(p->plane_chunk, p->C - c0);
-    int s = status_of(ulysses::launch_repack(0, Sr, Tr, p->Np, p->Hl, 1, p->C, c0, cc, p->token_stride,
+    int s = status_of(ulysses::launch_repack(0, Sg, Tg, p->Np, hg, 1, p->C, c0, cc, p->token_stride,
                                              p->plane_stride, st));
     if (s != ULYSSES_OK) return s;
   }
-  a.base = Tr;
-  a.out = OTr;
-  a.o_stride_r = p->Np * head_cols;
-  a.o_stride_n = head_cols;
+  a.base = Tg;
+  a.out = OTg;
+  a.o_stride_r = p->Np * cols;
+  a.o_stride_n = cols;
   int s = status_of(ulysses::launch_attn(a, st));
   if (s != ULYSSES_OK) return s;
-  return status_of(ulysses::launch_repack(1, OTr, OSr, p->Np, p->Hl, 1, 1, 0, 1, row, row, st));
+  return status_of(ulysses::launch_repack(1, OTg, OSg, p->Np, hg, 1, 1, 0, 1, row, row, st));
 }
 
 }  // namespace
@@ -613,23 +636,29 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
   uint8_t* hout = static_cast<uint8_t*>(host_out_seq);
   uint8_t* din = static_cast<uint8_t*>(dev_qkv_seq);
   uint8_t* dout = static_cast<uint8_t*>(dev_out_seq);
-  const size_t width = static_cast<size_t>(plan->Hl) * plan->D * 2, pitch = static_cast<size_t>(plan->H) * plan->D * 2;
 
   std::lock_guard<std::mutex> lock(g_pipe_mutex);
   ulysses::HostPipe* h = plan_pipe(plan);
   if (!h) return ULYSSES_ERR_CUDA;
+  const int32_t hg = h->group_heads, groups = h->n;
+  const size_t width = static_cast<size_t>(hg) * plan->D * 2, pitch = static_cast<size_t>(plan->H) * plan->D * 2;
+  const int64_t t_bytes = static_cast<int64_t>(plan->C) * plan->Np * hg * plan->D * 2;   // one group's head slab
+  const int64_t o_bytes = plan->Np * static_cast<int64_t>(hg) * plan->D * 2;
   // the copies start after everything already queued on the caller's stream
   if (cudaEventRecord(h->start, st) != cudaSuccess || cudaStreamWaitEvent(h->h2d, h->start, 0) != cudaSuccess)
     return status_of(cudaErrorUnknown);
-  for (int32_t r = 0; r < plan->P; ++r) {
-    if (copy_rank_input(plan, r, hin, din, h->h2d) != cudaSuccess || cudaEventRecord(h->in[r], h->h2d) != cudaSuccess)
+  for (int32_t g = 0; g < groups; ++g) {
+    if (copy_heads_in(plan, g * hg, hg, hin, din, h->h2d) != cudaSuccess ||
+        cudaEventRecord(h->in[g], h->h2d) != cudaSuccess)
       return status_of(cudaErrorUnknown);
   }
-  for (int32_t r = 0; r < plan->P; ++r) {
-    if (cudaStreamWaitEvent(st, h->in[r], 0) != cudaSuccess) return status_of(cudaErrorUnknown);
-    if ((s = rank_layer_impl(plan, r, din, dout, T, OT, fused, scale, st)) != ULYSSES_OK) return s;
-    if (cudaEventRecord(h->out[r], st) != cudaSuccess || cudaStreamWaitEvent(h->d2h, h->out[r], 0) != cudaSuccess ||
-        cudaMemcpy2DAsync(hout + r * width, pitch, dout + r * width, pitch, width, static_cast<size_t>(plan->Np),
+  for (int32_t g = 0; g < groups; ++g) {
+    if (cudaStreamWaitEvent(st, h->in[g], 0) != cudaSuccess) return status_of(cudaErrorUnknown);
+    uint8_t* Tg = fused ? nullptr : T + g * t_bytes;
+    uint8_t* OTg = fused ? nullptr : OT + g * o_bytes;
+    if ((s = group_layer_impl(plan, g * hg, hg, din, dout, Tg, OTg, fused, scale, st)) != ULYSSES_OK) return s;
+    if (cudaEventRecord(h->out[g], st) != cudaSuccess || cudaStreamWaitEvent(h->d2h, h->out[g], 0) != cudaSuccess ||
+        cudaMemcpy2DAsync(hout + g * width, pitch, dout + g * width, pitch, width, static_cast<size_t>(plan->Np),
                           cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess)
       return status_of(cudaErrorUnknown);
   }

@@ -26,6 +26,7 @@ CASES = [
     pytest.param(2, 1000, 4, [0, 300, 301, 777, 1000], False, 3, id="varlen"),
     pytest.param(2, 1024, 8, None, True, 4, id="causal"),
     pytest.param(2, 700, 4, [0, 256, 300, 700], True, 5, id="causal-varlen"),
+    pytest.param(2, 1000, 4, [0, 0, 300, 300, 1000], False, 6, id="varlen-empty-segments"),
 ]
 
 
@@ -81,6 +82,8 @@ def test_attention_backward_against_oracle(gpu, P, N, H, cu, causal, seed):
     for r in range(P):
         for j in range(Hl):
             for a, b in segs:
+                if b == a:
+                    continue
                 z = scale * (q[r, a:b, j] @ k[r, a:b, j].T) / math.log(2.0)
                 if causal:
                     z = np.where(np.arange(b - a)[None, :] > np.arange(b - a)[:, None], -np.inf, z)

@@ -25,6 +25,7 @@ CASES = [
     pytest.param(2, 640, 4, 3, "plane", None, 8, id="plane-major-P2"),
     pytest.param(2, 1000, 4, 3, "token", [0, 300, 301, 777, 1000], 9, id="varlen-4seq"),
     pytest.param(8, 2048, 16, 3, "token", [0, 1024, 1536, 2048], 10, id="varlen-P8"),
+    pytest.param(2, 1000, 4, 3, "token", [0, 300, 300, 777, 1000, 1000], 37, id="varlen-empty-segments"),
     pytest.param(1, 1, 1, 3, "token", None, 11, id="N1"),
     pytest.param(4, 5, 4, 3, "token", None, 12, id="N5-P4"),
 ]
@@ -115,6 +116,7 @@ CAUSAL_CASES = [
     pytest.param(1, 300, 2, None, 15, id="causal-P1"),
     pytest.param(2, 1000, 4, [0, 300, 301, 777, 1000], 16, id="causal-varlen"),
     pytest.param(2, 700, 4, [0, 256, 512, 700], 17, id="causal-varlen-aligned"),
+    pytest.param(2, 700, 4, [0, 0, 256, 256, 700], 18, id="causal-varlen-empty-segments"),
 ]
 
 

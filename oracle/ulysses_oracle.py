@@ -195,7 +195,7 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) ->
 
 def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
                     rows: np.ndarray | None = None, workers: int = 1,
-                    row_block: int = 256, causal: bool = False) -> np.ndarray:
+                    row_block: int = 256, causal: bool = False, decode=None) -> np.ndarray:
     """Step two of the layer: attention on every head-sharded slab.
 
     T: head-sharded ``[P, C, Np, Hl, D]`` uint16; planes 0, 1, 2 are Q, K, V
@@ -211,7 +211,12 @@ def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
     ``rows`` is None).  Query rows are independent, so they are evaluated
     ``row_block`` at a time to bound memory, and ``workers`` threads may take
     different (rank, head) slabs; neither changes any arithmetic.
+
+    ``decode`` maps the stored codes to fp64: bf16 bit patterns by default,
+    :func:`e4m3_bits_to_f64` for the FP8 variant.
     """
+    if decode is None:
+        decode = bf16_bits_to_f64
     P, C, Np, Hl, D = T.shape
     if C < 3:
         raise ValueError("need Q, K and V planes")
@@ -228,17 +233,17 @@ def attention_heads(T: np.ndarray, N: int, scale: float, cu_seqlens=None,
             sel = np.nonzero(seg_of == s)[0]
             if sel.size == 0:
                 continue
-            k = bf16_bits_to_f64(T[r, 1, a:b, j, :])
-            v = bf16_bits_to_f64(T[r, 2, a:b, j, :])
+            k = decode(T[r, 1, a:b, j, :])
+            v = decode(T[r, 2, a:b, j, :])
             if causal:
                 for i in sel:
                     n = int(rows[i])
-                    q = bf16_bits_to_f64(T[r, 0, n:n + 1, j, :])
+                    q = decode(T[r, 0, n:n + 1, j, :])
                     out[r, i, j, :] = attention_rows(q, k[:n + 1 - a], v[:n + 1 - a], scale)[0]
                 continue
             for i0 in range(0, sel.size, row_block):
                 part = sel[i0:i0 + row_block]
-                q = bf16_bits_to_f64(T[r, 0, rows[part], j, :])
+                q = decode(T[r, 0, rows[part], j, :])
                 out[r, part, j, :] = attention_rows(q, k, v, scale)
 
     slabs = [(r, j) for r in range(P) for j in range(Hl)]
@@ -307,6 +312,82 @@ def attention_flops(N: int, H: int, D: int, cu_seqlens=None, causal: bool = Fals
 def softmax_scale(D: int) -> float:
     """1/sqrt(D): the scale of the Ulysses layer (1/sqrt(128) for D = 128)."""
     return 1.0 / math.sqrt(D)
+
+
+# ---------------------------------------------------------------------------
+# FP8 variant: Q, K and V cast to E4M3 before attention
+# ---------------------------------------------------------------------------
+#
+# The layer page's MiniMax-H3 recipe (the TensorRT-LLM commit quoted on
+# "Ulysses context parallelism", prime-rl pull request) runs cuDNN FP8
+# attention with a "fused FP8 QK cast", and FA4's FP8 P V path
+# (FA4_FP8_PV_USE_FUSED_PACK in the FA4 JIT-cache test of "hao-ai-lab
+# FastVideo, compare aryan/h3-nvfp4-stack-speedups...main").  The pages fix no
+# scaling recipe; the plainest reading of "cast" is a direct conversion of each
+# bf16 value to the nearest E4M3 value (no scale factor), which the N(0,1)
+# inputs fit comfortably.  The attention is then the same softmax attention on
+# the cast values.
+#
+# E4M3 (the OCP 8-bit floating-point format "E4M3"): 1 sign bit, 4 exponent
+# bits with bias 7, 3 mantissa bits; exponent field 0 encodes subnormals
+# m/8 * 2^-6; exponent 15 with mantissa 7 is NaN (no infinities), so the
+# largest finite magnitude is 1.75 * 2^8 = 448.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Decode E4M3 codes (uint8) to fp64, from the format's definition."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 0xF) & ((b & 7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def _e4m3_table():
+    codes = np.arange(0x7F, dtype=np.uint8)          # non-negative finite codes, increasing value
+    return codes, e4m3_bits_to_f64(codes)
+
+
+def f64_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest E4M3 value, ties to the even code, saturating.
+
+    Magnitudes above 448 become 448 (the "satfinite" conversion); the sign is
+    kept, so negative values that round to zero give the code 0x80.  NaN maps
+    to 0x7F.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    codes, vals = _e4m3_table()
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(vals, a, side="left"), 0, vals.size - 1)   # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - vals[lo], vals[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (codes[hi] % 2 == 0))
+    c = np.where(pick_hi, codes[hi], codes[lo]).astype(np.uint8)
+    c = np.where(np.signbit(x), c | np.uint8(0x80), c).astype(np.uint8)
+    return np.where(np.isnan(x), np.uint8(0x7F), c).astype(np.uint8)
+
+
+def repack_fwd_fp8(S: np.ndarray, P: int) -> np.ndarray:
+    """Mode 0 with the cast: ``[Np, C, H, D]`` bf16 bits -> ``[P, C, Np, Hl, D]`` E4M3 codes.
+
+    The cast is elementwise, so it commutes with the index map: this is the
+    bf16 repack followed by the conversion of every element.
+    """
+    return f64_to_e4m3_bits(bf16_bits_to_f64(repack_fwd(S, P)))
+
+
+def layer_fwd_fp8(S: np.ndarray, P: int, N: int, scale: float, cu_seqlens=None,
+                  rows: np.ndarray | None = None, workers: int = 1, causal: bool = False) -> np.ndarray:
+    """The FP8 layer: repack with the E4M3 cast, attention on the cast values
+    (exact, fp64), inverse repack of the output."""
+    T8 = repack_fwd_fp8(S, P)
+    O = attention_heads(T8, N, scale, cu_seqlens=cu_seqlens, rows=rows, workers=workers, causal=causal,
+                        decode=e4m3_bits_to_f64)
+    return output_repack_bwd(O)
 
 
 # ---------------------------------------------------------------------------

@@ -464,3 +464,74 @@ def test_sampled_backward_equals_full_rows(causal):
     assert np.allclose(sq, dq[qr], rtol=0, atol=1e-12)
     assert np.allclose(sk, dk[kr], rtol=0, atol=1e-12)
     assert np.allclose(sv, dv[kr], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) cast
+
+def test_e4m3_decode_known_codes():
+    # values fixed by the format: bias 7, 3 mantissa bits, subnormals below 2^-6, max 448
+    table = {0x00: 0.0, 0x38: 1.0, 0x40: 2.0, 0x3C: 1.5, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x01: 2.0 ** -9,
+             0x07: 7 * 2.0 ** -9, 0x0F: 1.875 * 2.0 ** -6, 0xB8: -1.0, 0xFE: -448.0, 0x30: 0.5}
+    codes = np.array(list(table), dtype=np.uint8)
+    np.testing.assert_array_equal(orc.e4m3_bits_to_f64(codes), np.array(list(table.values())))
+    assert np.isnan(orc.e4m3_bits_to_f64(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+
+
+def test_e4m3_encode_rounding_ties_and_saturation():
+    cases = [
+        (1.0625, 0x38),        # halfway 1 / 1.125: even code (mantissa 0)
+        (1.1875, 0x3A),        # halfway 1.125 / 1.25: even code 1.25
+        (1.0624, 0x38), (1.0626, 0x39),
+        (2.0 ** -10, 0x00),    # halfway 0 / 2^-9: even code 0
+        (3 * 2.0 ** -10, 0x02),  # halfway 2^-9 / 2^-8: even code 2^-8
+        (464.0, 0x7E), (1e6, 0x7E), (-1e6, 0xFE),   # saturation to +-448
+        (-2.0 ** -11, 0x80),   # negative underflow keeps the sign
+        (240.0, 0x77), (0.3, 0x2A),
+    ]
+    x = np.array([c[0] for c in cases])
+    np.testing.assert_array_equal(orc.f64_to_e4m3_bits(x), np.array([c[1] for c in cases], dtype=np.uint8))
+    assert orc.f64_to_e4m3_bits(np.array([np.nan]))[0] == 0x7F
+
+
+def test_e4m3_round_trip_every_code_and_monotone():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = orc.e4m3_bits_to_f64(codes)
+    back = orc.f64_to_e4m3_bits(vals)
+    np.testing.assert_array_equal(orc.e4m3_bits_to_f64(back), vals)
+    np.testing.assert_array_equal(back[codes != 0x80], codes[codes != 0x80])
+    xs = np.linspace(-500, 500, 20001)
+    dec = orc.e4m3_bits_to_f64(orc.f64_to_e4m3_bits(xs))
+    assert np.all(np.diff(dec) >= 0)
+    # nearest: no representable value is closer than the chosen one
+    allv = orc.e4m3_bits_to_f64(np.arange(0x7F, dtype=np.uint8))
+    a = np.abs(xs[np.abs(xs) <= 448])
+    chosen = np.abs(orc.e4m3_bits_to_f64(orc.f64_to_e4m3_bits(a)))
+    best = np.min(np.abs(allv[None, :] - a[:, None]), axis=1)
+    np.testing.assert_allclose(np.abs(chosen - a), best, rtol=0, atol=0)
+
+
+def test_e4m3_cast_of_bf16_values_matches_torch():
+    torch = pytest.importorskip("torch")
+    if not hasattr(torch, "float8_e4m3fn"):
+        pytest.skip("torch without float8_e4m3fn")
+    rng = np.random.default_rng(11)
+    bits = _bf16_normal(rng, (4096,), scale=3.0)
+    x = orc.bf16_bits_to_f64(bits)
+    x = x[np.abs(x) <= 448]
+    want = torch.tensor(x, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(orc.f64_to_e4m3_bits(x), want)
+
+
+def test_fp8_layer_is_exact_attention_on_cast_values():
+    # the FP8 layer equals the bf16 layer's oracle run on inputs that are already
+    # E4M3 values (the cast is then the identity), and the cast commutes with mode 0
+    rng = np.random.default_rng(12)
+    P, N, H, C = 2, 200, 4, 3
+    S = _bf16_normal(rng, (N, C, H, 128))
+    S8 = orc.f64_to_e4m3_bits(orc.bf16_bits_to_f64(S))
+    S_exact = orc.f64_to_bf16_bits(orc.e4m3_bits_to_f64(S8))       # E4M3 values are bf16 values
+    np.testing.assert_array_equal(orc.e4m3_bits_to_f64(S8), orc.bf16_bits_to_f64(S_exact))
+    scale = 1.0 / math.sqrt(128)
+    np.testing.assert_allclose(orc.layer_fwd_fp8(S, P, N, scale), orc.layer_fwd(S_exact, P, N, scale),
+                               rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(orc.repack_fwd_fp8(S, P), orc.repack_fwd(S8.view(np.uint8), P))

@@ -37,8 +37,10 @@ WORKLOADS = {
     "prof8k": (4, 8192, 56, 3, 1, None),   # small case for profiler captures (352 MB input > L2)
     "stress250k": (4, 250_000, 56, 4, 4, None),   # repack fwd + bwd only, plus an N sweep
     "dit19k-causal": (4, 19_394, 56, 3, 1, None),
+    "dit19k-fp8": (4, 19_394, 56, 3, 1, None),
 }
 CAUSAL = {"dit19k-causal"}
+FP8 = {"dit19k-fp8"}
 SWEEP_N = (4096, 8192, 16384, 32768, 65536, 131072, 250_000)
 WORKLOAD_TEXT = {
     "tiny": "Tiny Ulysses layer P=2 N=1024 H=8 D=128 packed QKV bf16",
@@ -50,6 +52,8 @@ WORKLOAD_TEXT = {
     "stress250k": "Repack stress P=4 N=250000 H=56 D=128 packed QKVG bf16, one 896,000,000-byte plane per rank "
                   "per launch; repack fwd+bwd; N sweep 4096..250000",
     "dit19k-causal": "Video-DiT geometry with causal attention P=4 N=19394 H=56 D=128 packed QKV bf16",
+    "dit19k-fp8": "Video-DiT geometry, FP8 variant: Q/K/V cast to E4M3 in the repack, E4M3 attention, "
+                  "P=4 N=19394 H=56 D=128 packed QKV bf16 in and out",
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
@@ -339,6 +343,126 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def run_fp8(args, rank, world, local_rank):
+    """The FP8 layer: repack with the E4M3 cast -> E4M3 attention -> inverse repack (bf16 output)."""
+    import torch
+    import torch.distributed as dist
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    P, N, H, C, seed, cu = WORKLOADS[args.config]
+    Hl = H // P
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu)
+    Np = plan.padded_tokens
+    S = inputs.qkv_seq(N, H, P, C, seed, dev)
+    T8 = torch.empty((P, C, Np, Hl, 128), dtype=torch.uint8, device=dev)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    scale = 1.0 / math.sqrt(128)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        U.ulysses_repack_fwd_fp8(plan, S, T8, stream)
+        if evs:
+            evs[1].record(stream)
+        U.ulysses_attn_fwd_fp8(plan, T8, OT, scale, stream)
+        if evs:
+            evs[2].record(stream)
+        U.ulysses_repack_bwd(plan, OT, OS, 1, stream)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    if U.ulysses_last_device_error(plan) != 0:
+        raise RuntimeError("a kernel reported a device error during the timed region")
+    total_ms = start.elapsed_time(stop)
+
+    # end to end: pinned host input -> device, the FP8 layer through the C ABI, output -> pinned host
+    host_in = S.cpu().pin_memory()
+    host_out = torch.empty(OS.shape, dtype=OS.dtype).pin_memory()
+    dev_in = torch.empty_like(S)
+    ws = torch.empty(plan.workspace_bytes_fp8, dtype=torch.uint8, device=dev)
+    ne = max(3, min(args.steps, 10))
+    for _ in range(2):
+        dev_in.copy_(host_in, non_blocking=True)
+        U.ulysses_layer_fwd_fp8(plan, dev_in, OS, ws, stream=stream)
+        host_out.copy_(OS, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ne):
+        dev_in.copy_(host_in, non_blocking=True)
+        U.ulysses_layer_fwd_fp8(plan, dev_in, OS, ws, stream=stream)
+        host_out.copy_(OS, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / ne
+
+    vals = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = vals.tolist()
+    if rank != 0:
+        return None
+    pk, pk_kind = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]        # measured bf16 x the nominal fp8/bf16 ratio (4.5 / 2.25)
+    flops = attn_flops(N, H, cu)
+    at_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    rf_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    rb_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    rf_bytes = C * Np * H * 128 * 3          # read bf16, write E4M3
+    rb_bytes = 2 * Np * H * 128 * 2
+    attn_tflops = flops / (at_ms * 1e-3) / 1e12
+    ms_per_step = total_ms / args.steps
+    return {
+        "metric": "Ulysses layer µs; attn TFLOP/s and repack GB/s vs B200 peak",
+        "value": round(ms_per_step * 1000.0, 2), "unit": "us per layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 attention, bf16 in/out",
+        "data": "synthetic N(0,1) bf16, seeded",
+        "config": {"workload": WORKLOAD_TEXT[args.config], "name": args.config, "P": P, "N": N, "Np": Np, "H": H,
+                   "D": 128, "planes": C, "seed": seed,
+                   "step": "repack_fwd_fp8 + attn_fwd_fp8 + repack_bwd(output), one C-ABI call each",
+                   "replicas": world, "l2": f"inputs larger than L2 ({S.numel() * 2 / 1e6:.0f} MB per step)"},
+        "attn_us": round(at_ms * 1000, 2), "attn_tflops": round(attn_tflops, 1),
+        "repack_fwd_fp8_us": round(rf_ms * 1000, 2),
+        "repack_fwd_fp8_gbs": round(rf_bytes / (rf_ms * 1e-3) / 1e9, 1),
+        "repack_bwd_us": round(rb_ms * 1000, 2), "repack_bwd_gbs": round(rb_bytes / (rb_ms * 1e-3) / 1e9, 1),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<fp8>", "achieved": round(attn_tflops, 1),
+                     "peak": round(fp8_peak, 1), "peak_kind": f"{pk_kind} bf16 burst x 2 (E4M3 dense)",
+                     "unit": "TFLOP/s", "frac": round(attn_tflops / fp8_peak, 3), "traffic": None,
+                     "algorithmic_flops_per_launch": flops},
+        "e2e": {"value": round(e2e_ms * 1000, 2), "unit": "us per layer",
+                "h2d_bytes_per_step": host_in.numel() * 2, "d2h_bytes_per_step": host_out.numel() * 2,
+                "path": "pinned copies around ulysses_layer_fwd_fp8 on one stream"},
+        "gpu_launches": (math.ceil(C / plan.plane_chunk) + 2) * args.steps,
+        "clocks": clocks,
+    }
+
+
 def run_repack_stress(args, rank, world, local_rank):
     """Repack forward + backward at 250k tokens (QKVG), then a GB/s sweep over N."""
     import torch
@@ -525,6 +649,8 @@ def main():
     try:
         if args.config == "stress250k":
             line = run_repack_stress(args, rank, world, local_rank)
+        elif args.config in FP8:
+            line = run_fp8(args, rank, world, local_rank)
         else:
             line = run_ours(args, rank, world, local_rank)
         if line is not None:

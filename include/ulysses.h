@@ -182,6 +182,48 @@ int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* 
 int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, float softmax_scale,
                      void* stream);
 
+/* ---------------------------------------------------------------- FP8 (E4M3) variant
+ * The MiniMax-H3 recipe quoted in the prime-rl pull request "Ulysses context
+ * parallelism" runs cuDNN FP8 attention with a fused FP8 QK cast, and the
+ * layer page's FA4 wrappers have an FP8 P V path (FA4_FP8_PV_USE_FUSED_PACK).
+ * The pages fix no scaling recipe; here the cast is a direct conversion of
+ * each bf16 value of Q, K, V to the nearest E4M3 value (ties to even,
+ * saturating at +-448, no scale factor), the probabilities P are stored as
+ * E4M3 for the second product (they stay below 2^8), and accumulation,
+ * softmax and the output are as in the bf16 path.  Plane 3 (the gate) is cast
+ * and repacked with the others but not attended.
+ */
+
+/*
+ * Mode 0 with the cast: dst_heads_fp8 [P, C, Np, Hl, D] of one-byte E4M3
+ * codes, T8[r, c, n, j, d] = e4m3(S[n, c, r*Hl + j, d]).  Same window rule as
+ * ulysses_repack_fwd.  Errors: ARG (null or overlapping pointers), ALIGN,
+ * CUDA.
+ */
+int ulysses_repack_fwd_fp8(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads_fp8, void* stream);
+
+/*
+ * Step 2 on E4M3 operands: out_heads O_T [P, Np, Hl, D] (bf16) from
+ * qkv_heads_fp8 [P, C, Np, Hl, D] (planes 0, 1, 2 = Q, K, V as E4M3 codes).
+ * Segments and the causal flag as ulysses_attn_fwd.  Errors: ARG, ALIGN,
+ * CUDA.
+ */
+int ulysses_attn_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_heads_fp8, void* out_heads,
+                         float softmax_scale, void* stream);
+
+/* Workspace of ulysses_layer_fwd_fp8: T8 (one byte per element) then O_T (bf16),
+ * each 256-byte aligned. */
+size_t ulysses_workspace_bytes_fp8(const ulysses_plan_t* plan);
+
+/*
+ * The FP8 layer with softmax_scale = 1/sqrt(D): ulysses_repack_fwd_fp8 ->
+ * ulysses_attn_fwd_fp8 -> ulysses_repack_bwd(planes = 1), out_seq O_S
+ * [Np, H, D] bf16 from qkv_seq (bf16, plan strides).  Errors: ARG, ALIGN,
+ * WORKSPACE, CUDA.
+ */
+int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------- training
  * The gradient of the layer.  The FastVideo transport carries gradients back
  * through the inverse map under the forward's plan (_FusedUlyssesA2A.backward

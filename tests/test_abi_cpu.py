@@ -117,9 +117,18 @@ def test_launch_argument_checks_before_any_device_work():
     assert hl(h, 0x30000000, 0x30000000, 0x10000, 0x90000000, None, 0, 1, None) == _lib.ULYSSES_ERR_ARG
     assert hl(h, 0x30000000, 0x20000000, 0x10000, 0x10000, None, 0, 1, None) == _lib.ULYSSES_ERR_ARG
     assert hl(h, 0x30000000, 0x20000000, 0x10000, 0x90000000, None, 0, 3, None) == _lib.ULYSSES_ERR_ARG
+    # FP8 variant
+    assert lib.ulysses_repack_fwd_fp8(h, None, 0x10000, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_repack_fwd_fp8(h, 0x10008, 0x90000000, None) == _lib.ULYSSES_ERR_ALIGN
+    assert lib.ulysses_repack_fwd_fp8(h, 0x10000, 0x10000 + 4096, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_attn_fwd_fp8(h, 0x10000, 0x10000, 0.1, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_attn_fwd_fp8(h, 0x10000, 0x90000000, 0.0, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_layer_fwd_fp8(h, 0x10000, 0x90000000, None, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
+    assert lib.ulysses_workspace_bytes_fp8(h) == ((1024 * 3 * 8 * 128 + 255) // 256 * 256 + 1024 * 8 * 128 * 2)
     # a gate-less plan cannot run attention
     p2 = U.ulysses_plan(1024, 8, 128, 2, 2)
     assert lib.ulysses_attn_fwd(p2.handle, 0x10000, 0x90000000, 0.1, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_attn_fwd_fp8(p2.handle, 0x10000, 0x90000000, 0.1, None) == _lib.ULYSSES_ERR_ARG
 
 
 def test_strerror_covers_every_code():

@@ -132,3 +132,43 @@ def test_full_layer_causal_dit19k(gpu):
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
     lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
     assert np.array_equal(lay, orc.output_repack_bwd(got))
+
+
+def test_full_layer_fp8_dit19k(gpu):
+    """FP8 variant at the Video-DiT size, in the benchmark's call sequence: the
+    cast bit-exact plane by plane, 1024 seeded rows per head against exact
+    attention on the cast values (per-element E4M3 bound of the FP8 parity
+    tests: 2^-4 of the attention of |V| plus 2^-8 of the value plus 2e-3;
+    mean-abs 2e-3)."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    P, N, H, C, seed = 4, 19_394, 56, 3, 1
+    plan = U.ulysses_plan(N, H, 128, P, C)
+    Np, Hl = plan.padded_tokens, H // P
+    S = inputs.qkv_seq(N, H, P, C, seed, gpu)
+    T8 = torch.empty((P, C, Np, Hl, 128), dtype=torch.uint8, device=gpu)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    scale = 1.0 / math.sqrt(128)
+    U.ulysses_repack_fwd_fp8(plan, S, T8)
+    U.ulysses_attn_fwd_fp8(plan, T8, OT, scale)
+    U.ulysses_repack_bwd(plan, OT, OS, 1)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    T8_bits = T8.cpu().numpy()
+    for c in range(C):
+        want = orc.f64_to_e4m3_bits(orc.bf16_bits_to_f64(orc.repack_fwd(inputs.host_bits(S[:, c:c + 1]), P)))
+        assert np.array_equal(T8_bits[:, c:c + 1], want), f"plane {c}"
+    rows = orc.sample_rows(N, 1024, seed)
+    ref = orc.attention_heads(T8_bits, N, scale, rows=rows, workers=_cores(), decode=orc.e4m3_bits_to_f64)
+    T8_bits[:, 2] &= np.uint8(0x7F)
+    A = orc.attention_heads(T8_bits, N, scale, rows=rows, workers=_cores(), decode=orc.e4m3_bits_to_f64)
+    idx = torch.from_numpy(rows).to(gpu)
+    got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.all(err <= 2.0 ** -4 * A + 2.0 ** -8 * np.abs(ref) + 2e-3), float(err.max())
+    assert err.mean() <= MEAN_ABS, err.mean()
+    lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(lay, orc.output_repack_bwd(got))
+    assert not OS[N:].any()

@@ -15,15 +15,18 @@ from ._lib import (  # noqa: F401
     strerror,
     ulysses_attn_bwd,
     ulysses_attn_fwd,
+    ulysses_attn_fwd_fp8,
     ulysses_attn_fwd_lse,
     ulysses_last_device_error,
     ulysses_layer_bwd,
     ulysses_layer_fwd,
+    ulysses_layer_fwd_fp8,
     ulysses_layer_fwd_fused_noalloc,
     ulysses_layer_fwd_host,
     ulysses_plan,
     ulysses_prologue_repack_fwd,
     ulysses_repack_bwd,
     ulysses_repack_fwd,
+    ulysses_repack_fwd_fp8,
     ulysses_selftest_exp2_poly,
 )

@@ -35,7 +35,8 @@ EXPORTS = (
     "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
     "ulysses_layer_fwd_fused_noalloc", "ulysses_selftest_wait_timeout", "ulysses_prologue_repack_fwd",
     "ulysses_lse_bytes", "ulysses_attn_fwd_lse", "ulysses_attn_bwd_workspace_bytes", "ulysses_attn_bwd",
-    "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd",
+    "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd", "ulysses_repack_fwd_fp8", "ulysses_attn_fwd_fp8",
+    "ulysses_workspace_bytes_fp8", "ulysses_layer_fwd_fp8",
 )
 
 
@@ -114,6 +115,14 @@ def load() -> ctypes.CDLL:
         lib.ulysses_layer_fwd_fused_noalloc.restype = ctypes.c_int
         lib.ulysses_selftest_wait_timeout.argtypes = [vp, i64, vp]
         lib.ulysses_selftest_wait_timeout.restype = ctypes.c_int
+        lib.ulysses_repack_fwd_fp8.argtypes = [vp, vp, vp, vp]
+        lib.ulysses_repack_fwd_fp8.restype = ctypes.c_int
+        lib.ulysses_attn_fwd_fp8.argtypes = [vp, vp, vp, ctypes.c_float, vp]
+        lib.ulysses_attn_fwd_fp8.restype = ctypes.c_int
+        lib.ulysses_workspace_bytes_fp8.argtypes = [vp]
+        lib.ulysses_workspace_bytes_fp8.restype = sz
+        lib.ulysses_layer_fwd_fp8.argtypes = [vp, vp, vp, vp, sz, vp]
+        lib.ulysses_layer_fwd_fp8.restype = ctypes.c_int
         lib.ulysses_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
         lib.ulysses_selftest_exp2_poly.restype = ctypes.c_int
         _handle = lib
@@ -177,6 +186,10 @@ class Plan:
     @property
     def workspace_bytes(self) -> int:
         return load().ulysses_workspace_bytes(self.handle)
+
+    @property
+    def workspace_bytes_fp8(self) -> int:
+        return load().ulysses_workspace_bytes_fp8(self.handle)
 
     @property
     def lse_bytes(self) -> int:
@@ -271,6 +284,24 @@ def ulysses_repack_bwd(plan: Plan, src_heads, dst_seq, planes: int, stream=None)
 def ulysses_attn_fwd(plan: Plan, qkv_heads, out_heads, softmax_scale: float, stream=None) -> None:
     _check(load().ulysses_attn_fwd(plan.handle, _ptr(qkv_heads), _ptr(out_heads), float(softmax_scale),
                                    _stream(stream)), "ulysses_attn_fwd")
+
+
+def ulysses_repack_fwd_fp8(plan: Plan, src_seq, dst_heads_fp8, stream=None) -> None:
+    _check(load().ulysses_repack_fwd_fp8(plan.handle, _ptr(src_seq), _ptr(dst_heads_fp8), _stream(stream)),
+           "ulysses_repack_fwd_fp8")
+
+
+def ulysses_attn_fwd_fp8(plan: Plan, qkv_heads_fp8, out_heads, softmax_scale: float, stream=None) -> None:
+    _check(load().ulysses_attn_fwd_fp8(plan.handle, _ptr(qkv_heads_fp8), _ptr(out_heads), float(softmax_scale),
+                                       _stream(stream)), "ulysses_attn_fwd_fp8")
+
+
+def ulysses_layer_fwd_fp8(plan: Plan, qkv_seq, out_seq, workspace, workspace_bytes: int | None = None,
+                          stream=None) -> None:
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().ulysses_layer_fwd_fp8(plan.handle, _ptr(qkv_seq), _ptr(out_seq), _ptr(workspace),
+                                        int(workspace_bytes), _stream(stream)), "ulysses_layer_fwd_fp8")
 
 
 def ulysses_layer_fwd(plan: Plan, qkv_seq, out_seq, workspace=None, workspace_bytes: int | None = None,

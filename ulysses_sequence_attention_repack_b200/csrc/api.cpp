@@ -36,6 +36,7 @@ inline int64_t heads_bytes(const ulysses_plan_t* p, int32_t planes) {
   return static_cast<int64_t>(p->P) * planes * p->Np * p->Hl * p->D * 2;
 }
 inline int64_t out_seq_bytes(const ulysses_plan_t* p) { return p->Np * p->H * p->D * 2; }
+inline int64_t heads_bytes_fp8(const ulysses_plan_t* p, int32_t planes) { return heads_bytes(p, planes) / 2; }
 
 // Launch-time device check: the plan's error word lives on one device.
 int device_ready(const ulysses_plan_t* p) {
@@ -92,7 +93,7 @@ inline int64_t lse_bytes(const ulysses_plan_t* p) {
 }
 
 int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, float scale, cudaStream_t st,
-              float* lse = nullptr) {
+              float* lse = nullptr, int fp8 = 0) {
   ulysses::AttnLaunch a;
   a.base = base;
   a.fused = fused;
@@ -117,7 +118,18 @@ int attn_impl(const ulysses_plan_t* p, const void* base, int fused, void* out, f
   a.plan = p;
   a.lse = lse;
   a.lse_stride = ulysses::lse_row_stride(p->Np);
+  a.fp8 = fp8;
   return status_of(ulysses::launch_attn(a, st));
+}
+
+int repack_fwd_fp8_impl(const ulysses_plan_t* p, const void* src, void* dst, cudaStream_t st) {
+  for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
+    const int32_t cc = std::min(p->plane_chunk, p->C - c0);
+    int s = status_of(ulysses::launch_repack_fp8(src, dst, p->Np, p->H, p->P, p->C, c0, cc, p->token_stride,
+                                                 p->plane_stride, st));
+    if (s != ULYSSES_OK) return s;
+  }
+  return ULYSSES_OK;
 }
 
 // ---------------------------------------------------------------- host-buffer layer, pipelined by head group
@@ -473,6 +485,56 @@ int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* ou
   int s = device_ready(plan);
   if (s != ULYSSES_OK) return s;
   return attn_impl(plan, qkv_heads, 0, out_heads, softmax_scale, static_cast<cudaStream_t>(stream));
+}
+
+int ulysses_repack_fwd_fp8(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads_fp8, void* stream) {
+  if (!plan || !src_seq || !dst_heads_fp8) return ULYSSES_ERR_ARG;
+  if (!aligned16(src_seq) || !aligned16(dst_heads_fp8)) return ULYSSES_ERR_ALIGN;
+  if (overlap(src_seq, seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride), dst_heads_fp8,
+              heads_bytes_fp8(plan, plan->C)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  return repack_fwd_fp8_impl(plan, src_seq, dst_heads_fp8, static_cast<cudaStream_t>(stream));
+}
+
+int ulysses_attn_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_heads_fp8, void* out_heads, float softmax_scale,
+                         void* stream) {
+  if (!plan || !qkv_heads_fp8 || !out_heads) return ULYSSES_ERR_ARG;
+  if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
+  if (!aligned16(qkv_heads_fp8) || !aligned16(out_heads)) return ULYSSES_ERR_ALIGN;
+  if (overlap(qkv_heads_fp8, heads_bytes_fp8(plan, plan->C), out_heads, heads_bytes(plan, 1))) return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  return attn_impl(plan, qkv_heads_fp8, 0, out_heads, softmax_scale, static_cast<cudaStream_t>(stream), nullptr, 1);
+}
+
+size_t ulysses_workspace_bytes_fp8(const ulysses_plan_t* plan) {
+  if (!plan) return 0;
+  return static_cast<size_t>(align_up(heads_bytes_fp8(plan, plan->C), 256) + align_up(heads_bytes(plan, 1), 256));
+}
+
+int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!plan || !qkv_seq || !out_seq) return ULYSSES_ERR_ARG;
+  if (plan->C < 3) return ULYSSES_ERR_ARG;
+  if (!aligned16(qkv_seq) || !aligned16(out_seq)) return ULYSSES_ERR_ALIGN;
+  const int64_t in_bytes = seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride);
+  if (overlap(qkv_seq, in_bytes, out_seq, out_seq_bytes(plan))) return ULYSSES_ERR_ARG;
+  if (!workspace || workspace_bytes < ulysses_workspace_bytes_fp8(plan)) return ULYSSES_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ULYSSES_ERR_ALIGN;
+  const int64_t ws = static_cast<int64_t>(ulysses_workspace_bytes_fp8(plan));
+  if (overlap(workspace, ws, qkv_seq, in_bytes) || overlap(workspace, ws, out_seq, out_seq_bytes(plan)))
+    return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* T8 = static_cast<uint8_t*>(workspace);
+  uint8_t* OT = T8 + align_up(heads_bytes_fp8(plan, plan->C), 256);
+  if ((s = repack_fwd_fp8_impl(plan, qkv_seq, T8, st)) != ULYSSES_OK) return s;
+  if ((s = attn_impl(plan, T8, 0, OT, 1.0f / std::sqrt(static_cast<float>(plan->D)), st, nullptr, 1)) != ULYSSES_OK)
+    return s;
+  return repack_bwd_impl(plan, OT, out_seq, 1, st);
 }
 
 size_t ulysses_lse_bytes(const ulysses_plan_t* plan) { return plan ? static_cast<size_t>(lse_bytes(plan)) : 0; }

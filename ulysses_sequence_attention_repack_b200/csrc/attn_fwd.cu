@@ -73,16 +73,22 @@ constexpr int BM = 128;            // query rows per tile
 constexpr int BN = 128;            // keys per tile
 constexpr int HD = 128;            // head dim
 constexpr int kUnitRows = 2 * BM;  // query rows per work unit (two tiles)
-constexpr uint32_t kHalfBytes = BM * 64 * 2;   // one 128-row x 64-column swizzled box: 16 KB
-constexpr uint32_t kTileBytes = 2 * kHalfBytes;  // 128 x 128 bf16: 32 KB
+constexpr uint32_t kBoxBytes = BM * 128;  // one TMA box: 128 rows x 128 bytes, 128B-swizzled (16 KB)
 constexpr int kStages = 2;
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s per wait
 
-// shared memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffQ = 0;                                  // [2 tiles][2 halves] 64 KB
-constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;             // [stages] 64 KB
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;       // [stages] 64 KB
-constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+// Tile geometry per element type.  A 128 x 128 tile is two boxes of 64 bf16
+// columns (32 KB) or one box of 128 E4M3 columns (16 KB).
+template <bool kFp8>
+struct Geo {
+  static constexpr int kBoxes = kFp8 ? 1 : 2;
+  static constexpr uint32_t kTileBytes = kBoxes * kBoxBytes;
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr uint32_t kOffQ = 0;                                  // [2 tiles]
+  static constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;             // [stages]
+  static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;       // [stages]
+  static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+};
 // barrier indices
 enum {
   B_QFULL0 = 0, B_QFULL1, B_QEMPTY,
@@ -93,15 +99,21 @@ enum {
   B_PHALF0, B_PHALF1,
   B_DONE, B_COUNT
 };
-constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;           // TMEM base address
-constexpr uint32_t kOffAbort = kOffSlot + 4;
-constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;          // + alignment slack
+template <bool kFp8>
+struct Smem {
+  static constexpr uint32_t kOffBar = Geo<kFp8>::kOffBar;
+  static constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;     // TMEM base address
+  static constexpr uint32_t kOffAbort = kOffSlot + 4;
+  static constexpr uint32_t kBytes = kOffAbort + 4 + 1024;        // + alignment slack
+};
 
 // TMEM columns
 constexpr uint32_t kColS0 = 0, kColO0 = 256;
 
 constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);    // Q, K both K-major (head dim contiguous)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, 0, 1);   // P from TMEM, V MN-major (head dim contiguous)
+constexpr uint32_t kIdescS8 = idesc_e4m3_f32(BM, BN, 0, 0);   // the same for E4M3 operands
+constexpr uint32_t kIdescPV8 = idesc_e4m3_f32(BM, HD, 0, 1);
 
 struct SegDesc {
   int32_t start;       // first query row and first key
@@ -166,6 +178,30 @@ __device__ __forceinline__ void exp_store_half(const float* s, int half, f2 scal
   tmem_st32(tS + 32 * half, pk);
 }
 
+// The E4M3 variant of exp_store_half: the same 64 probabilities, stored as
+// 16 columns of four E4M3 codes at P columns [16 half, 16 half + 16).  The
+// row sum uses the fp32 values.  P stays below 2^8 (the running max moves
+// when it grows by more than 8), inside E4M3's range of 448.
+__device__ __forceinline__ void exp_store_half_fp8(const float* s, int half, f2 scale2, f2 negm2, f2 (&acc)[4],
+                                                   uint32_t tS) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const float* sc = s + 64 * half + 4 * c;
+    const f2 x0 = ffma2(f2{sc[0], sc[1]}, scale2, negm2);
+    const f2 x1 = ffma2(f2{sc[2], sc[3]}, scale2, negm2);
+    f2 e0, e1;
+    e0.x = ex2_approx(x0.x);
+    e0.y = ex2_approx(x0.y);
+    e1.x = ex2_approx(x1.x);
+    e1.y = ex2_approx(x1.y);
+    acc[(2 * c) & 3] = fadd2(acc[(2 * c) & 3], e0);
+    acc[(2 * c + 1) & 3] = fadd2(acc[(2 * c + 1) & 3], e1);
+    pk[c] = pack_e4m3x4(e0.x, e0.y, e1.x, e1.y);
+  }
+  tmem_st16(tS + 16 * half, pk);
+}
+
 // Number of 128-key tiles a unit visits: the whole segment, or (causal) the
 // keys up to the unit's last query row.
 __device__ __forceinline__ int unit_kv_tiles(const AttnParams& p, const SegDesc& sd, const Unit& w) {
@@ -182,8 +218,15 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// kFp8: Q, K, V are E4M3 codes (one byte per element) and P is stored as
+// E4M3 for the P V product; otherwise everything is bf16.
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ AttnParams p) {
+  using G = Geo<kFp8>;
+  constexpr uint32_t kTileBytes = G::kTileBytes;
+  constexpr uint32_t kOffQ = G::kOffQ, kOffK = G::kOffK, kOffV = G::kOffV, kOffBar = G::kOffBar;
+  constexpr uint32_t kOffSlot = Smem<kFp8>::kOffSlot, kOffAbort = Smem<kFp8>::kOffAbort;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -245,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (uc > 0 && !(ok = mbar_wait(BAR(B_QEMPTY), (uc - 1) & 1, g))) break;
         for (int i = 0; i < 2; ++i) {
           mbar_arrive_expect_tx(BAR(B_QFULL0 + i), kTileBytes);
-          for (int h = 0; h < 2; ++h)
-            tma_load_5d(sbase + kOffQ + (2 * i + h) * kHalfBytes, &tmap, BAR(B_QFULL0 + i), 64 * h, hc,
+          for (int h = 0; h < G::kBoxes; ++h)
+            tma_load_5d(sbase + kOffQ + i * kTileBytes + h * kBoxBytes, &tmap, BAR(B_QFULL0 + i), 64 * h, hc,
                         w.q0 + i * BM, 0, rc);
         }
         const int nkv = unit_kv_tiles(p, sd, w);
@@ -256,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t s = kc % kStages, ph = (kc / kStages) & 1;
             if (kc >= kStages && !(ok = mbar_wait(BAR(B_KEMPTY0 + s), ph ^ 1, g))) break;
             mbar_arrive_expect_tx(BAR(B_KFULL0 + s), kTileBytes);
-            for (int h = 0; h < 2; ++h)
-              tma_load_5d(sbase + kOffK + s * kTileBytes + h * kHalfBytes, &tmap, BAR(B_KFULL0 + s), 64 * h, hc,
+            for (int h = 0; h < G::kBoxes; ++h)
+              tma_load_5d(sbase + kOffK + s * kTileBytes + h * kBoxBytes, &tmap, BAR(B_KFULL0 + s), 64 * h, hc,
                           kv0, 1, rc);
             ++kc;
           }
@@ -265,8 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t s = vc % kStages, ph = (vc / kStages) & 1;
             if (vc >= kStages && !(ok = mbar_wait(BAR(B_VEMPTY0 + s), ph ^ 1, g))) break;
             mbar_arrive_expect_tx(BAR(B_VFULL0 + s), kTileBytes);
-            for (int h = 0; h < 2; ++h)
-              tma_load_5d(sbase + kOffV + s * kTileBytes + h * kHalfBytes, &tmap, BAR(B_VFULL0 + s), 64 * h, hc,
+            for (int h = 0; h < G::kBoxes; ++h)
+              tma_load_5d(sbase + kOffV + s * kTileBytes + h * kBoxBytes, &tmap, BAR(B_VFULL0 + s), 64 * h, hc,
                           kv0, 2, rc);
             ++vc;
           }
@@ -289,19 +332,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       // descriptors computed once; each group of 8 MMAs is one asm block
       const uint64_t dQ0 = desc_sw128(sbase + kOffQ, 16, 1024);
-      const uint64_t dQ1 = desc_sw128(sbase + kOffQ + 2 * kHalfBytes, 16, 1024);
+      const uint64_t dQ1 = desc_sw128(sbase + kOffQ + kTileBytes, 16, 1024);
       const uint64_t dK0 = desc_sw128(sbase + kOffK, 16, 1024);
       const uint64_t dK1 = desc_sw128(sbase + kOffK + kTileBytes, 16, 1024);
-      const uint64_t dV0 = desc_sw128(sbase + kOffV, kHalfBytes, 1024);
-      const uint64_t dV1 = desc_sw128(sbase + kOffV + kTileBytes, kHalfBytes, 1024);
+      // V is read MN-major: the leading byte offset steps to the second
+      // 64-column box of a bf16 tile (an E4M3 tile's 128 columns are one box)
+      const uint64_t dV0 = desc_sw128(sbase + kOffV, kBoxBytes, 1024);
+      const uint64_t dV1 = desc_sw128(sbase + kOffV + kTileBytes, kBoxBytes, 1024);
       auto issue_s = [&](int i, uint32_t ks) {
-        mma_ss_k128(tmem + kColS0 + 128 * i, i ? dQ1 : dQ0, ks ? dK1 : dK0, kIdescS, 0);
+        if (kFp8)
+          mma_ss_f8_k128(tmem + kColS0 + 128 * i, i ? dQ1 : dQ0, ks ? dK1 : dK0, kIdescS8, 0);
+        else
+          mma_ss_k128(tmem + kColS0 + 128 * i, i ? dQ1 : dQ0, ks ? dK1 : dK0, kIdescS, 0);
       };
-      // O_i (+)= P_i V over keys [64 h, 64 h + 64): P columns [32 h, 32 h + 32),
-      // V rows 64 h.. (8 KB further in each 64-column atom: +512 descriptor units)
+      // O_i (+)= P_i V over keys [64 h, 64 h + 64): P columns [32 h, 32 h + 32)
+      // (bf16 pairs) or [16 h, 16 h + 16) (E4M3 quads), V rows 64 h.. (8 KB
+      // further in each 128-byte-wide box: +512 descriptor units)
       auto issue_pv_half = [&](int i, uint32_t vs, int h, uint32_t acc) {
-        mma_ts_k64(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 32 * h, (vs ? dV1 : dV0) + 512 * h, kIdescPV,
-                   acc);
+        if (kFp8)
+          mma_ts_f8_k64(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 16 * h, (vs ? dV1 : dV0) + 512 * h,
+                        kIdescPV8, acc);
+        else
+          mma_ts_k64(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 32 * h, (vs ? dV1 : dV0) + 512 * h,
+                     kIdescPV, acc);
       };
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
         Unit w;
@@ -447,14 +500,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // first half is handed to the MMA warp before the second is computed.
         // Masked tiles use MUFU ex2 only, so masked keys give exact zeros.
         const bool emu = !masked;
-        if (emu)
+        if (kFp8)
+          exp_store_half_fp8(s, 0, scale2, negm2, acc, tS);
+        else if (emu)
           exp_store_half<true>(s, 0, scale2, negm2, acc, tS);
         else
           exp_store_half<false>(s, 0, scale2, negm2, acc, tS);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR(B_PHALF0 + wg));
-        if (emu)
+        if (kFp8)
+          exp_store_half_fp8(s, 1, scale2, negm2, acc, tS);
+        else if (emu)
           exp_store_half<true>(s, 1, scale2, negm2, acc, tS);
         else
           exp_store_half<false>(s, 1, scale2, negm2, acc, tS);
@@ -527,6 +584,23 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+template <bool kFp8>
+cudaError_t launch_kernel(const CUtensorMap& tmap, const AttnParams& p, int grid, int dev, cudaStream_t stream) {
+  static bool attr_set[64] = {false};
+  if (dev < 64 && !attr_set[dev]) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<kFp8>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != static_cast<int>(kLaunchRegs)) return cudaErrorInvalidConfiguration;   // see register split
+    e = cudaFuncSetAttribute(attn_fwd_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<kFp8>::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  attn_fwd_kernel<kFp8><<<grid, kThreads, Smem<kFp8>::kBytes, stream>>>(tmap, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
@@ -534,6 +608,8 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   EncodeTiledFn encode = get_encode_fn();
   if (!encode) return cudaErrorNotSupported;
 
+  if (a.fp8 && a.fused) return cudaErrorInvalidValue;   // the E4M3 variant reads head-sharded T8 only
+  const cuuint64_t eb = a.fp8 ? 1 : 2;                  // bytes per element
   // 5-D view (d, head, token, plane, rank) of the Q/K/V source
   cuuint64_t dims[5], strides[4];
   dims[0] = HD;
@@ -542,10 +618,10 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
     dims[2] = a.Np;
     dims[3] = a.C;
     dims[4] = a.P;
-    strides[0] = HD * 2;
-    strides[1] = static_cast<cuuint64_t>(a.Hl) * HD * 2;
-    strides[2] = static_cast<cuuint64_t>(a.Np) * a.Hl * HD * 2;
-    strides[3] = static_cast<cuuint64_t>(a.C) * a.Np * a.Hl * HD * 2;
+    strides[0] = HD * eb;
+    strides[1] = static_cast<cuuint64_t>(a.Hl) * HD * eb;
+    strides[2] = static_cast<cuuint64_t>(a.Np) * a.Hl * HD * eb;
+    strides[3] = static_cast<cuuint64_t>(a.C) * a.Np * a.Hl * HD * eb;
   } else {
     dims[1] = a.H;
     dims[2] = a.Np;
@@ -556,12 +632,14 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
     strides[2] = static_cast<cuuint64_t>(a.plane_stride) * 2;
     strides[3] = std::max<cuuint64_t>(strides[1] * a.Np, strides[2] * a.C);
   }
-  cuuint32_t box[5] = {64, 1, BM, 1, 1};
+  // one box is 128 rows of 128 bytes: 64 bf16 or 128 E4M3 columns
+  cuuint32_t box[5] = {a.fp8 ? 128u : 64u, 1, BM, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap tmap;
-  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(a.base), dims, strides, box,
-                       estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult cr = encode(&tmap, a.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                       const_cast<void*>(a.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
   AttnParams p;
@@ -608,19 +686,8 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set[64] = {false};
-  if (dev < 64 && !attr_set[dev]) {
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_kernel);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != static_cast<int>(kLaunchRegs)) return cudaErrorInvalidConfiguration;   // see register split
-    e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
   const int grid = std::min(units, sms);
-  attn_fwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmap, p);
-  return cudaGetLastError();
+  return a.fp8 ? launch_kernel<true>(tmap, p, grid, dev, stream) : launch_kernel<false>(tmap, p, grid, dev, stream);
 }
 
 }  // namespace ulysses

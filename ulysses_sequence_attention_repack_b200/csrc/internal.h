@@ -39,6 +39,12 @@ namespace ulysses {
 cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
                           int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream);
 
+// Mode 0 with the E4M3 cast (FP8 attention variant) over planes [c0, c0 + cc):
+// head side [P, Ctot, Np, Hl, D] of one-byte codes.
+cudaError_t launch_repack_fp8(const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
+                              int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
+                              cudaStream_t stream);
+
 // Prologue (per-head RMSNorm + partial RoPE on planes 0 and 1) fused with one
 // mode-0 repack launch over planes [c0, c0 + cc).
 cudaError_t launch_prologue_repack(const void* src, void* dst, const void* wq, const void* wk, const void* cos,
@@ -59,6 +65,7 @@ struct AttnLaunch {
   const ulysses_plan_t* plan;
   float* lse = nullptr;          // optional log2-domain LSE output [P*Hl][lse_stride]
   int64_t lse_stride = 0;
+  int fp8 = 0;                   // 1: base holds E4M3 codes [P, C, Np, Hl, D] (fused must be 0)
 };
 
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream);

@@ -98,7 +98,89 @@ __global__ void __launch_bounds__(kRepackThreads) repack_kernel(const int4* __re
   }
 }
 
+// Mode 0 with the E4M3 cast of the FP8 attention variant:
+//   T8[r, c, n, j, d] = e4m3(S[n, c, r*Hl + j, d])
+// Same traversal as repack_kernel<0>; each 16-byte load of 8 bf16 values
+// becomes one 8-byte store of 8 E4M3 codes (round to nearest even,
+// saturating at +-448: cvt.rn.satfinite).
+__device__ __forceinline__ uint32_t e4m3x4(uint32_t w01, uint32_t w23) {
+  uint16_t a, b;
+  // each 32-bit word holds two bf16 values, the lower-indexed one in bits 0-15;
+  // cvt puts its first source in the high byte
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+      : "=h"(a)
+      : "f"(__uint_as_float(w01 & 0xFFFF0000u)), "f"(__uint_as_float(w01 << 16)));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+      : "=h"(b)
+      : "f"(__uint_as_float(w23 & 0xFFFF0000u)), "f"(__uint_as_float(w23 << 16)));
+  return static_cast<uint32_t>(a) | (static_cast<uint32_t>(b) << 16);
+}
+
+__global__ void __launch_bounds__(kRepackThreads) repack_fp8_kernel(const int4* __restrict__ src,
+                                                                    uint2* __restrict__ dst, int64_t Np,
+                                                                    int32_t H, int32_t Hl, int32_t Ctot,
+                                                                    int32_t c0, int32_t cc, int64_t tok_stride,
+                                                                    int64_t plane_stride) {
+  __shared__ int64_t head_off[kMaxHeads];
+  constexpr int D = 128;
+  const int64_t rank_stride = static_cast<int64_t>(Ctot) * Np * Hl * D;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    const int r = h / Hl, j = h - (h / Hl) * Hl;
+    head_off[h] = r * rank_stride + static_cast<int64_t>(j) * D;
+  }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = Np * cc;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int vec_per_row = H * (D / 8);
+
+  for (int64_t row = warp0; row < rows; row += nwarps) {
+    const int c = c0 + static_cast<int>(row / Np);
+    const int64_t n = row - (row / Np) * Np;
+    const int64_t seq_base = n * tok_stride + c * plane_stride;
+    const int64_t head_base = (static_cast<int64_t>(c) * Np + n) * Hl * D;
+    for (int k0 = 0; k0 < vec_per_row; k0 += 32 * kUnroll) {
+      int4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int k = k0 + u * 32 + lane;
+        if (k < vec_per_row) v[u] = ld_stream(src + ((seq_base + static_cast<int64_t>(k) * 8) >> 3));
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int k = k0 + u * 32 + lane;
+        if (k < vec_per_row) {
+          const int64_t head_el = head_base + head_off[k >> 4] + (k & 15) * 8;   // one byte per element
+          uint2 o;
+          o.x = e4m3x4(static_cast<uint32_t>(v[u].x), static_cast<uint32_t>(v[u].y));
+          o.y = e4m3x4(static_cast<uint32_t>(v[u].z), static_cast<uint32_t>(v[u].w));
+          dst[head_el >> 3] = o;
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_repack_fp8(const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
+                              int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
+                              cudaStream_t stream) {
+  if (H > kMaxHeads || P < 1 || H % P != 0) return cudaErrorInvalidValue;
+  const int64_t rows = Np * cc;
+  if (rows == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int warps_per_cta = kRepackThreads / 32;
+  const int64_t want = (rows + warps_per_cta - 1) / warps_per_cta;
+  const int grid = static_cast<int>(want < static_cast<int64_t>(sms) * 8 ? want : static_cast<int64_t>(sms) * 8);
+  repack_fp8_kernel<<<grid, kRepackThreads, 0, stream>>>(static_cast<const int4*>(src), static_cast<uint2*>(dst),
+                                                         Np, H, H / P, Ctot, c0, cc, tok_stride, plane_stride);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
                           int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream) {

@@ -38,9 +38,10 @@ WORKLOADS = {
     "stress250k": (4, 250_000, 56, 4, 4, None),   # repack fwd + bwd only, plus an N sweep
     "dit19k-causal": (4, 19_394, 56, 3, 1, None),
     "dit19k-fp8": (4, 19_394, 56, 3, 1, None),
+    "prof8k-fp8": (4, 8192, 56, 3, 1, None),   # small FP8 case for profiler captures
 }
 CAUSAL = {"dit19k-causal"}
-FP8 = {"dit19k-fp8"}
+FP8 = {"dit19k-fp8", "prof8k-fp8"}
 SWEEP_N = (4096, 8192, 16384, 32768, 65536, 131072, 250_000)
 WORKLOAD_TEXT = {
     "tiny": "Tiny Ulysses layer P=2 N=1024 H=8 D=128 packed QKV bf16",
@@ -52,6 +53,7 @@ WORKLOAD_TEXT = {
     "stress250k": "Repack stress P=4 N=250000 H=56 D=128 packed QKVG bf16, one 896,000,000-byte plane per rank "
                   "per launch; repack fwd+bwd; N sweep 4096..250000",
     "dit19k-causal": "Video-DiT geometry with causal attention P=4 N=19394 H=56 D=128 packed QKV bf16",
+    "prof8k-fp8": "Profiling case, FP8 variant, P=4 N=8192 H=56 D=128 packed QKV bf16 in and out",
     "dit19k-fp8": "Video-DiT geometry, FP8 variant: Q/K/V cast to E4M3 in the repack, E4M3 attention, "
                   "P=4 N=19394 H=56 D=128 packed QKV bf16 in and out",
 }
@@ -453,7 +455,8 @@ def run_fp8(args, rank, world, local_rank):
         "repack_bwd_us": round(rb_ms * 1000, 2), "repack_bwd_gbs": round(rb_bytes / (rb_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<fp8>", "achieved": round(attn_tflops, 1),
                      "peak": round(fp8_peak, 1), "peak_kind": f"{pk_kind} bf16 burst x 2 (E4M3 dense)",
-                     "unit": "TFLOP/s", "frac": round(attn_tflops / fp8_peak, 3), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(attn_tflops / fp8_peak, 3),
+                     "traffic": recorded_traffic("attn_fwd_kernel_fp8", args.config),
                      "algorithmic_flops_per_launch": flops},
         "e2e": {"value": round(e2e_ms * 1000, 2), "unit": "us per layer",
                 "h2d_bytes_per_step": host_in.numel() * 2, "d2h_bytes_per_step": host_out.numel() * 2,

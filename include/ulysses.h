@@ -183,8 +183,9 @@ int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* ou
                      void* stream);
 
 /* ---------------------------------------------------------------- FP8 (E4M3) variant
- * The MiniMax-H3 recipe quoted in the prime-rl pull request "Ulysses context
- * parallelism" runs cuDNN FP8 attention with a fused FP8 QK cast, and the
+ * The MiniMax-H3 recipe branch described on "Request FA4's 2-CTA kernel for
+ * MiniMax-H3 on SM103 and SM107" (TensorRT-LLM pull request 21275) runs
+ * cuDNN FP8 attention with Q and K cast to FP8 in a fused step, and the
  * layer page's FA4 wrappers have an FP8 P V path (FA4_FP8_PV_USE_FUSED_PACK).
  * The pages fix no scaling recipe; here the cast is a direct conversion of
  * each bf16 value of Q, K, V to the nearest E4M3 value (ties to even,

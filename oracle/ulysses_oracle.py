@@ -318,9 +318,10 @@ def softmax_scale(D: int) -> float:
 # FP8 variant: Q, K and V cast to E4M3 before attention
 # ---------------------------------------------------------------------------
 #
-# The layer page's MiniMax-H3 recipe (the TensorRT-LLM commit quoted on
-# "Ulysses context parallelism", prime-rl pull request) runs cuDNN FP8
-# attention with a "fused FP8 QK cast", and FA4's FP8 P V path
+# The MiniMax-H3 recipe branch described on "Request FA4's 2-CTA kernel for
+# MiniMax-H3 on SM103 and SM107" (NVIDIA TensorRT-LLM pull request 21275, its
+# commit merging the recipe branches) runs cuDNN FP8 attention with Q and K
+# cast to FP8 in a fused step, and FA4 has an FP8 P V path
 # (FA4_FP8_PV_USE_FUSED_PACK in the FA4 JIT-cache test of "hao-ai-lab
 # FastVideo, compare aryan/h3-nvfp4-stack-speedups...main").  The pages fix no
 # scaling recipe; the plainest reading of "cast" is a direct conversion of each

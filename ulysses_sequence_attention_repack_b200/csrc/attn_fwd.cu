@@ -30,6 +30,10 @@
 //               of group 1 releases the K/V ring slots.
 // TMEM: S0 | S1 | O0 | O1, 128 fp32 columns each (all 512 columns).
 //
+// FP8 variant (template flag kFp8): Q, K, V arrive as E4M3 codes (cast in the
+// repack), the two products are tcgen05 kind::f8f6f4 MMAs, and P is stored as
+// E4M3 (four codes per TMEM column).  Everything else is shared.
+//
 // Every wait is bounded: on timeout the kernel sets an error bit, skips the
 // remaining work, waits (bounded) for its own in-flight copies and MMAs,
 // frees TMEM and returns.

@@ -79,6 +79,7 @@ struct SegB {
   int32_t tile_end;        // rows this segment's units cover (Np for the segment ending at N)
   int32_t ntile;           // 128-row units per (rank, head)
   int32_t unit_base;
+  int32_t pair_base;       // causal schedule: first pair of units of this segment
 };
 
 struct BwdParams {
@@ -89,6 +90,7 @@ struct BwdParams {
   unsigned int* err;
   int32_t N, Np, Hl, P, causal;
   int32_t num_units, nseg;
+  int32_t num_pairs, paired;   // causal schedule (see unit_of_cta_b)
   float scale, scale_log2;
   SegB seg[ULYSSES_MAX_SEQS];
 };
@@ -109,6 +111,33 @@ __device__ __forceinline__ bool decode_b(const BwdParams& p, int u, UnitB& w) {
   w.j = rh - w.r * p.Hl;
   w.row0 = p.seg[s].start + tb * BT;
   return local >= 0 && w.r < p.P;
+}
+
+// The k-th work unit of this CTA: 1 (w filled), 0 (no units left), 2 (an
+// empty slot: skip), -1 (decodes outside the problem).  With the causal mask
+// a unit's cost is linear in its tile index (pass A: the query blocks at or
+// after its keys; pass B: the key blocks up to its queries), so the tiles of
+// each (segment, rank, head) are paired as (ntile - 1 - i, i), pairs of equal
+// cost, and CTA b takes pairs b, b + G, ...; the middle tile of an odd count
+// leaves an empty slot.  Otherwise CTA b takes units b, b + G, ... .
+__device__ __forceinline__ int unit_of_cta_b(const BwdParams& p, int k, UnitB& w) {
+  if (!p.paired) {
+    const int u = blockIdx.x + k * gridDim.x;
+    if (u >= p.num_units) return 0;
+    return decode_b(p, u, w) ? 1 : -1;
+  }
+  const int pp = blockIdx.x + (k >> 1) * gridDim.x;
+  if (pp >= p.num_pairs) return 0;
+  int s = 0;
+  while (s + 1 < p.nseg && pp >= p.seg[s + 1].pair_base) ++s;
+  const int nt = p.seg[s].ntile;
+  const int half = (nt + 1) >> 1;
+  const int local = pp - p.seg[s].pair_base;
+  const int rh = local / half;
+  const int i = local - rh * half;
+  const int tb = (k & 1) ? i : nt - 1 - i;
+  if ((k & 1) && tb >= nt - 1 - i) return 2;   // the unpaired middle tile
+  return decode_b(p, p.seg[s].unit_base + rh * nt + tb, w) ? 1 : -1;
 }
 
 // Streamed blocks of a unit: pass A visits query blocks [first, start + ceil((end - start)/128)),
@@ -305,9 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t xc = 0, uc = 0, x0c = 0, x1c = 0;   // blocks, units, copies issued per tile barrier
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+      for (int k = 0; ok; ++k) {
         UnitB w;
-        if (!decode_b(p, u, w)) {
+        const int st = unit_of_cta_b(p, k, w);
+        if (st == 0) break;
+        if (st == 2) continue;
+        if (st < 0) {
           atomicOr(p.err, kErrBadUnit);
           break;
         }
@@ -357,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++xc;
         }
+        ++uc;
       }
       // no copy may be in flight when the CTA exits
       if (uc > 0) drain_wait_b(BAR(B_FFULL), (uc - 1) & 1);
@@ -379,9 +412,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto xdesc = [&](uint32_t s, int t, uint32_t lbo) {
         return desc_sw128(sbase + kOffX + s * 2 * kTileBytes + t * kTileBytes, lbo, 1024);
       };
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+      for (int k = 0; ok; ++k) {
         UnitB w;
-        if (!decode_b(p, u, w)) break;
+        const int st = unit_of_cta_b(p, k, w);
+        if (st == 0 || st < 0) break;
+        if (st == 2) continue;
         const SegB& sd = p.seg[w.seg];
         int first, count;
         stream_range<kPassA>(p, sd, w, first, count);
@@ -435,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         xc += count;
         mma_commit(BAR(B_OFULL));
         mma_commit(BAR(B_FEMPTY));
+        ++uc;
       }
       mma_commit(BAR(B_DONE));
       drain_wait_b(BAR(B_DONE), 0);
@@ -453,9 +489,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float* srow = reinterpret_cast<const float*>(smem + kOffRow);
     uint32_t sc = 0, uc = 0, xc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+    for (int k = 0; ok; ++k) {
       UnitB w;
-      if (!decode_b(p, u, w)) break;
+      const int st = unit_of_cta_b(p, k, w);
+      if (st == 0 || st < 0) break;
+      if (st == 2) continue;
       const SegB& sd = p.seg[w.seg];
       const int end = sd.end;
       int first, count;
@@ -572,6 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_OEMPTY));
+      ++uc;
     }
   }
 
@@ -679,7 +718,7 @@ cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
   std::stable_sort(order, order + nseg, [&](int x, int y) {
     return (pl->segs[x].end - pl->segs[x].start) > (pl->segs[y].end - pl->segs[y].start);
   });
-  int units = 0;
+  int units = 0, pairs = 0;
   for (int k = 0; k < nseg; ++k) {
     const ulysses::Segment& sg = pl->segs[order[k]];
     SegB& d = p.seg[k];
@@ -688,10 +727,14 @@ cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
     d.tile_end = (sg.end == pl->N) ? static_cast<int32_t>(Np) : sg.end;
     d.ntile = (d.tile_end - d.start + BT - 1) / BT;
     d.unit_base = units;
+    d.pair_base = pairs;
     units += d.ntile * static_cast<int>(P * Hl);
+    pairs += (d.ntile + 1) / 2 * static_cast<int>(P * Hl);
   }
   p.nseg = nseg;
   p.num_units = units;
+  p.num_pairs = pairs;
+  p.paired = (p.causal && units >= 2 * sms) ? 1 : 0;   // two units per SM at least, or the pairs idle SMs
   if (units == 0) return cudaSuccess;
   cudaError_t e = launch_pass<true>(tq, td, p, sms, stream);    // dK, dV
   if (e != cudaSuccess) return e;

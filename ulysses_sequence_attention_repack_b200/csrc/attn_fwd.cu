@@ -125,6 +125,7 @@ struct SegDesc {
   int32_t q_end;       // one past the last query row this segment writes (Np for the last segment)
   int32_t nqb;         // 256-row query blocks
   int32_t unit_base;   // first work unit of this segment
+  int32_t pair_base;   // causal schedule: first pair of query blocks of this segment
 };
 
 struct AttnParams {
@@ -137,6 +138,8 @@ struct AttnParams {
   int32_t Hl, P, fused;
   int32_t causal;                  // query n sees keys m <= n only
   int32_t num_units, nseg;
+  int32_t num_pairs;               // causal schedule: pairs of query blocks over all segments and heads
+  int32_t paired;                  // 1: the causal pair schedule (enough units for two per CTA)
   float scale_log2;
   SegDesc seg[ULYSSES_MAX_SEQS];   // longest first
 };
@@ -157,6 +160,39 @@ __device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& w)
   w.j = rh - w.r * p.Hl;
   w.q0 = p.seg[s].start + qb * kUnitRows;
   return local >= 0 && w.r < p.P;
+}
+
+// The k-th work unit of this CTA.  Returns 1 with w filled, 0 when the CTA
+// has no units left, 2 for an empty slot of the schedule (skip it), -1 if a
+// unit decodes outside the problem.
+//   Non-causal: every unit of a segment visits the same key tiles, and CTA b
+//   takes units b, b + G, b + 2G, ... (G = gridDim.x).
+//   Causal: a unit visits the key tiles up to its last query row, so its cost
+//   grows with its query block qb.  The blocks of each (segment, rank, head)
+//   are paired as (nqb - 1 - i, i), pairs of equal total cost, and CTA b takes
+//   pairs b, b + G, ... (both units of a pair, the costlier first); the middle
+//   block of an odd count has no partner, which leaves an empty slot.  Plain
+//   round robin would leave the busiest CTA with ~1.2x the average work at
+//   the Video-DiT size.  With fewer than two units per SM the pairs would
+//   idle half the SMs, so small causal problems keep the plain schedule.
+__device__ __forceinline__ int unit_of_cta(const AttnParams& p, int k, Unit& w) {
+  if (!p.paired) {
+    const int u = blockIdx.x + k * gridDim.x;
+    if (u >= p.num_units) return 0;
+    return decode_unit(p, u, w) ? 1 : -1;
+  }
+  const int pp = blockIdx.x + (k >> 1) * gridDim.x;
+  if (pp >= p.num_pairs) return 0;
+  int s = 0;
+  while (s + 1 < p.nseg && pp >= p.seg[s + 1].pair_base) ++s;
+  const int nqb = p.seg[s].nqb;
+  const int half = (nqb + 1) >> 1;
+  const int local = pp - p.seg[s].pair_base;
+  const int rh = local / half;
+  const int i = local - rh * half;
+  const int qb = (k & 1) ? i : nqb - 1 - i;
+  if ((k & 1) && qb >= nqb - 1 - i) return 2;   // the unpaired middle block
+  return decode_unit(p, p.seg[s].unit_base + rh * nqb + qb, w) ? 1 : -1;
 }
 
 // P = exp2(s * scale_log2 - m) for columns [64 half, 64 half + 64) of one row,
@@ -292,9 +328,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kc = 0, vc = 0, uc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+      for (int k = 0; ok; ++k) {
         Unit w;
-        if (!decode_unit(p, u, w)) {
+        const int st = unit_of_cta(p, k, w);
+        if (st == 0) break;
+        if (st == 2) continue;
+        if (st < 0) {
           atomicOr(p.err, kErrBadUnit);
           break;
         }
@@ -330,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++vc;
           }
         }
+        ++uc;
       }
       // drain: every copy this thread issued has landed before the CTA exits
       if (uc > 0) {
@@ -372,9 +412,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts_k64(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 32 * h, (vs ? dV1 : dV0) + 512 * h,
                      kIdescPV, acc);
       };
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+      for (int k = 0; ok; ++k) {
         Unit w;
-        if (!decode_unit(p, u, w)) break;
+        const int st = unit_of_cta(p, k, w);
+        if (st == 0 || st < 0) break;
+        if (st == 2) continue;
         const SegDesc& sd = p.seg[w.seg];
         const int nkv = unit_kv_tiles(p, sd, w);
         if (!(ok = mbar_wait(BAR(B_QFULL0), uc & 1, g))) break;
@@ -418,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           ++vc;
         }
+        ++uc;
       }
       // drain: all MMAs this thread issued are complete before TMEM is freed
       mma_commit(BAR(B_DONE));
@@ -436,9 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t sc = 0, uc = 0;
     uint32_t kslot = 0, vslot = 0;   // K / V ring fills consumed (warpgroup 1 releases them)
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++uc) {
+    for (int k = 0; ok; ++k) {
       Unit w;
-      if (!decode_unit(p, u, w)) break;
+      const int st = unit_of_cta(p, k, w);
+      if (st == 0 || st < 0) break;
+      if (st == 2) continue;
       const SegDesc& sd = p.seg[w.seg];
       const int nkv = unit_kv_tiles(p, sd, w);
       float m_used = -INFINITY;   // running max, log2 units (scaled)
@@ -577,6 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           dst[v] = q;
         }
       }
+      ++uc;
     }
   }
 
@@ -688,7 +734,7 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   std::stable_sort(order, order + nseg, [&](int x, int y) {
     return (pl->segs[x].end - pl->segs[x].start) > (pl->segs[y].end - pl->segs[y].start);
   });
-  int units = 0;
+  int units = 0, pairs = 0;
   for (int k = 0; k < nseg; ++k) {
     const ulysses::Segment& sg = pl->segs[order[k]];
     SegDesc& d = p.seg[k];
@@ -697,15 +743,19 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
     d.q_end = (sg.end == a.N) ? static_cast<int32_t>(a.Np) : sg.end;
     d.nqb = (d.q_end - d.start + kUnitRows - 1) / kUnitRows;
     d.unit_base = units;
+    d.pair_base = pairs;
     units += d.nqb * a.P * a.Hl;
+    pairs += (d.nqb + 1) / 2 * a.P * a.Hl;
   }
   p.nseg = nseg;
   p.num_units = units;
+  p.num_pairs = pairs;
   if (units == 0) return cudaSuccess;
 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  p.paired = (p.causal && units >= 2 * sms) ? 1 : 0;
   const int grid = std::min(units, sms);
   return a.fp8 ? launch_kernel<true>(tmap, p, grid, dev, stream) : launch_kernel<false>(tmap, p, grid, dev, stream);
 }

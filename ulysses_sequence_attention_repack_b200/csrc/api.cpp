@@ -154,8 +154,9 @@ struct HostPipe {
   cudaEvent_t start = nullptr, done = nullptr;
   cudaEvent_t* in = nullptr;
   cudaEvent_t* out = nullptr;
-  int32_t n = 0;            // events per array (= head groups)
-  int32_t group_heads = 0;  // heads per group (divides Hl)
+  int32_t n = 0;            // head groups (events per array)
+  int32_t* h0 = nullptr;    // first head of each group
+  int32_t* hg = nullptr;    // heads of each group (a group never spans two ranks)
 };
 
 }  // namespace ulysses
@@ -176,6 +177,8 @@ void destroy_pipe(ulysses::HostPipe* h) {
   }
   delete[] h->in;
   delete[] h->out;
+  delete[] h->h0;
+  delete[] h->hg;
   delete h;
   cudaGetLastError();
 }
@@ -183,8 +186,7 @@ void destroy_pipe(ulysses::HostPipe* h) {
 // Heads per group: the smallest divisor of Hl whose attention launch still
 // fills every SM about three times over (256-row work units per head, as the
 // attention kernel tiles them), so the groups stay efficient while the
-// pipeline's fill and drain (one group's copy in, one group's kernels and
-// copy out) stay short.
+// pipeline's fill (one group's copy in) stays short.
 int32_t host_group_heads(const ulysses_plan_t* p, int sms) {
   int64_t units_per_head = 0;
   for (int32_t s = 0; s < p->num_seqs; ++s) {
@@ -204,12 +206,35 @@ ulysses::HostPipe* plan_pipe(const ulysses_plan_t* p) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   ulysses::HostPipe* h = new (std::nothrow) ulysses::HostPipe;
   if (!h) return nullptr;
-  h->group_heads = host_group_heads(p, sms);
-  const int32_t groups = p->H / h->group_heads;
+  // Groups of hg heads, except that the last rank tapers (hg, then about
+  // half of what is left each time, down to one head): after the last input
+  // copy only the last, smallest group's kernels and output copy remain, the
+  // pipeline's drain.  A smaller group fills fewer SMs, but the kernels are
+  // waiting for the copies there anyway.
+  const int32_t hg = host_group_heads(p, sms);
+  int32_t groups = (p->P - 1) * (p->Hl / hg);
+  for (int32_t left = p->Hl; left > 0; ++groups) left -= std::min(hg, left > 1 ? (left + 1) / 2 : 1);
   h->in = new (std::nothrow) cudaEvent_t[groups]();
   h->out = new (std::nothrow) cudaEvent_t[groups]();
-  bool ok = h->in && h->out;
-  if (ok) h->n = groups;
+  h->h0 = new (std::nothrow) int32_t[groups];
+  h->hg = new (std::nothrow) int32_t[groups];
+  bool ok = h->in && h->out && h->h0 && h->hg;
+  if (ok) {
+    h->n = groups;
+    int32_t g = 0, head = 0;
+    for (int32_t r = 0; r + 1 < p->P; ++r)
+      for (int32_t k = 0; k < p->Hl / hg; ++k, ++g, head += hg) {
+        h->h0[g] = head;
+        h->hg[g] = hg;
+      }
+    for (int32_t left = p->Hl; left > 0; ++g) {
+      const int32_t size = std::min(hg, left > 1 ? (left + 1) / 2 : 1);
+      h->h0[g] = head;
+      h->hg[g] = size;
+      head += size;
+      left -= size;
+    }
+  }
   ok = ok && cudaStreamCreateWithFlags(&h->h2d, cudaStreamNonBlocking) == cudaSuccess;
   ok = ok && cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking) == cudaSuccess;
   ok = ok && cudaEventCreateWithFlags(&h->start, cudaEventDisableTiming) == cudaSuccess;
@@ -702,25 +727,30 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
   std::lock_guard<std::mutex> lock(g_pipe_mutex);
   ulysses::HostPipe* h = plan_pipe(plan);
   if (!h) return ULYSSES_ERR_CUDA;
-  const int32_t hg = h->group_heads, groups = h->n;
-  const size_t width = static_cast<size_t>(hg) * plan->D * 2, pitch = static_cast<size_t>(plan->H) * plan->D * 2;
-  const int64_t t_bytes = static_cast<int64_t>(plan->C) * plan->Np * hg * plan->D * 2;   // one group's head slab
-  const int64_t o_bytes = plan->Np * static_cast<int64_t>(hg) * plan->D * 2;
+  const int32_t groups = h->n;
+  const size_t head_bytes = static_cast<size_t>(plan->D) * 2, pitch = static_cast<size_t>(plan->H) * plan->D * 2;
   // the copies start after everything already queued on the caller's stream
   if (cudaEventRecord(h->start, st) != cudaSuccess || cudaStreamWaitEvent(h->h2d, h->start, 0) != cudaSuccess)
     return status_of(cudaErrorUnknown);
   for (int32_t g = 0; g < groups; ++g) {
-    if (copy_heads_in(plan, g * hg, hg, hin, din, h->h2d) != cudaSuccess ||
+    if (copy_heads_in(plan, h->h0[g], h->hg[g], hin, din, h->h2d) != cudaSuccess ||
         cudaEventRecord(h->in[g], h->h2d) != cudaSuccess)
       return status_of(cudaErrorUnknown);
   }
+  // with fused = 0 the groups' head slabs and attention outputs sit one after
+  // another in the workspace (they add up to the whole T and O_T)
+  int64_t t_off = 0, o_off = 0;
   for (int32_t g = 0; g < groups; ++g) {
+    const int32_t h0 = h->h0[g], hg = h->hg[g];
+    const size_t off = h0 * head_bytes, width = hg * head_bytes;
     if (cudaStreamWaitEvent(st, h->in[g], 0) != cudaSuccess) return status_of(cudaErrorUnknown);
-    uint8_t* Tg = fused ? nullptr : T + g * t_bytes;
-    uint8_t* OTg = fused ? nullptr : OT + g * o_bytes;
-    if ((s = group_layer_impl(plan, g * hg, hg, din, dout, Tg, OTg, fused, scale, st)) != ULYSSES_OK) return s;
+    uint8_t* Tg = fused ? nullptr : T + t_off;
+    uint8_t* OTg = fused ? nullptr : OT + o_off;
+    t_off += static_cast<int64_t>(plan->C) * plan->Np * static_cast<int64_t>(width);
+    o_off += plan->Np * static_cast<int64_t>(width);
+    if ((s = group_layer_impl(plan, h0, hg, din, dout, Tg, OTg, fused, scale, st)) != ULYSSES_OK) return s;
     if (cudaEventRecord(h->out[g], st) != cudaSuccess || cudaStreamWaitEvent(h->d2h, h->out[g], 0) != cudaSuccess ||
-        cudaMemcpy2DAsync(hout + g * width, pitch, dout + g * width, pitch, width, static_cast<size_t>(plan->Np),
+        cudaMemcpy2DAsync(hout + off, pitch, dout + off, pitch, width, static_cast<size_t>(plan->Np),
                           cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess)
       return status_of(cudaErrorUnknown);
   }

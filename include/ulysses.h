@@ -303,7 +303,9 @@ int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out
  * group g's kernels on `stream`, which overlap the device->host copy of group
  * g-1's output columns.  A group is the smallest divisor of H/P heads whose
  * attention launch still fills every SM about three times over (at most one
- * rank).  With fused = 0 the workspace holds the groups' head slabs one after
+ * rank); the last rank's groups shrink (that size, then about half of what
+ * is left each time, down to one head), so that little work remains after
+ * the last input copy.  With fused = 0 the workspace holds the groups' head slabs one after
  * another (its size is ulysses_workspace_bytes() as for the device layer; its
  * layout is internal).  The copies run on two streams owned by the plan
  * (created with their events by the plan's first call of this function,

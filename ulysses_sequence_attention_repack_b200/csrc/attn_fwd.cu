@@ -225,9 +225,10 @@ __device__ __forceinline__ void exp_store_half(const float* s, int half, f2 scal
 // operands the tensor core needs half the cycles of bf16 and the MUFU unit
 // limits the loop, so with kEmu one group of four keys in kFp8EmuEvery is
 // exponentiated on the FMA pipe (exp2_poly2, relative error 7.5e-5, far below
-// E4M3's 2^-4): measured 3.7% faster at the Video-DiT size (1 in 2: slower,
-// 1 in 8: 2% faster).
-constexpr int kFp8EmuEvery = 4;
+// E4M3's 2^-4).  Measured against no emulation at the Video-DiT size
+// (19,394 tokens) and the 104k-token size: 1 in 8 is 7.3% and 3.6% faster,
+// 1 in 4 4.3% and 0%, 1 in 16 1.4% and 0%, 1 in 3 or 2 slower than 1 in 4.
+constexpr int kFp8EmuEvery = 8;
 template <bool kEmu>
 __device__ __forceinline__ void exp_store_half_fp8(const float* s, int half, f2 scale2, f2 negm2, f2 (&acc)[4],
                                                    uint32_t tS) {

@@ -77,12 +77,11 @@ def pct(xs, q):
 
 
 def tensor_peak(pk):
-    """Dense bf16 denominator for the attention kernel: the burst GEMM figure.
-    The SM clock sampled while the layer steps run stays near its 1965 MHz
-    maximum (the sustained GEMM figure was taken at ~1340 MHz, where a
-    tensor-saturating kernel settles under the power cap), so the kernel is
-    compared with the peak of the same clock regime; the fraction of the
-    sustained figure is reported beside it."""
+    """Dense bf16 denominator for the attention kernel: the burst GEMM figure,
+    the stricter of the two measured ones.  The power cap is flagged while
+    the layer steps run, but the sampled SM clock stays near its maximum, so
+    the sustained figure (taken where a tensor-saturating kernel settles
+    under the cap) is reported beside it rather than used."""
     return pk["bf16_tflops"], "bf16 burst"
 
 

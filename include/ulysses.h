@@ -75,6 +75,8 @@ enum {
  * segment), as in the causal flash wrapper of the prime-rl Ulysses context
  * parallelism pull request. */
 #define ULYSSES_PLAN_CAUSAL 1u
+/* Most ranks the multi-GPU push calls address (one NVLink domain). */
+#define ULYSSES_MAX_PUSH_RANKS 64
 
 typedef struct ulysses_plan_s ulysses_plan_t;
 
@@ -224,6 +226,55 @@ size_t ulysses_workspace_bytes_fp8(const ulysses_plan_t* plan);
  */
 int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
                           size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- multi-GPU push
+ * Steps 1 and 3 across P real GPUs, one process per GPU: rank q owns the
+ * sequence rows [q*Nl, (q+1)*Nl).  These are the all-to-all exchanges of
+ * "Ulysses performance on GB200" (fine-grained remote stores into each peer's
+ * window, one plane at a time, 1 GiB per rank), done as a push: each rank
+ * writes its data straight into the other ranks' buffers with plain 16-byte
+ * stores through peer pointers.  The pointers are device addresses valid on
+ * the calling rank's device -- CUDA IPC (or VMM) mappings of the peers'
+ * allocations over NVLink, or local buffers when the ranks are emulated on
+ * one GPU.  No TMA and no multicast reads or writes peer memory.
+ *
+ * Every rank creates the plan with the same global arguments (N, H, P,
+ * planes, cu_seqlens, flags); the shards use the default token-interleaved
+ * layout (token_stride = C*H*D, plane_stride = H*D), otherwise
+ * ULYSSES_ERR_UNSUPPORTED, as is P > ULYSSES_MAX_PUSH_RANKS.
+ *
+ *   shard       S_q : [Nl, C, H, D] on rank q; row i is sequence row q*Nl + i
+ *                     (rows at or past N are padding and must be zero)
+ *   head slab   T_r : [C, Np, Hl, D] on rank r (rank r's slab of T)
+ *   out shard   O_q : [Nl, planes, H, D] on rank q ([Nl, H, D] for the layer)
+ *
+ * Pointer tables are HOST arrays of P device pointers indexed by rank; each
+ * must be 16-byte aligned, non-null, and must not overlap the call's source.
+ * The calls only store: the caller orders the exchange, i.e. rank r reads T_r
+ * (or O_r) only after every rank's push into it has completed, with a
+ * stream-ordered barrier (an NCCL all-reduce of one word on the same stream,
+ * or a symmetric-memory barrier).  Errors: ARG (rank out of range, null or
+ * overlapping pointer), ALIGN, UNSUPPORTED, CUDA.
+ */
+
+/* Step 1 pushed by rank `rank`: dst_heads[r][c, rank*Nl + i, j, :] =
+ * src_shard[i, c, r*Hl + j, :] for every rank r, plane c and row i < Nl.  One
+ * launch per plane chunk (at most 1 GiB per rank, as ulysses_repack_fwd). */
+int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_shard,
+                            void* const* dst_heads, void* stream);
+
+/* Steps 2 and 3 in one kernel on rank `rank`: attention over the rank's head
+ * slab `heads` (T_r, all Np rows; segments, causal flag and pad rows as
+ * ulysses_attn_fwd), each output row n stored by the epilogue straight into
+ * its owning rank q = n / Nl:  dst_seq[q][n - q*Nl, rank*Hl + j, :] = O(n, j). */
+int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* heads, void* const* dst_seq,
+                          float softmax_scale, void* stream);
+
+/* Step 3 alone, pushed by rank `rank` from its head rows src_heads
+ * [planes, Np, Hl, D]: dst_seq[q][i, c, rank*Hl + j, :] =
+ * src_heads[c, q*Nl + i, j, :] into [Nl, planes, H, D] shards (1 <= planes <= C). */
+int ulysses_repack_bwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_heads,
+                            void* const* dst_seq, int32_t planes, void* stream);
 
 /* ---------------------------------------------------------------- training
  * The gradient of the layer.  The FastVideo transport carries gradients back

@@ -1,0 +1,170 @@
+"""The multi-GPU push calls with the P ranks emulated on one GPU, through the C ABI.
+
+Every rank's buffer is its own allocation and every pointer table holds those
+buffers, so the kernels address P separate destinations exactly as they would
+peer mappings; each rank's launch is independent (no launch waits for
+another), and the results are read after all of them.  The exchange computes
+the Ulysses map itself, so the pushed slabs must equal the oracle's mode 0 /
+mode 1 bit for bit, and the fused attention-push must equal the one-GPU layer
+bit for bit (same kernel, same tile order per work unit), which the parity
+suite holds to the fp64 oracle; one case is also checked against the oracle
+here.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import ulysses_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+# (P, N, H, C, cu_seqlens, causal, seed)
+CASES = [
+    pytest.param(2, 1024, 8, 3, None, False, 60, id="tiny-P2"),
+    pytest.param(4, 1001, 8, 3, None, False, 61, id="ragged-P4-N1001"),
+    pytest.param(4, 777, 8, 4, None, False, 62, id="qkvg-P4-N777"),
+    pytest.param(8, 2048, 16, 3, [0, 1024, 1536, 2048], False, 63, id="varlen-P8"),
+    pytest.param(2, 1000, 4, 3, [0, 300, 300, 777, 1000], True, 64, id="causal-varlen-P2"),
+    pytest.param(4, 5, 4, 3, None, False, 65, id="N5-P4"),
+    pytest.param(1, 300, 2, 3, None, False, 66, id="P1"),
+]
+
+
+def _bits(t):
+    from ulysses_sequence_attention_repack_b200 import inputs
+    return inputs.host_bits(t)
+
+
+def _setup(gpu, P, N, H, C, cu, causal, seed):
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu, causal=causal)
+    Np, Nl, Hl = plan.padded_tokens, plan.rows_per_rank, H // P
+    S = inputs.qkv_seq(N, H, P, C, seed, gpu)
+    shards = [S[q * Nl:(q + 1) * Nl].clone() for q in range(P)]
+    T = [torch.empty((C, Np, Hl, 128), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for t in T:
+        t.fill_(float("nan"))
+    return plan, S, shards, T
+
+
+@pytest.mark.parametrize("P,N,H,C,cu,causal,seed", CASES)
+def test_push_exchange_and_fused_attention(gpu, P, N, H, C, cu, causal, seed):
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    plan, S, shards, T = _setup(gpu, P, N, H, C, cu, causal, seed)
+    Np, Nl, Hl = plan.padded_tokens, plan.rows_per_rank, H // P
+    scale = 1.0 / math.sqrt(128)
+    # step 1: every rank pushes its shard into every rank's head slab
+    for q in range(P):
+        U.ulysses_repack_fwd_push(plan, q, shards[q], T)
+    # steps 2 + 3: each rank's attention stores its rows into the owners' shards
+    O = [torch.full((Nl, H, 128), float("nan"), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for r in range(P):
+        U.ulysses_attn_fwd_push(plan, r, T[r], O, scale)
+    # the one-GPU layer on the same input
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_layer_fwd(plan, S, OS, ws, fused=0)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    T_ref = orc.repack_fwd(_bits(S), P)
+    for r in range(P):
+        assert np.array_equal(_bits(T[r]), T_ref[r]), f"head slab of rank {r}"
+    got = np.concatenate([_bits(o) for o in O], axis=0)
+    assert np.array_equal(got, _bits(OS))
+
+
+@pytest.mark.parametrize("P,N,H,C,cu,causal,seed", CASES)
+def test_push_inverse_round_trip(gpu, P, N, H, C, cu, causal, seed):
+    """Mode 1 pushed by every rank: all C planes back restores the shards, and
+    the attention output plane gives the layer's output."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    plan, S, shards, T = _setup(gpu, P, N, H, C, cu, causal, seed)
+    Np, Nl, Hl = plan.padded_tokens, plan.rows_per_rank, H // P
+    for q in range(P):
+        U.ulysses_repack_fwd_push(plan, q, shards[q], T)
+    back = [torch.full((Nl, C, H, 128), float("nan"), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for r in range(P):
+        U.ulysses_repack_bwd_push(plan, r, T[r], back, C)
+    # one plane: the head-sharded attention output of the one-GPU path
+    Tg = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, Tg)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_attn_fwd(plan, Tg, OT, 1.0 / math.sqrt(128))
+    O1 = [torch.full((Nl, 1, H, 128), float("nan"), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for r in range(P):
+        U.ulysses_repack_bwd_push(plan, r, OT[r], O1, 1)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    for q in range(P):
+        assert np.array_equal(_bits(back[q]), _bits(shards[q])), f"shard of rank {q}"
+    got = np.concatenate([_bits(o)[:, 0] for o in O1], axis=0)
+    assert np.array_equal(got, orc.repack_bwd(_bits(OT)[:, None])[:, 0])
+
+
+def test_push_attention_against_oracle(gpu):
+    """The fused attention-push output against the fp64 oracle (the layer's
+    max-abs 2e-2 / mean-abs 2e-3), pad rows exactly zero."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    P, N, H, C = 4, 1001, 8, 3
+    plan, S, shards, T = _setup(gpu, P, N, H, C, None, False, 67)
+    Nl = plan.rows_per_rank
+    scale = 1.0 / math.sqrt(128)
+    for q in range(P):
+        U.ulysses_repack_fwd_push(plan, q, shards[q], T)
+    O = [torch.empty((Nl, H, 128), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for r in range(P):
+        U.ulysses_attn_fwd_push(plan, r, T[r], O, scale)
+    torch.cuda.synchronize()
+    got = torch.cat(O, 0).float().cpu().numpy().astype(np.float64)
+    ref = orc.layer_fwd(_bits(S), P, N, scale)
+    err = np.abs(got - ref)[:N]
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+    assert np.all(got[N:] == 0)
+
+
+_PEER_SCRIPT = r"""
+import math, os, sys
+import torch, torch.distributed as dist
+sys.path.insert(0, os.getcwd())
+import ulysses_sequence_attention_repack_b200 as U
+from ulysses_sequence_attention_repack_b200 import inputs, peer
+dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % int(sys.argv[1]), rank=0, world_size=1)
+dev = torch.device("cuda", 0)
+torch.cuda.set_device(dev)
+N, H, C = 1000, 4, 3
+plan = U.ulysses_plan(N, H, 128, 1, C)
+layer = peer.PeerLayer(plan)
+S = inputs.qkv_seq(N, H, 1, C, 68, dev)
+out = layer(S).clone()
+ref = torch.empty((plan.padded_tokens, H, 128), dtype=torch.bfloat16, device=dev)
+U.ulysses_layer_fwd(plan, S, ref, torch.empty(plan.workspace_bytes, dtype=torch.uint8, device=dev), fused=0)
+torch.cuda.synchronize()
+assert U.ulysses_last_device_error(plan) == 0
+assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), "peer layer differs from the one-GPU layer"
+del layer
+dist.destroy_process_group()
+print("peer-layer-ok")
+"""
+
+
+def test_peer_layer_one_rank_through_symmetric_memory(gpu):
+    """PeerLayer end to end on a one-rank group (the only multi-process shape a
+    one-GPU machine can run): symmetric-memory slabs, the push kernels and the
+    barriers, equal to the one-GPU layer bit for bit."""
+    import os
+    import socket
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    r = subprocess.run([sys.executable, "-c", _PEER_SCRIPT, str(port)], cwd=root, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0 and "peer-layer-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

@@ -60,3 +60,61 @@ def test_all_to_all_processes_match_oracle_repack(tmp_path, world, Nl, C, H):
         assert np.array_equal(np.load(tmp_path / f"heads{r}.npy"), T[r])
         Nl_ = S.shape[0] // world
         assert np.array_equal(np.load(tmp_path / f"back{r}.npy"), S[r * Nl_:(r + 1) * Nl_])
+
+
+def _agree_worker(rank, world, port, Ns, result_dir):
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import peer
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        plan = U.ulysses_plan(Ns[rank], 8, 128, world, 3)
+        try:
+            peer.agree_plan(plan)
+            verdict = "ok"
+        except ValueError as e:
+            verdict = "refused: " + str(e)
+        with open(os.path.join(result_dir, f"agree{rank}.txt"), "w") as f:
+            f.write(verdict)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("Ns,expect_ok", [((1024, 1024), True), ((1024, 1000), False)])
+def test_ranks_agree_on_the_plan(tmp_path, Ns, expect_ok):
+    """Every rank of the multi-GPU layer checks that all ranks hold the same
+    plan before any peer store; a mismatch is refused on every rank."""
+    world = len(Ns)
+    mp.start_processes(_agree_worker, args=(world, _free_port(), Ns, str(tmp_path)), nprocs=world,
+                       start_method="spawn")
+    verdicts = [(tmp_path / f"agree{r}.txt").read_text() for r in range(world)]
+    if expect_ok:
+        assert verdicts == ["ok"] * world
+    else:
+        assert all(v.startswith("refused: plans differ across ranks: ranks [1]") for v in verdicts), verdicts
+
+
+def _world_mismatch_worker(rank, world, port, result_dir):
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import peer
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        plan = U.ulysses_plan(1024, 8, 128, 4, 3)   # four ranks planned, two present
+        try:
+            peer.agree_plan(plan)
+            verdict = "ok"
+        except ValueError as e:
+            verdict = "refused: " + str(e)
+        with open(os.path.join(result_dir, f"world{rank}.txt"), "w") as f:
+            f.write(verdict)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_group_size_must_match_the_plan(tmp_path):
+    mp.start_processes(_world_mismatch_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2, start_method="spawn")
+    for r in range(2):
+        assert (tmp_path / f"world{r}.txt").read_text() == "refused: the plan has P=4 ranks but the group has 2"

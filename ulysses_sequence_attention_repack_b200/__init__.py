@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     ulysses_attn_fwd,
     ulysses_attn_fwd_fp8,
     ulysses_attn_fwd_lse,
+    ulysses_attn_fwd_push,
     ulysses_last_device_error,
     ulysses_layer_bwd,
     ulysses_layer_fwd,
@@ -26,7 +27,9 @@ from ._lib import (  # noqa: F401
     ulysses_plan,
     ulysses_prologue_repack_fwd,
     ulysses_repack_bwd,
+    ulysses_repack_bwd_push,
     ulysses_repack_fwd,
     ulysses_repack_fwd_fp8,
+    ulysses_repack_fwd_push,
     ulysses_selftest_exp2_poly,
 )

@@ -36,7 +36,8 @@ EXPORTS = (
     "ulysses_layer_fwd_fused_noalloc", "ulysses_selftest_wait_timeout", "ulysses_prologue_repack_fwd",
     "ulysses_lse_bytes", "ulysses_attn_fwd_lse", "ulysses_attn_bwd_workspace_bytes", "ulysses_attn_bwd",
     "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd", "ulysses_repack_fwd_fp8", "ulysses_attn_fwd_fp8",
-    "ulysses_workspace_bytes_fp8", "ulysses_layer_fwd_fp8",
+    "ulysses_workspace_bytes_fp8", "ulysses_layer_fwd_fp8", "ulysses_repack_fwd_push", "ulysses_attn_fwd_push",
+    "ulysses_repack_bwd_push",
 )
 
 
@@ -123,6 +124,12 @@ def load() -> ctypes.CDLL:
         lib.ulysses_workspace_bytes_fp8.restype = sz
         lib.ulysses_layer_fwd_fp8.argtypes = [vp, vp, vp, vp, sz, vp]
         lib.ulysses_layer_fwd_fp8.restype = ctypes.c_int
+        lib.ulysses_repack_fwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), vp]
+        lib.ulysses_repack_fwd_push.restype = ctypes.c_int
+        lib.ulysses_attn_fwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), ctypes.c_float, vp]
+        lib.ulysses_attn_fwd_push.restype = ctypes.c_int
+        lib.ulysses_repack_bwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), i32, vp]
+        lib.ulysses_repack_bwd_push.restype = ctypes.c_int
         lib.ulysses_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
         lib.ulysses_selftest_exp2_poly.restype = ctypes.c_int
         _handle = lib
@@ -174,6 +181,11 @@ class Plan:
     @property
     def padded_tokens(self) -> int:
         return load().ulysses_plan_padded_tokens(self.handle)
+
+    @property
+    def rows_per_rank(self) -> int:
+        """Nl = Np / P: the sequence rows each rank owns."""
+        return self.padded_tokens // self.P
 
     @property
     def plane_chunk(self) -> int:
@@ -284,6 +296,41 @@ def ulysses_repack_bwd(plan: Plan, src_heads, dst_seq, planes: int, stream=None)
 def ulysses_attn_fwd(plan: Plan, qkv_heads, out_heads, softmax_scale: float, stream=None) -> None:
     _check(load().ulysses_attn_fwd(plan.handle, _ptr(qkv_heads), _ptr(out_heads), float(softmax_scale),
                                    _stream(stream)), "ulysses_attn_fwd")
+
+
+def _ptr_table(ptrs):
+    """Host array of device pointers (tensors or int addresses), indexed by rank."""
+    if ptrs is None:
+        return None
+    vals = [_ptr(t) for t in ptrs]
+    return (ctypes.c_void_p * max(1, len(vals)))(*vals)
+
+
+def ulysses_repack_fwd_push(plan: Plan, rank: int, src_shard, dst_heads, stream=None) -> None:
+    """Rank `rank` pushes its shard [Nl, C, H, D] into every rank's head slab
+    dst_heads[r] = T_r [C, Np, Hl, D] (device pointers, one per rank)."""
+    if dst_heads is not None and len(dst_heads) != plan.P:
+        raise UlyssesError(ULYSSES_ERR_ARG, "ulysses_repack_fwd_push: one destination per rank")
+    _check(load().ulysses_repack_fwd_push(plan.handle, int(rank), _ptr(src_shard), _ptr_table(dst_heads),
+                                          _stream(stream)), "ulysses_repack_fwd_push")
+
+
+def ulysses_attn_fwd_push(plan: Plan, rank: int, heads, dst_seq, softmax_scale: float, stream=None) -> None:
+    """Attention over rank `rank`'s head slab T_r with each output row stored
+    into its owning rank's shard dst_seq[q] = O_q [Nl, H, D]."""
+    if dst_seq is not None and len(dst_seq) != plan.P:
+        raise UlyssesError(ULYSSES_ERR_ARG, "ulysses_attn_fwd_push: one destination per rank")
+    _check(load().ulysses_attn_fwd_push(plan.handle, int(rank), _ptr(heads), _ptr_table(dst_seq),
+                                        float(softmax_scale), _stream(stream)), "ulysses_attn_fwd_push")
+
+
+def ulysses_repack_bwd_push(plan: Plan, rank: int, src_heads, dst_seq, planes: int, stream=None) -> None:
+    """Rank `rank` pushes its head rows [planes, Np, Hl, D] into every rank's
+    shard dst_seq[q] = [Nl, planes, H, D]."""
+    if dst_seq is not None and len(dst_seq) != plan.P:
+        raise UlyssesError(ULYSSES_ERR_ARG, "ulysses_repack_bwd_push: one destination per rank")
+    _check(load().ulysses_repack_bwd_push(plan.handle, int(rank), _ptr(src_heads), _ptr_table(dst_seq), int(planes),
+                                          _stream(stream)), "ulysses_repack_bwd_push")
 
 
 def ulysses_repack_fwd_fp8(plan: Plan, src_seq, dst_heads_fp8, stream=None) -> None:

@@ -13,7 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libulysses.so")
-SOURCES = ["api.cpp", "repack.cu", "prologue.cu", "attn_fwd.cu", "attn_bwd.cu", "selftest.cu", "noalloc.cu"]
+SOURCES = ["api.cpp", "repack.cu", "prologue.cu", "attn_fwd.cu", "attn_bwd.cu", "selftest.cu", "noalloc.cu",
+           "transport.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -318,6 +318,28 @@ int group_layer_impl(const ulysses_plan_t* p, int32_t h0, int32_t hg, const uint
   return status_of(ulysses::launch_repack(1, OTg, OSg, p->Np, hg, 1, 1, 0, 1, row, row, st));
 }
 
+// Multi-GPU push: the plan must describe the default token-interleaved
+// layout, which is also the layout of every rank's shard.
+bool push_layout_ok(const ulysses_plan_t* p) {
+  return p->P <= ULYSSES_MAX_PUSH_RANKS && p->token_stride == static_cast<int64_t>(p->C) * p->H * p->D &&
+         p->plane_stride == static_cast<int64_t>(p->H) * p->D;
+}
+
+// Copies the caller's P destination pointers into a kernel table.  Each must
+// be non-null and 16-byte aligned, and none may overlap the source range.
+int push_table(const ulysses_plan_t* p, void* const* ptrs, int64_t dst_bytes, const void* src, int64_t src_bytes,
+               ulysses::PushTable* t) {
+  if (!ptrs) return ULYSSES_ERR_ARG;
+  std::memset(t, 0, sizeof(*t));
+  for (int32_t r = 0; r < p->P; ++r) {
+    if (!ptrs[r]) return ULYSSES_ERR_ARG;
+    if (!aligned16(ptrs[r])) return ULYSSES_ERR_ALIGN;
+    if (overlap(src, src_bytes, ptrs[r], dst_bytes)) return ULYSSES_ERR_ARG;
+    t->p[r] = ptrs[r];
+  }
+  return ULYSSES_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -758,6 +780,87 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
   if (cudaEventRecord(h->done, h->d2h) != cudaSuccess || cudaStreamWaitEvent(st, h->done, 0) != cudaSuccess)
     return status_of(cudaErrorUnknown);
   return ULYSSES_OK;
+}
+
+int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_shard,
+                            void* const* dst_heads, void* stream) {
+  if (!plan || !src_shard || !dst_heads || rank < 0 || rank >= plan->P) return ULYSSES_ERR_ARG;
+  if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
+  if (!aligned16(src_shard)) return ULYSSES_ERR_ALIGN;
+  const int64_t shard_bytes = plan->Nl * plan->C * plan->H * plan->D * 2;
+  const int64_t slab_bytes = static_cast<int64_t>(plan->C) * plan->Np * plan->Hl * plan->D * 2;
+  ulysses::PushTable t;
+  int s = push_table(plan, dst_heads, slab_bytes, src_shard, shard_bytes, &t);
+  if (s != ULYSSES_OK) return s;
+  if ((s = device_ready(plan)) != ULYSSES_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int32_t c0 = 0; c0 < plan->C; c0 += plan->plane_chunk) {
+    const int32_t cc = std::min(plan->plane_chunk, plan->C - c0);
+    s = status_of(ulysses::launch_push(0, src_shard, t, plan->Nl, plan->Np, plan->H, plan->P, plan->C, c0, cc, rank,
+                                       st));
+    if (s != ULYSSES_OK) return s;
+  }
+  return ULYSSES_OK;
+}
+
+int ulysses_repack_bwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_heads, void* const* dst_seq,
+                            int32_t planes, void* stream) {
+  if (!plan || !src_heads || !dst_seq || rank < 0 || rank >= plan->P || planes < 1 || planes > plan->C)
+    return ULYSSES_ERR_ARG;
+  if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
+  if (!aligned16(src_heads)) return ULYSSES_ERR_ALIGN;
+  const int64_t slab_bytes = static_cast<int64_t>(planes) * plan->Np * plan->Hl * plan->D * 2;
+  const int64_t shard_bytes = plan->Nl * planes * plan->H * plan->D * 2;
+  ulysses::PushTable t;
+  int s = push_table(plan, dst_seq, shard_bytes, src_heads, slab_bytes, &t);
+  if (s != ULYSSES_OK) return s;
+  if ((s = device_ready(plan)) != ULYSSES_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int32_t c0 = 0; c0 < planes; c0 += plan->plane_chunk) {
+    const int32_t cc = std::min(plan->plane_chunk, planes - c0);
+    s = status_of(ulysses::launch_push(1, src_heads, t, plan->Nl, plan->Np, plan->H, plan->P, planes, c0, cc, rank,
+                                       st));
+    if (s != ULYSSES_OK) return s;
+  }
+  return ULYSSES_OK;
+}
+
+int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* heads, void* const* dst_seq,
+                          float softmax_scale, void* stream) {
+  if (!plan || !heads || !dst_seq || rank < 0 || rank >= plan->P) return ULYSSES_ERR_ARG;
+  if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
+  if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
+  if (!aligned16(heads)) return ULYSSES_ERR_ALIGN;
+  const int64_t slab_bytes = static_cast<int64_t>(plan->C) * plan->Np * plan->Hl * plan->D * 2;
+  const int64_t shard_bytes = plan->Nl * plan->H * plan->D * 2;
+  ulysses::PushTable t;
+  int s = push_table(plan, dst_seq, shard_bytes, heads, slab_bytes, &t);
+  if (s != ULYSSES_OK) return s;
+  if ((s = device_ready(plan)) != ULYSSES_OK) return s;
+  // this rank's heads start at column rank*Hl of every destination row
+  for (int32_t q = 0; q < plan->P; ++q)
+    t.p[q] = static_cast<uint8_t*>(t.p[q]) + static_cast<int64_t>(rank) * plan->Hl * plan->D * 2;
+  ulysses::AttnLaunch a;
+  a.base = heads;
+  a.fused = 0;
+  a.Np = plan->Np;
+  a.N = plan->N;
+  a.H = plan->Hl;   // one rank's slab: a one-rank problem of Hl heads
+  a.P = 1;
+  a.Hl = plan->Hl;
+  a.C = plan->C;
+  a.tok_stride = plan->token_stride;
+  a.plane_stride = plan->plane_stride;
+  a.out = t.p[0];
+  a.o_stride_r = 0;
+  a.o_stride_n = static_cast<int64_t>(plan->H) * plan->D;
+  a.o_stride_j = plan->D;
+  a.scale = softmax_scale;
+  a.plan = plan;
+  a.push = &t;
+  a.push_rows = plan->Nl;
+  a.push_ranks = plan->P;
+  return status_of(ulysses::launch_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
 int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream) {

@@ -141,7 +141,9 @@ struct AttnParams {
   int32_t num_pairs;               // causal schedule: pairs of query blocks over all segments and heads
   int32_t paired;                  // 1: the causal pair schedule (enough units for two per CTA)
   float scale_log2;
+  int64_t push_rows;               // > 0: row n is stored to push.p[n / push_rows] (multi-GPU push)
   SegDesc seg[ULYSSES_MAX_SEQS];   // longest first
+  PushTable push;
 };
 
 struct Unit {
@@ -607,8 +609,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.lse && n < sd.q_end && n < p.Np)
         p.lse[(static_cast<int64_t>(w.r) * p.Hl + w.j) * p.lse_stride + n] = m_used + log2f(l);
       if (n < sd.q_end && n < p.Np) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + w.r * p.o_stride_r + static_cast<int64_t>(n) * p.o_stride_n +
-                                              w.j * p.o_stride_j);
+        __nv_bfloat16* obase = p.out + w.r * p.o_stride_r;
+        int64_t orow = n;
+        if (p.push_rows > 0) {   // the owning rank's shard, through its peer pointer
+          const int64_t q = n / p.push_rows;
+          obase = static_cast<__nv_bfloat16*>(p.push.p[q]);
+          orow = n - q * p.push_rows;
+        }
+        uint4* dst = reinterpret_cast<uint4*>(obase + orow * p.o_stride_n + w.j * p.o_stride_j);
         const bool pad = n >= p.N;   // pad rows are written as zeros
         const float inv = 1.0f / l;
         const float* o = reinterpret_cast<const float*>(&oraw[0][0]);
@@ -725,6 +733,15 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   p.fused = a.fused;
   p.causal = pl->causal;
   p.scale_log2 = a.scale * 1.4426950408889634f;
+  if (a.push_rows > 0) {
+    // every output row n < Np must map to a table entry n / push_rows
+    if (!a.push || a.push_ranks < 1 || a.push_ranks > ULYSSES_MAX_PUSH_RANKS || a.push_rows * a.push_ranks < a.Np)
+      return cudaErrorInvalidValue;
+    for (int q = 0; q < a.push_ranks; ++q)
+      if (!a.push->p[q]) return cudaErrorInvalidValue;
+    p.push_rows = a.push_rows;
+    p.push = *a.push;
+  }
 
   // Non-empty segments, longest first.  The segment that ends at N also
   // covers the pad query rows [N, Np), which are written as zeros.

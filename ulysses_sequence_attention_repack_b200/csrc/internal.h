@@ -52,6 +52,18 @@ cudaError_t launch_prologue_repack(const void* src, void* dst, const void* wq, c
                                    int32_t Ctot, int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
                                    cudaStream_t stream);
 
+// Destination table of the multi-GPU push (a kernel parameter): entry r is
+// rank r's buffer (a peer mapping, or a local buffer when ranks are emulated).
+struct PushTable {
+  void* p[ULYSSES_MAX_PUSH_RANKS];
+};
+
+// One push launch over planes [c0, c0 + cc) by rank `rank` (transport.cu).
+//   dir = 0: shard [Nl, C, H, D] -> dst.p[r] = T_r [C, Np, Hl, D], rows rank*Nl + i
+//   dir = 1: head rows [C, Np, Hl, D] -> dst.p[q] = [Nl, C, H, D], heads rank*Hl + j
+cudaError_t launch_push(int dir, const void* src, const PushTable& dst, int64_t Nl, int64_t Np, int32_t H,
+                        int32_t P, int32_t C, int32_t c0, int32_t cc, int32_t rank, cudaStream_t stream);
+
 // Attention launch description (filled by api.cpp).
 struct AttnLaunch {
   const void* base;        // Q/K/V source buffer
@@ -66,6 +78,11 @@ struct AttnLaunch {
   float* lse = nullptr;          // optional log2-domain LSE output [P*Hl][lse_stride]
   int64_t lse_stride = 0;
   int fp8 = 0;                   // 1: base holds E4M3 codes [P, C, Np, Hl, D] (fused must be 0)
+  // multi-GPU push epilogue: when push_rows > 0, output row n goes to
+  // push->p[n / push_rows] + (n % push_rows) * o_stride_n + j * o_stride_j
+  const PushTable* push = nullptr;
+  int64_t push_rows = 0;
+  int32_t push_ranks = 0;        // entries of push in use (push_rows * push_ranks >= Np)
 };
 
 cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream);

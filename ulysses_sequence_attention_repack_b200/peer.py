@@ -1,0 +1,92 @@
+"""The Ulysses layer across P GPUs, one process per GPU, over peer memory.
+
+Rank q holds the sequence rows [q*Nl, (q+1)*Nl) of the input as a shard
+[Nl, C, H, D] (token-interleaved).  One forward is
+
+  1. ``ulysses_repack_fwd_push``: rank q stores, for every rank r, its rows of
+     r's heads into r's head slab T_r [C, Np, Hl, D] through a peer pointer
+     (step 1, the all-to-all of the transport page, as a push);
+  2. a stream-ordered barrier: every rank's stores into T_r have completed;
+  3. ``ulysses_attn_fwd_push``: attention over T_r, whose epilogue stores each
+     output row into its owning rank's output shard [Nl, H, D] (steps 2 and 3
+     in one kernel);
+  4. a barrier: every output shard is complete.
+
+The slabs and shards are allocated in PyTorch's symmetric memory, which maps
+every rank's allocation into every peer (NVLink over NVSwitch) and provides
+the barrier; every byte of the layer is moved and computed by this library's
+kernels.  All ranks must build the plan with the same arguments; the
+constructor checks that (``agree_plan``).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+from ._lib import Plan, ulysses_attn_fwd_push, ulysses_repack_fwd_push
+
+
+def plan_signature(plan: Plan) -> tuple:
+    """What every rank's plan must agree on."""
+    return (plan.N, plan.H, plan.D, plan.P, plan.planes,
+            None if plan.cu_seqlens is None else tuple(plan.cu_seqlens), plan.causal)
+
+
+def agree_plan(plan: Plan, group=None) -> None:
+    """Raise ValueError on every rank unless the group has P ranks that all
+    hold the same plan (a collective: every rank of the group must call it)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    sigs = [None] * world
+    dist.all_gather_object(sigs, plan_signature(plan), group=group)
+    if world != plan.P:
+        raise ValueError(f"the plan has P={plan.P} ranks but the group has {world}")
+    bad = [r for r, s in enumerate(sigs) if s != sigs[0]]
+    if bad:
+        raise ValueError(f"plans differ across ranks: ranks {bad} disagree with rank 0 ({sigs[0]} vs {sigs[bad[0]]})")
+
+
+class PeerLayer:
+    """One rank of the layer over P GPUs (softmax scale 1/sqrt(D) by default).
+
+    ``forward(shard)`` returns this rank's output shard [Nl, H, D]; the tensor
+    is reused by the next forward, so copy it to keep it.  Everything runs on
+    the current CUDA stream.
+    """
+
+    def __init__(self, plan: Plan, group=None, device=None, softmax_scale: float | None = None):
+        import torch
+        import torch.distributed as dist
+        from torch.distributed import _symmetric_memory as symm
+        # no NVLink multicast object is needed: the kernels use plain peer stores
+        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
+        agree_plan(plan, group)
+        self.plan = plan
+        self.group = group if group is not None else dist.group.WORLD
+        self.rank = dist.get_rank(self.group)
+        self.device = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(plan.D)
+        C, Np, Nl, H = plan.planes, plan.padded_tokens, plan.rows_per_rank, plan.H
+        Hl = H // plan.P
+        self.heads = symm.empty(C, Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
+        self.out = symm.empty(Nl, H, plan.D, dtype=torch.bfloat16, device=self.device)
+        self._heads_h = symm.rendezvous(self.heads, self.group)
+        self._out_h = symm.rendezvous(self.out, self.group)
+        self.heads_ptrs = self._peer_ptrs(self._heads_h, self.heads)
+        self.out_ptrs = self._peer_ptrs(self._out_h, self.out)
+
+    def _peer_ptrs(self, handle, local) -> list[int]:
+        """Every rank's address of the same tensor, as mapped on this device."""
+        ptrs = [int(p) for p in handle.buffer_ptrs]
+        off = local.data_ptr() - ptrs[self.rank]
+        return [p + off for p in ptrs]
+
+    def forward(self, shard):
+        """shard: this rank's rows [Nl, C, H, D] (bf16, on this rank's device)."""
+        ulysses_repack_fwd_push(self.plan, self.rank, shard, self.heads_ptrs)
+        self._heads_h.barrier(channel=0)
+        ulysses_attn_fwd_push(self.plan, self.rank, self.heads, self.out_ptrs, self.scale)
+        self._out_h.barrier(channel=1)
+        return self.out
+
+    __call__ = forward

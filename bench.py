@@ -262,6 +262,37 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     fused_ms = f0.elapsed_time(f1) / nf
 
+    # the multi-GPU push path with its P ranks emulated on this GPU: each rank
+    # pushes its shard (rows of S) into every head slab (slabs of T), then each
+    # rank's attention stores its rows into the owners' output shards (rows of OS)
+    Nl = plan.rows_per_rank
+    shards = [S[q * Nl:(q + 1) * Nl] for q in range(P)]
+    slabs = [T[r] for r in range(P)]
+    outs = [OS[q * Nl:(q + 1) * Nl] for q in range(P)]
+
+    def push_layer(evs=None):
+        if evs:
+            evs[0].record(stream)
+        for q in range(P):
+            U.ulysses_repack_fwd_push(plan, q, shards[q], slabs, stream)
+        if evs:
+            evs[1].record(stream)
+        for r in range(P):
+            U.ulysses_attn_fwd_push(plan, r, slabs[r], outs, scale, stream)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(3):
+        push_layer()
+    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        push_layer(pevs[k])
+    torch.cuda.synchronize()
+    push_ms = statistics.mean(e[0].elapsed_time(e[2]) for e in pevs)
+    push_rf_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in pevs)
+    if U.ulysses_last_device_error(plan) != 0:
+        raise RuntimeError("a kernel reported a device error in the push path")
+
     # step 1 with the QKV prologue fused in (RMSNorm + partial RoPE on Q and K,
     # rotary_dim 96 as in the pages), timed on the same input
     g = torch.Generator(device=dev)
@@ -374,6 +405,8 @@ def run_ours(args, rank, world, local_rank):
                                                                        pk["bf16_tflops"]), 3),
                       "spec_2250": round(attn_tflops / SPEC_PEAKS["bf16_tflops"], 3)},
         "fused_layer_us": round(fused_ms * 1000, 2),
+        "push_layer_us": round(push_ms * 1000, 2),
+        "push_repack_fwd_gbs": round(rf_bytes / (push_rf_ms * 1e-3) / 1e9, 1),
         "attn_bwd_us": round(bwd_ms * 1000, 2),
         "attn_bwd_tflops": round(2.5 * flops / (bwd_ms * 1e-3) / 1e12, 1),
         "prologue_repack_fwd_us": round(prologue_ms * 1000, 2),

@@ -4,7 +4,8 @@ Repack: bit-exact against the oracle's index map (at 250k tokens one plane of
 896,000,000 bytes per rank at a time).  Attention: a seeded subset of 4096
 query rows per head against the fp64 oracle (rows 0, N-1 and every segment
 boundary always included), max-abs <= 2e-2 and mean-abs <= 2e-3; the fused
-layer equals the unfused layer bit for bit everywhere.
+layer and the emulated multi-GPU push path equal the unfused layer bit for bit
+everywhere.
 """
 import math
 import os
@@ -65,6 +66,21 @@ def test_full_layer(gpu, name):
         del s_c
     # the fused layer never materialises T: it must still equal the unfused one
     assert torch.equal(OS, OSf)
+    # the multi-GPU push path with the ranks emulated, as the benchmark times
+    # it: the pushed slabs and the attention-push shards equal the one-GPU ones
+    Nl = plan.rows_per_rank
+    T2 = torch.empty_like(T)
+    slabs = [T2[r] for r in range(P)]
+    for q in range(P):
+        U.ulysses_repack_fwd_push(plan, q, S[q * Nl:(q + 1) * Nl], slabs)
+    OSp = torch.empty_like(OS)
+    outs = [OSp[q * Nl:(q + 1) * Nl] for q in range(P)]
+    for r in range(P):
+        U.ulysses_attn_fwd_push(plan, r, slabs[r], outs, scale)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    assert torch.equal(T2, T) and torch.equal(OSp, OS)
+    del T2, OSp
 
     # step 2 on sampled rows (T is now known to equal the oracle's repack)
     rows = orc.sample_rows(N, ROWS_PER_HEAD, seed, cu)

@@ -274,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
         if evs:
             evs[0].record(stream)
         for q in range(P):
-            U.ulysses_repack_fwd_push(plan, q, shards[q], slabs, stream)
+            U.ulysses_repack_fwd_push(plan, q, shards[q], slabs, stream=stream)
         if evs:
             evs[1].record(stream)
         for r in range(P):

@@ -243,10 +243,17 @@ int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void*
  * layout (token_stride = C*H*D, plane_stride = H*D), otherwise
  * ULYSSES_ERR_UNSUPPORTED, as is P > ULYSSES_MAX_PUSH_RANKS.
  *
- *   shard       S_q : [Nl, C, H, D] on rank q; row i is sequence row q*Nl + i
- *                     (rows at or past N are padding and must be zero)
- *   head slab   T_r : [C, Np, Hl, D] on rank r (rank r's slab of T)
+ *   shard       S_q : [Nl, planes, H, D] on rank q; row i is sequence row
+ *                     q*Nl + i (rows at or past N are padding and must be zero)
+ *   head slab   T_r : [planes, Np, Hl, D] on rank r (rank r's slab of T)
  *   out shard   O_q : [Nl, planes, H, D] on rank q ([Nl, H, D] for the layer)
+ * (planes = C for the layer's input, 1 for its output, 3 for Q/K/V gradients).
+ *
+ * For training, a rank keeps its head-sharded output and log-sum-exp
+ * (ulysses_attn_fwd_lse_slab, then ulysses_repack_bwd_push of the output),
+ * pushes the output gradient into the dO slabs (ulysses_repack_fwd_push with
+ * planes = 1), runs ulysses_attn_bwd_slab and pushes dQ, dK, dV back
+ * (ulysses_repack_bwd_push with planes = 3).
  *
  * Pointer tables are HOST arrays of P device pointers indexed by rank; each
  * must be 16-byte aligned, non-null, and must not overlap the call's source.
@@ -257,11 +264,14 @@ int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void*
  * overlapping pointer), ALIGN, UNSUPPORTED, CUDA.
  */
 
-/* Step 1 pushed by rank `rank`: dst_heads[r][c, rank*Nl + i, j, :] =
- * src_shard[i, c, r*Hl + j, :] for every rank r, plane c and row i < Nl.  One
- * launch per plane chunk (at most 1 GiB per rank, as ulysses_repack_fwd). */
+/* Step 1 pushed by rank `rank`, on the first `planes` planes (1..C; C for
+ * the layer's Q, K, V, 1 for an output gradient): src_shard [Nl, planes, H, D]
+ * into head slabs [planes, Np, Hl, D],
+ *   dst_heads[r][c, rank*Nl + i, j, :] = src_shard[i, c, r*Hl + j, :]
+ * for every rank r, plane c and row i < Nl.  One launch per plane chunk (at
+ * most 1 GiB per rank, as ulysses_repack_fwd). */
 int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_shard,
-                            void* const* dst_heads, void* stream);
+                            void* const* dst_heads, int32_t planes, void* stream);
 
 /* Steps 2 and 3 in one kernel on rank `rank`: attention over the rank's head
  * slab `heads` (T_r, all Np rows; segments, causal flag and pad rows as
@@ -275,6 +285,23 @@ int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* 
  * src_heads[c, q*Nl + i, j, :] into [Nl, planes, H, D] shards (1 <= planes <= C). */
 int ulysses_repack_bwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_heads,
                             void* const* dst_seq, int32_t planes, void* stream);
+
+/* Attention over ONE rank's head slab of the plan (steps 2 of the multi-GPU
+ * layer for training): heads T_r [C, Np, Hl, D] -> out_heads [Np, Hl, D] and
+ * lse [Hl][stride] (ulysses_lse_bytes(plan) / P bytes; the stride as
+ * ulysses_attn_fwd_lse).  Segments, causal flag and pad rows as
+ * ulysses_attn_fwd.  Errors: as ulysses_attn_fwd_lse. */
+int ulysses_attn_fwd_lse_slab(const ulysses_plan_t* plan, const void* heads, void* out_heads, void* lse,
+                              float softmax_scale, void* stream);
+
+/* The attention backward of one rank's slab: (dQ, dK, dV) [3, Np, Hl, D] from
+ * heads T_r, its out_heads and lse (ulysses_attn_fwd_lse_slab) and the output
+ * gradient dout_heads [Np, Hl, D]; the workspace is
+ * ulysses_attn_bwd_workspace_bytes(plan) / P bytes.  Errors: as
+ * ulysses_attn_bwd. */
+int ulysses_attn_bwd_slab(const ulysses_plan_t* plan, const void* heads, const void* out_heads,
+                          const void* dout_heads, const void* lse, void* dqkv_heads, void* workspace,
+                          size_t workspace_bytes, float softmax_scale, void* stream);
 
 /* ---------------------------------------------------------------- training
  * The gradient of the layer.  The FastVideo transport carries gradients back

@@ -146,16 +146,19 @@ def test_push_argument_checks_before_any_device_work():
 
     good = table(0x40000000, 0x50000000)
     ok_codes = (_lib.ULYSSES_ERR_CUDA,)
-    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, good, None) in ok_codes
-    assert lib.ulysses_repack_fwd_push(h, 2, 0x10000, good, None) == _lib.ULYSSES_ERR_ARG       # rank >= P
-    assert lib.ulysses_repack_fwd_push(h, -1, 0x10000, good, None) == _lib.ULYSSES_ERR_ARG
-    assert lib.ulysses_repack_fwd_push(h, 0, None, good, None) == _lib.ULYSSES_ERR_ARG
-    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, None, None) == _lib.ULYSSES_ERR_ARG
-    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, table(0x40000000, 0), None) == _lib.ULYSSES_ERR_ARG
-    assert lib.ulysses_repack_fwd_push(h, 0, 0x10008, good, None) == _lib.ULYSSES_ERR_ALIGN
-    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, table(0x40000000, 0x50000004), None) == _lib.ULYSSES_ERR_ALIGN
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, good, 3, None) in ok_codes
+    assert lib.ulysses_repack_fwd_push(h, 2, 0x10000, good, 3, None) == _lib.ULYSSES_ERR_ARG       # rank >= P
+    assert lib.ulysses_repack_fwd_push(h, -1, 0x10000, good, 3, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_repack_fwd_push(h, 0, None, good, 3, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, None, 3, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, good, 0, None) == _lib.ULYSSES_ERR_ARG       # planes < 1
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, good, 4, None) == _lib.ULYSSES_ERR_ARG       # planes > C
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, good, 1, None) in ok_codes
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, table(0x40000000, 0), 3, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10008, good, 3, None) == _lib.ULYSSES_ERR_ALIGN
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, table(0x40000000, 0x50000004), 3, None) == _lib.ULYSSES_ERR_ALIGN
     # a destination slab overlapping the source shard
-    assert lib.ulysses_repack_fwd_push(h, 1, 0x10000, table(0x40000000, 0x10000 + 4096), None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_repack_fwd_push(h, 1, 0x10000, table(0x40000000, 0x10000 + 4096), 3, None) == _lib.ULYSSES_ERR_ARG
     assert lib.ulysses_attn_fwd_push(h, 1, 0x10000, good, 0.1, None) in ok_codes
     assert lib.ulysses_attn_fwd_push(h, 1, 0x10000, good, 0.0, None) == _lib.ULYSSES_ERR_ARG
     assert lib.ulysses_attn_fwd_push(h, 3, 0x10000, good, 0.1, None) == _lib.ULYSSES_ERR_ARG
@@ -165,7 +168,7 @@ def test_push_argument_checks_before_any_device_work():
     assert lib.ulysses_repack_bwd_push(h, 0, 0x10000, good, 4, None) == _lib.ULYSSES_ERR_ARG
     # shards use the token-interleaved layout only
     pm = U.ulysses_plan(1024, 8, 128, 2, 3, 8 * 128, 1024 * 8 * 128)
-    assert lib.ulysses_repack_fwd_push(pm.handle, 0, 0x10000, good, None) == _lib.ULYSSES_ERR_UNSUPPORTED
+    assert lib.ulysses_repack_fwd_push(pm.handle, 0, 0x10000, good, 3, None) == _lib.ULYSSES_ERR_UNSUPPORTED
     assert lib.ulysses_attn_fwd_push(pm.handle, 0, 0x10000, good, 0.1, None) == _lib.ULYSSES_ERR_UNSUPPORTED
     # the binding wants one destination per rank
     with pytest.raises(U.UlyssesError):

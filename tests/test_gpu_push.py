@@ -148,6 +148,23 @@ torch.cuda.synchronize()
 assert U.ulysses_last_device_error(plan) == 0
 assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), "peer layer differs from the one-GPU layer"
 del layer
+# training through autograd, against the one-GPU autograd layer
+from ulysses_sequence_attention_repack_b200 import autograd as A
+tl = peer.PeerLayer(plan, training=True)
+g = torch.Generator(device=dev)
+g.manual_seed(69)
+dOut = torch.randn((plan.padded_tokens, H, 128), generator=g, device=dev).to(torch.bfloat16)
+x = S.clone().requires_grad_(True)
+y = peer.peer_ulysses_attention(x, tl)
+y.backward(dOut)
+x2 = S.clone().requires_grad_(True)
+y2 = A.ulysses_attention(x2, plan)
+y2.backward(dOut)
+torch.cuda.synchronize()
+assert U.ulysses_last_device_error(plan) == 0
+assert torch.equal(y.view(torch.int16), y2.view(torch.int16)), "training forward differs"
+assert torch.equal(x.grad.view(torch.int16), x2.grad.view(torch.int16)), "gradient differs"
+del tl
 dist.destroy_process_group()
 print("peer-layer-ok")
 """
@@ -156,7 +173,9 @@ print("peer-layer-ok")
 def test_peer_layer_one_rank_through_symmetric_memory(gpu):
     """PeerLayer end to end on a one-rank group (the only multi-process shape a
     one-GPU machine can run): symmetric-memory slabs, the push kernels and the
-    barriers, equal to the one-GPU layer bit for bit."""
+    barriers, equal to the one-GPU layer bit for bit; then a training step
+    through autograd, output and input gradient equal to the one-GPU
+    autograd layer's bit for bit."""
     import os
     import socket
     import subprocess
@@ -168,3 +187,69 @@ def test_peer_layer_one_rank_through_symmetric_memory(gpu):
     r = subprocess.run([sys.executable, "-c", _PEER_SCRIPT, str(port)], cwd=root, capture_output=True, text=True,
                        timeout=300)
     assert r.returncode == 0 and "peer-layer-ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
+
+
+TRAIN_CASES = [
+    pytest.param(2, 1024, 8, 3, None, False, 70, id="train-P2"),
+    pytest.param(4, 1001, 8, 4, None, False, 71, id="train-ragged-qkvg-P4"),
+    pytest.param(2, 1000, 4, 3, [0, 300, 300, 777, 1000], True, 72, id="train-causal-varlen-P2"),
+]
+
+
+@pytest.mark.parametrize("P,N,H,C,cu,causal,seed", TRAIN_CASES)
+def test_push_training_path_equals_one_gpu_backward(gpu, P, N, H, C, cu, causal, seed):
+    """The multi-GPU training path with the ranks emulated: per-slab attention
+    with lse, output pushed back, dO pushed into the slabs, the per-slab
+    backward, gradients pushed to their owners.  Output, lse and gradients
+    equal the one-GPU layer and ulysses_layer_bwd bit for bit."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    plan, S, shards, T = _setup(gpu, P, N, H, C, cu, causal, seed)
+    Np, Nl, Hl = plan.padded_tokens, plan.rows_per_rank, H // P
+    scale = 1.0 / math.sqrt(128)
+    g = torch.Generator(device=gpu)
+    g.manual_seed(seed + 1000)
+    dOut = torch.randn((Np, H, 128), generator=g, device=gpu).to(torch.bfloat16)
+    dOut[N:] = 0
+    # forward
+    for q in range(P):
+        U.ulysses_repack_fwd_push(plan, q, shards[q], T)
+    OTr = [torch.empty((Np, Hl, 128), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    lser = [torch.empty(plan.slab_lse_bytes // 4, dtype=torch.float32, device=gpu) for _ in range(P)]
+    O = [torch.full((Nl, H, 128), float("nan"), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for r in range(P):
+        U.ulysses_attn_fwd_lse_slab(plan, T[r], OTr[r], lser[r], scale)
+        U.ulysses_repack_bwd_push(plan, r, OTr[r], O, 1)
+    # backward
+    dOs = [dOut[q * Nl:(q + 1) * Nl].clone() for q in range(P)]
+    dOT = [torch.full((1, Np, Hl, 128), float("nan"), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for q in range(P):
+        U.ulysses_repack_fwd_push(plan, q, dOs[q], dOT, 1)
+    dq = [torch.empty((3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    G = [torch.full((Nl, 3, H, 128), float("nan"), dtype=torch.bfloat16, device=gpu) for _ in range(P)]
+    for r in range(P):
+        ws = torch.empty(plan.slab_attn_bwd_workspace_bytes, dtype=torch.uint8, device=gpu)
+        U.ulysses_attn_bwd_slab(plan, T[r], OTr[r], dOT[r], lser[r], dq[r], ws, scale)
+        U.ulysses_repack_bwd_push(plan, r, dq[r], G, 3)
+    # the one-GPU path
+    Tg = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=gpu)
+    U.ulysses_repack_fwd(plan, S, Tg)
+    U.ulysses_attn_fwd_lse(plan, Tg, OT, lse, scale)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_bwd(plan, OT, OS, 1)
+    dS = torch.zeros_like(S)
+    wsl = torch.empty(plan.layer_bwd_workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_layer_bwd(plan, Tg, OT, lse, dOut, dS, wsl)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    assert np.array_equal(np.concatenate([_bits(o) for o in O], 0), _bits(OS))
+    stride = plan.lse_row_stride
+    lse_h = lse.cpu().numpy().reshape(P, Hl, stride)[:, :, :Np]     # entries past Np are never written
+    for r in range(P):
+        mine = lser[r].cpu().numpy().reshape(Hl, stride)[:, :Np]
+        assert np.array_equal(mine, lse_h[r]), f"lse of rank {r}"
+        assert np.array_equal(_bits(OTr[r]), _bits(OT[r])), f"output slab of rank {r}"
+    got = np.concatenate([_bits(x) for x in G], 0)
+    assert np.array_equal(got, _bits(dS)[:, :3])

@@ -14,9 +14,11 @@ from ._lib import (  # noqa: F401
     load,
     strerror,
     ulysses_attn_bwd,
+    ulysses_attn_bwd_slab,
     ulysses_attn_fwd,
     ulysses_attn_fwd_fp8,
     ulysses_attn_fwd_lse,
+    ulysses_attn_fwd_lse_slab,
     ulysses_attn_fwd_push,
     ulysses_last_device_error,
     ulysses_layer_bwd,

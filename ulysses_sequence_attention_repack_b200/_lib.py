@@ -37,7 +37,7 @@ EXPORTS = (
     "ulysses_lse_bytes", "ulysses_attn_fwd_lse", "ulysses_attn_bwd_workspace_bytes", "ulysses_attn_bwd",
     "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd", "ulysses_repack_fwd_fp8", "ulysses_attn_fwd_fp8",
     "ulysses_workspace_bytes_fp8", "ulysses_layer_fwd_fp8", "ulysses_repack_fwd_push", "ulysses_attn_fwd_push",
-    "ulysses_repack_bwd_push",
+    "ulysses_repack_bwd_push", "ulysses_attn_fwd_lse_slab", "ulysses_attn_bwd_slab",
 )
 
 
@@ -124,12 +124,16 @@ def load() -> ctypes.CDLL:
         lib.ulysses_workspace_bytes_fp8.restype = sz
         lib.ulysses_layer_fwd_fp8.argtypes = [vp, vp, vp, vp, sz, vp]
         lib.ulysses_layer_fwd_fp8.restype = ctypes.c_int
-        lib.ulysses_repack_fwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), vp]
+        lib.ulysses_repack_fwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), i32, vp]
         lib.ulysses_repack_fwd_push.restype = ctypes.c_int
         lib.ulysses_attn_fwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), ctypes.c_float, vp]
         lib.ulysses_attn_fwd_push.restype = ctypes.c_int
         lib.ulysses_repack_bwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), i32, vp]
         lib.ulysses_repack_bwd_push.restype = ctypes.c_int
+        lib.ulysses_attn_fwd_lse_slab.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp]
+        lib.ulysses_attn_fwd_lse_slab.restype = ctypes.c_int
+        lib.ulysses_attn_bwd_slab.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, ctypes.c_float, vp]
+        lib.ulysses_attn_bwd_slab.restype = ctypes.c_int
         lib.ulysses_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
         lib.ulysses_selftest_exp2_poly.restype = ctypes.c_int
         _handle = lib
@@ -217,6 +221,16 @@ class Plan:
         return load().ulysses_attn_bwd_workspace_bytes(self.handle)
 
     @property
+    def slab_lse_bytes(self) -> int:
+        """lse bytes of one rank's slab (ulysses_attn_fwd_lse_slab)."""
+        return self.lse_bytes // self.P
+
+    @property
+    def slab_attn_bwd_workspace_bytes(self) -> int:
+        """Workspace of ulysses_attn_bwd_slab."""
+        return self.attn_bwd_workspace_bytes // self.P
+
+    @property
     def layer_bwd_workspace_bytes(self) -> int:
         return load().ulysses_layer_bwd_workspace_bytes(self.handle)
 
@@ -279,6 +293,22 @@ def ulysses_attn_bwd(plan: Plan, qkv_heads, out_heads, dout_heads, lse, dqkv_hea
                                    _stream(stream)), "ulysses_attn_bwd")
 
 
+def ulysses_attn_fwd_lse_slab(plan: Plan, heads, out_heads, lse, softmax_scale: float, stream=None) -> None:
+    """Attention over one rank's head slab [C, Np, Hl, D] with its lse."""
+    _check(load().ulysses_attn_fwd_lse_slab(plan.handle, _ptr(heads), _ptr(out_heads), _ptr(lse),
+                                            float(softmax_scale), _stream(stream)), "ulysses_attn_fwd_lse_slab")
+
+
+def ulysses_attn_bwd_slab(plan: Plan, heads, out_heads, dout_heads, lse, dqkv_heads, workspace,
+                          softmax_scale: float, workspace_bytes: int | None = None, stream=None) -> None:
+    """The attention backward of one rank's head slab: dqkv_heads [3, Np, Hl, D]."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(load().ulysses_attn_bwd_slab(plan.handle, _ptr(heads), _ptr(out_heads), _ptr(dout_heads), _ptr(lse),
+                                        _ptr(dqkv_heads), _ptr(workspace), int(workspace_bytes),
+                                        float(softmax_scale), _stream(stream)), "ulysses_attn_bwd_slab")
+
+
 def ulysses_layer_bwd(plan: Plan, qkv_heads, out_heads, lse, dout_seq, dqkv_seq, workspace,
                       workspace_bytes: int | None = None, stream=None) -> None:
     if workspace_bytes is None:
@@ -306,12 +336,15 @@ def _ptr_table(ptrs):
     return (ctypes.c_void_p * max(1, len(vals)))(*vals)
 
 
-def ulysses_repack_fwd_push(plan: Plan, rank: int, src_shard, dst_heads, stream=None) -> None:
-    """Rank `rank` pushes its shard [Nl, C, H, D] into every rank's head slab
-    dst_heads[r] = T_r [C, Np, Hl, D] (device pointers, one per rank)."""
+def ulysses_repack_fwd_push(plan: Plan, rank: int, src_shard, dst_heads, planes: int | None = None,
+                            stream=None) -> None:
+    """Rank `rank` pushes its shard [Nl, planes, H, D] into every rank's head
+    slab dst_heads[r] = T_r [planes, Np, Hl, D] (device pointers, one per
+    rank); planes defaults to the plan's C."""
     if dst_heads is not None and len(dst_heads) != plan.P:
         raise UlyssesError(ULYSSES_ERR_ARG, "ulysses_repack_fwd_push: one destination per rank")
-    _check(load().ulysses_repack_fwd_push(plan.handle, int(rank), _ptr(src_shard), _ptr_table(dst_heads),
+    planes = plan.planes if planes is None else int(planes)
+    _check(load().ulysses_repack_fwd_push(plan.handle, int(rank), _ptr(src_shard), _ptr_table(dst_heads), planes,
                                           _stream(stream)), "ulysses_repack_fwd_push")
 
 

@@ -340,6 +340,18 @@ int push_table(const ulysses_plan_t* p, void* const* ptrs, int64_t dst_bytes, co
   return ULYSSES_OK;
 }
 
+// One rank's view of a plan: the same sequence geometry (N, Np, segments,
+// causal flag, device error word) over that rank's Hl heads, as a one-rank
+// problem whose head-sharded buffers are the rank's slabs.
+ulysses_plan_t slab_view(const ulysses_plan_t* p) {
+  ulysses_plan_t v = *p;
+  v.P = 1;
+  v.H = p->Hl;
+  v.Nl = p->Np;
+  v.pipe = nullptr;
+  return v;
+}
+
 }  // namespace
 
 extern "C" {
@@ -783,20 +795,21 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
 }
 
 int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_shard,
-                            void* const* dst_heads, void* stream) {
-  if (!plan || !src_shard || !dst_heads || rank < 0 || rank >= plan->P) return ULYSSES_ERR_ARG;
+                            void* const* dst_heads, int32_t planes, void* stream) {
+  if (!plan || !src_shard || !dst_heads || rank < 0 || rank >= plan->P || planes < 1 || planes > plan->C)
+    return ULYSSES_ERR_ARG;
   if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
   if (!aligned16(src_shard)) return ULYSSES_ERR_ALIGN;
-  const int64_t shard_bytes = plan->Nl * plan->C * plan->H * plan->D * 2;
-  const int64_t slab_bytes = static_cast<int64_t>(plan->C) * plan->Np * plan->Hl * plan->D * 2;
+  const int64_t shard_bytes = plan->Nl * planes * plan->H * plan->D * 2;
+  const int64_t slab_bytes = static_cast<int64_t>(planes) * plan->Np * plan->Hl * plan->D * 2;
   ulysses::PushTable t;
   int s = push_table(plan, dst_heads, slab_bytes, src_shard, shard_bytes, &t);
   if (s != ULYSSES_OK) return s;
   if ((s = device_ready(plan)) != ULYSSES_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int32_t c0 = 0; c0 < plan->C; c0 += plan->plane_chunk) {
-    const int32_t cc = std::min(plan->plane_chunk, plan->C - c0);
-    s = status_of(ulysses::launch_push(0, src_shard, t, plan->Nl, plan->Np, plan->H, plan->P, plan->C, c0, cc, rank,
+  for (int32_t c0 = 0; c0 < planes; c0 += plan->plane_chunk) {
+    const int32_t cc = std::min(plan->plane_chunk, planes - c0);
+    s = status_of(ulysses::launch_push(0, src_shard, t, plan->Nl, plan->Np, plan->H, plan->P, planes, c0, cc, rank,
                                        st));
     if (s != ULYSSES_OK) return s;
   }
@@ -861,6 +874,22 @@ int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* 
   a.push_rows = plan->Nl;
   a.push_ranks = plan->P;
   return status_of(ulysses::launch_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+int ulysses_attn_fwd_lse_slab(const ulysses_plan_t* plan, const void* heads, void* out_heads, void* lse,
+                              float softmax_scale, void* stream) {
+  if (!plan) return ULYSSES_ERR_ARG;
+  const ulysses_plan_t v = slab_view(plan);
+  return ulysses_attn_fwd_lse(&v, heads, out_heads, lse, softmax_scale, stream);
+}
+
+int ulysses_attn_bwd_slab(const ulysses_plan_t* plan, const void* heads, const void* out_heads,
+                          const void* dout_heads, const void* lse, void* dqkv_heads, void* workspace,
+                          size_t workspace_bytes, float softmax_scale, void* stream) {
+  if (!plan) return ULYSSES_ERR_ARG;
+  const ulysses_plan_t v = slab_view(plan);
+  return ulysses_attn_bwd(&v, heads, out_heads, dout_heads, lse, dqkv_heads, workspace, workspace_bytes,
+                          softmax_scale, stream);
 }
 
 int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream) {

@@ -12,6 +12,16 @@ Rank q holds the sequence rows [q*Nl, (q+1)*Nl) of the input as a shard
      in one kernel);
   4. a barrier: every output shard is complete.
 
+For training (``training=True``) step 3 keeps this rank's head-sharded
+output and log-sum-exp (``ulysses_attn_fwd_lse_slab``, then
+``ulysses_repack_bwd_push`` of the output), and the backward is
+
+  5. ``ulysses_repack_fwd_push`` of the output gradient (one plane) into
+     every rank's dO slab, a barrier;
+  6. ``ulysses_attn_bwd_slab``: dQ, dK, dV of this rank's heads;
+  7. ``ulysses_repack_bwd_push`` of the three gradient planes into their
+     owners' gradient shards, a barrier.
+
 The slabs and shards are allocated in PyTorch's symmetric memory, which maps
 every rank's allocation into every peer (NVLink over NVSwitch) and provides
 the barrier; every byte of the layer is moved and computed by this library's
@@ -20,10 +30,12 @@ constructor checks that (``agree_plan``).
 """
 from __future__ import annotations
 
+import functools
 import math
 import os
 
-from ._lib import Plan, ulysses_attn_fwd_push, ulysses_repack_fwd_push
+from ._lib import (Plan, ulysses_attn_bwd_slab, ulysses_attn_fwd_lse_slab, ulysses_attn_fwd_push,
+                   ulysses_repack_bwd_push, ulysses_repack_fwd_push)
 
 
 def plan_signature(plan: Plan) -> tuple:
@@ -54,7 +66,8 @@ class PeerLayer:
     the current CUDA stream.
     """
 
-    def __init__(self, plan: Plan, group=None, device=None, softmax_scale: float | None = None):
+    def __init__(self, plan: Plan, group=None, device=None, softmax_scale: float | None = None,
+                 training: bool = False):
         import torch
         import torch.distributed as dist
         from torch.distributed import _symmetric_memory as symm
@@ -74,6 +87,20 @@ class PeerLayer:
         self._out_h = symm.rendezvous(self.out, self.group)
         self.heads_ptrs = self._peer_ptrs(self._heads_h, self.heads)
         self.out_ptrs = self._peer_ptrs(self._out_h, self.out)
+        self.training = bool(training)
+        if self.training:
+            # this rank's output and lse for the backward, the dO slab and the
+            # gradient shard the peers push into, and the backward's scratch
+            self.out_heads = torch.empty(Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
+            self.lse = torch.empty(plan.slab_lse_bytes // 4, dtype=torch.float32, device=self.device)
+            self.dout_heads = symm.empty(1, Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
+            self.dqkv_heads = torch.empty(3, Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
+            self.grad = symm.empty(Nl, 3, H, plan.D, dtype=torch.bfloat16, device=self.device)
+            self.bwd_ws = torch.empty(plan.slab_attn_bwd_workspace_bytes, dtype=torch.uint8, device=self.device)
+            self._dout_h = symm.rendezvous(self.dout_heads, self.group)
+            self._grad_h = symm.rendezvous(self.grad, self.group)
+            self.dout_ptrs = self._peer_ptrs(self._dout_h, self.dout_heads)
+            self.grad_ptrs = self._peer_ptrs(self._grad_h, self.grad)
 
     def _peer_ptrs(self, handle, local) -> list[int]:
         """Every rank's address of the same tensor, as mapped on this device."""
@@ -85,8 +112,61 @@ class PeerLayer:
         """shard: this rank's rows [Nl, C, H, D] (bf16, on this rank's device)."""
         ulysses_repack_fwd_push(self.plan, self.rank, shard, self.heads_ptrs)
         self._heads_h.barrier(channel=0)
-        ulysses_attn_fwd_push(self.plan, self.rank, self.heads, self.out_ptrs, self.scale)
+        if self.training:
+            ulysses_attn_fwd_lse_slab(self.plan, self.heads, self.out_heads, self.lse, self.scale)
+            ulysses_repack_bwd_push(self.plan, self.rank, self.out_heads, self.out_ptrs, 1)
+        else:
+            ulysses_attn_fwd_push(self.plan, self.rank, self.heads, self.out_ptrs, self.scale)
         self._out_h.barrier(channel=1)
         return self.out
 
     __call__ = forward
+
+    def backward(self, dout_shard):
+        """dout_shard: the gradient of this rank's output rows [Nl, H, D].
+        Returns this rank's (dQ, dK, dV) rows [Nl, 3, H, D] (reused by the
+        next backward).  Needs ``training=True`` and the forward of the same
+        input just before it on every rank."""
+        if not self.training:
+            raise RuntimeError("PeerLayer was built without training=True")
+        ulysses_repack_fwd_push(self.plan, self.rank, dout_shard, self.dout_ptrs, 1)
+        self._dout_h.barrier(channel=0)
+        ulysses_attn_bwd_slab(self.plan, self.heads, self.out_heads, self.dout_heads, self.lse, self.dqkv_heads,
+                              self.bwd_ws, self.scale)
+        ulysses_repack_bwd_push(self.plan, self.rank, self.dqkv_heads, self.grad_ptrs, 3)
+        self._grad_h.barrier(channel=1)
+        return self.grad
+
+
+@functools.lru_cache(maxsize=None)
+def _autograd():
+    import torch
+
+    class PeerUlyssesAttention(torch.autograd.Function):
+        """``out = PeerUlyssesAttention.apply(shard, layer)`` on every rank, with
+        ``layer`` a ``PeerLayer(..., training=True)``: the rank's output rows
+        [Nl, H, D] (a fresh tensor), and in the backward the gradient of its
+        input rows [Nl, C, H, D] (planes >= 3, a gate, get zeros)."""
+
+        @staticmethod
+        def forward(ctx, shard, layer):
+            ctx.layer = layer
+            ctx.planes = shard.shape[1]
+            return layer.forward(shard).clone()
+
+        @staticmethod
+        def backward(ctx, dout):
+            layer = ctx.layer
+            g = layer.backward(dout.to(torch.bfloat16).contiguous())
+            if ctx.planes == 3:
+                return g.clone(), None
+            full = torch.zeros((g.shape[0], ctx.planes) + tuple(g.shape[2:]), dtype=g.dtype, device=g.device)
+            full[:, :3].copy_(g)
+            return full, None
+
+    return PeerUlyssesAttention
+
+
+def peer_ulysses_attention(shard, layer: PeerLayer):
+    """Functional form: this rank's output rows, differentiable through ``layer``."""
+    return _autograd().apply(shard, layer)

@@ -286,6 +286,29 @@ int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* 
 int ulysses_repack_bwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_heads,
                             void* const* dst_seq, int32_t planes, void* stream);
 
+/* ---- all-to-all fallback (no peer access): the collective moves the bytes,
+ * these kernels pack and unpack them.  Chunk r of each buffer is what rank r
+ * receives (or sent), in rank order, as an all-to-all with equal splits
+ * (ncclAllToAll, torch.distributed.all_to_all_single) expects. */
+
+/* Plane `plane` of src_shard [Nl, planes, H, D] (planes = C for the layer's
+ * input, 1 for an output gradient) -> send [P, Nl, Hl, D]:
+ *   send[r, i, j, :] = src_shard[i, plane, r*Hl + j, :].
+ * After the exchange, rank r's receive buffer [P, Nl, Hl, D] is that plane of
+ * its head slab, rows in rank order.  Errors: ARG (planes outside 1..8, plane
+ * outside 0..planes-1, null or overlapping pointers), ALIGN, UNSUPPORTED, CUDA. */
+int ulysses_a2a_pack(const ulysses_plan_t* plan, const void* src_shard, int32_t planes, int32_t plane, void* send,
+                     void* stream);
+
+/* The output direction: a plane of a rank's head-sharded rows [Np, Hl, D] is
+ * already [P, Nl, Hl, D] in destination order; after the exchange,
+ * recv [P, Nl, Hl, D] (chunk r = rank r's heads of this rank's rows) goes to
+ * plane `plane` of out_shard [Nl, planes, H, D]:
+ *   out_shard[i, plane, r*Hl + j, :] = recv[r, i, j, :].
+ * Errors: as ulysses_a2a_pack. */
+int ulysses_a2a_unpack(const ulysses_plan_t* plan, const void* recv, void* out_shard, int32_t planes, int32_t plane,
+                       void* stream);
+
 /* Attention over ONE rank's head slab of the plan (steps 2 of the multi-GPU
  * layer for training): heads T_r [C, Np, Hl, D] -> out_heads [Np, Hl, D] and
  * lse [Hl][stride] (ulysses_lse_bytes(plan) / P bytes; the stride as

@@ -170,6 +170,27 @@ def test_push_argument_checks_before_any_device_work():
     pm = U.ulysses_plan(1024, 8, 128, 2, 3, 8 * 128, 1024 * 8 * 128)
     assert lib.ulysses_repack_fwd_push(pm.handle, 0, 0x10000, good, 3, None) == _lib.ULYSSES_ERR_UNSUPPORTED
     assert lib.ulysses_attn_fwd_push(pm.handle, 0, 0x10000, good, 0.1, None) == _lib.ULYSSES_ERR_UNSUPPORTED
+    # the all-to-all fallback's pack and unpack
+    assert lib.ulysses_a2a_pack(h, 0x10000, 3, 2, 0x40000000, None) in ok_codes
+    assert lib.ulysses_a2a_pack(h, 0x10000, 3, 3, 0x40000000, None) == _lib.ULYSSES_ERR_ARG      # plane >= planes
+    assert lib.ulysses_a2a_pack(h, 0x10000, 0, 0, 0x40000000, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_a2a_pack(h, 0x10000, 9, 0, 0x40000000, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_a2a_pack(h, 0x10008, 3, 0, 0x40000000, None) == _lib.ULYSSES_ERR_ALIGN
+    assert lib.ulysses_a2a_pack(h, 0x10000, 3, 0, 0x10000 + 512, None) == _lib.ULYSSES_ERR_ARG   # overlap
+    assert lib.ulysses_a2a_unpack(h, 0x10000, 0x40000000, 3, 1, None) in ok_codes
+    assert lib.ulysses_a2a_unpack(h, 0x10000, 0x40000000, 1, 1, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_a2a_unpack(h, 0x10000, 0x10000, 1, 0, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_a2a_pack(pm.handle, 0x10000, 3, 0, 0x40000000, None) == _lib.ULYSSES_ERR_UNSUPPORTED
+    # one rank's slab: the one-GPU checks on the slab's sizes
+    assert lib.ulysses_attn_fwd_lse_slab(h, 0x10000, 0x40000000, 0x50000000, 0.1, None) in ok_codes
+    assert lib.ulysses_attn_fwd_lse_slab(h, 0x10000, 0x10000, 0x50000000, 0.1, None) == _lib.ULYSSES_ERR_ARG
+    assert lib.ulysses_attn_fwd_lse_slab(None, 0x10000, 0x40000000, 0x50000000, 0.1, None) == _lib.ULYSSES_ERR_ARG
+    small = plan.slab_attn_bwd_workspace_bytes
+    assert small * 2 == plan.attn_bwd_workspace_bytes
+    assert lib.ulysses_attn_bwd_slab(h, 0x10000, 0x20000000, 0x30000000, 0x40000000, 0x50000000, 0x60000000,
+                                     small - 16, 0.1, None) == _lib.ULYSSES_ERR_WORKSPACE
+    assert lib.ulysses_attn_bwd_slab(h, 0x10000, 0x20000000, 0x30000000, 0x40000000, 0x50000000, 0x60000000,
+                                     small, 0.1, None) in ok_codes
     # the binding wants one destination per rank
     with pytest.raises(U.UlyssesError):
         U.ulysses_repack_fwd_push(plan, 0, 0x10000, [0x40000000], stream=0)

@@ -165,6 +165,16 @@ assert U.ulysses_last_device_error(plan) == 0
 assert torch.equal(y.view(torch.int16), y2.view(torch.int16)), "training forward differs"
 assert torch.equal(x.grad.view(torch.int16), x2.grad.view(torch.int16)), "gradient differs"
 del tl
+# the all-to-all fallback (NCCL moves the bytes): the same output and gradient
+cl = peer.CollectiveLayer(plan, training=True)
+x3 = S.clone().requires_grad_(True)
+y3 = peer.peer_ulysses_attention(x3, cl)
+y3.backward(dOut)
+torch.cuda.synchronize()
+assert U.ulysses_last_device_error(plan) == 0
+assert torch.equal(y3.view(torch.int16), y2.view(torch.int16)), "collective forward differs"
+assert torch.equal(x3.grad.view(torch.int16), x2.grad.view(torch.int16)), "collective gradient differs"
+del cl
 dist.destroy_process_group()
 print("peer-layer-ok")
 """
@@ -175,7 +185,8 @@ def test_peer_layer_one_rank_through_symmetric_memory(gpu):
     one-GPU machine can run): symmetric-memory slabs, the push kernels and the
     barriers, equal to the one-GPU layer bit for bit; then a training step
     through autograd, output and input gradient equal to the one-GPU
-    autograd layer's bit for bit."""
+    autograd layer's bit for bit, with PeerLayer and with the all-to-all
+    fallback (CollectiveLayer, NCCL)."""
     import os
     import socket
     import subprocess
@@ -253,3 +264,47 @@ def test_push_training_path_equals_one_gpu_backward(gpu, P, N, H, C, cu, causal,
         assert np.array_equal(_bits(OTr[r]), _bits(OT[r])), f"output slab of rank {r}"
     got = np.concatenate([_bits(x) for x in G], 0)
     assert np.array_equal(got, _bits(dS)[:, :3])
+
+
+@pytest.mark.parametrize("P,N,H,C,seed", [pytest.param(4, 1001, 8, 3, 73, id="P4-N1001"),
+                                          pytest.param(2, 777, 4, 4, 74, id="P2-qkvg"),
+                                          pytest.param(8, 2048, 16, 3, 75, id="P8")])
+def test_all_to_all_pack_unpack(gpu, P, N, H, C, seed):
+    """The all-to-all fallback's kernels, with the collective emulated by
+    moving the equal-split chunks between the ranks' buffers: the head slabs
+    equal the oracle's mode 0 bit for bit, the unpacked output equals the
+    one-GPU layer's rows, and a three-plane unpack lands in its plane."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    plan, S, shards, _ = _setup(gpu, P, N, H, C, None, False, seed)
+    Np, Nl, Hl = plan.padded_tokens, plan.rows_per_rank, H // P
+    send = [[torch.empty((P, Nl, Hl, 128), dtype=torch.bfloat16, device=gpu) for _ in range(C)] for _ in range(P)]
+    for q in range(P):
+        for c in range(C):
+            U.ulysses_a2a_pack(plan, shards[q], C, c, send[q][c])
+    # the exchange: rank r receives chunk r of every rank's send buffer, in rank order
+    heads = [torch.stack([torch.cat([send[q][c][r] for q in range(P)], 0) for c in range(C)], 0) for r in range(P)]
+    Tg = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, Tg)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_attn_fwd(plan, Tg, OT, 1.0 / math.sqrt(128))
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_bwd(plan, OT, OS, 1)
+    outs, three = [], []
+    for q in range(P):
+        recv = torch.stack([OT[r, q * Nl:(q + 1) * Nl] for r in range(P)], 0).contiguous()
+        o = torch.full((Nl, H, 128), float("nan"), dtype=torch.bfloat16, device=gpu)
+        U.ulysses_a2a_unpack(plan, recv, o, 1, 0)
+        g = torch.zeros((Nl, 3, H, 128), dtype=torch.bfloat16, device=gpu)
+        U.ulysses_a2a_unpack(plan, recv, g, 3, 1)
+        outs.append(o)
+        three.append(g)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    T_ref = orc.repack_fwd(_bits(S), P)
+    for r in range(P):
+        assert np.array_equal(_bits(heads[r]), T_ref[r]), f"head slab of rank {r}"
+    assert np.array_equal(np.concatenate([_bits(o) for o in outs], 0), _bits(OS))
+    for q in range(P):
+        g = _bits(three[q])
+        assert np.array_equal(g[:, 1], _bits(outs[q])) and not g[:, 0].any() and not g[:, 2].any()

@@ -13,6 +13,8 @@ from ._lib import (  # noqa: F401
     library_path,
     load,
     strerror,
+    ulysses_a2a_pack,
+    ulysses_a2a_unpack,
     ulysses_attn_bwd,
     ulysses_attn_bwd_slab,
     ulysses_attn_fwd,

@@ -37,7 +37,8 @@ EXPORTS = (
     "ulysses_lse_bytes", "ulysses_attn_fwd_lse", "ulysses_attn_bwd_workspace_bytes", "ulysses_attn_bwd",
     "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd", "ulysses_repack_fwd_fp8", "ulysses_attn_fwd_fp8",
     "ulysses_workspace_bytes_fp8", "ulysses_layer_fwd_fp8", "ulysses_repack_fwd_push", "ulysses_attn_fwd_push",
-    "ulysses_repack_bwd_push", "ulysses_attn_fwd_lse_slab", "ulysses_attn_bwd_slab",
+    "ulysses_repack_bwd_push", "ulysses_attn_fwd_lse_slab", "ulysses_attn_bwd_slab", "ulysses_a2a_pack",
+    "ulysses_a2a_unpack",
 )
 
 
@@ -130,6 +131,10 @@ def load() -> ctypes.CDLL:
         lib.ulysses_attn_fwd_push.restype = ctypes.c_int
         lib.ulysses_repack_bwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), i32, vp]
         lib.ulysses_repack_bwd_push.restype = ctypes.c_int
+        lib.ulysses_a2a_pack.argtypes = [vp, vp, i32, i32, vp, vp]
+        lib.ulysses_a2a_pack.restype = ctypes.c_int
+        lib.ulysses_a2a_unpack.argtypes = [vp, vp, vp, i32, i32, vp]
+        lib.ulysses_a2a_unpack.restype = ctypes.c_int
         lib.ulysses_attn_fwd_lse_slab.argtypes = [vp, vp, vp, vp, ctypes.c_float, vp]
         lib.ulysses_attn_fwd_lse_slab.restype = ctypes.c_int
         lib.ulysses_attn_bwd_slab.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, ctypes.c_float, vp]
@@ -291,6 +296,18 @@ def ulysses_attn_bwd(plan: Plan, qkv_heads, out_heads, dout_heads, lse, dqkv_hea
     _check(load().ulysses_attn_bwd(plan.handle, _ptr(qkv_heads), _ptr(out_heads), _ptr(dout_heads), _ptr(lse),
                                    _ptr(dqkv_heads), _ptr(workspace), int(workspace_bytes), float(softmax_scale),
                                    _stream(stream)), "ulysses_attn_bwd")
+
+
+def ulysses_a2a_pack(plan: Plan, src_shard, planes: int, plane: int, send, stream=None) -> None:
+    """Plane `plane` of a shard [Nl, planes, H, D] -> all-to-all send buffer [P, Nl, Hl, D]."""
+    _check(load().ulysses_a2a_pack(plan.handle, _ptr(src_shard), int(planes), int(plane), _ptr(send),
+                                   _stream(stream)), "ulysses_a2a_pack")
+
+
+def ulysses_a2a_unpack(plan: Plan, recv, out_shard, planes: int, plane: int, stream=None) -> None:
+    """All-to-all receive buffer [P, Nl, Hl, D] -> plane `plane` of a shard [Nl, planes, H, D]."""
+    _check(load().ulysses_a2a_unpack(plan.handle, _ptr(recv), _ptr(out_shard), int(planes), int(plane),
+                                     _stream(stream)), "ulysses_a2a_unpack")
 
 
 def ulysses_attn_fwd_lse_slab(plan: Plan, heads, out_heads, lse, softmax_scale: float, stream=None) -> None:

@@ -876,6 +876,40 @@ int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* 
   return status_of(ulysses::launch_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
+int ulysses_a2a_pack(const ulysses_plan_t* plan, const void* src_shard, int32_t planes, int32_t plane, void* send,
+                     void* stream) {
+  if (!plan || !src_shard || !send || planes < 1 || planes > kMaxPlanes || plane < 0 || plane >= planes)
+    return ULYSSES_ERR_ARG;
+  if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
+  if (!aligned16(src_shard) || !aligned16(send)) return ULYSSES_ERR_ALIGN;
+  const int64_t row = static_cast<int64_t>(plan->H) * plan->D;
+  const int64_t shard_bytes = plan->Nl * planes * row * 2;
+  const int64_t send_bytes = plan->Nl * row * 2;
+  if (overlap(src_shard, shard_bytes, send, send_bytes)) return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  // mode 0 over the shard's Nl rows, one plane: send [P, 1, Nl, Hl, D]
+  const uint8_t* src = static_cast<const uint8_t*>(src_shard) + static_cast<int64_t>(plane) * row * 2;
+  return status_of(ulysses::launch_repack(0, src, send, plan->Nl, plan->H, plan->P, 1, 0, 1, planes * row, row,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int ulysses_a2a_unpack(const ulysses_plan_t* plan, const void* recv, void* out_shard, int32_t planes, int32_t plane,
+                       void* stream) {
+  if (!plan || !recv || !out_shard || planes < 1 || planes > kMaxPlanes || plane < 0 || plane >= planes)
+    return ULYSSES_ERR_ARG;
+  if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
+  if (!aligned16(recv) || !aligned16(out_shard)) return ULYSSES_ERR_ALIGN;
+  const int64_t row = static_cast<int64_t>(plan->H) * plan->D;
+  if (overlap(recv, plan->Nl * row * 2, out_shard, plan->Nl * planes * row * 2)) return ULYSSES_ERR_ARG;
+  int s = device_ready(plan);
+  if (s != ULYSSES_OK) return s;
+  // mode 1 over Nl rows, one plane: recv [P, 1, Nl, Hl, D] -> plane `plane` of [Nl, planes, H, D]
+  uint8_t* dst = static_cast<uint8_t*>(out_shard) + static_cast<int64_t>(plane) * row * 2;
+  return status_of(ulysses::launch_repack(1, recv, dst, plan->Nl, plan->H, plan->P, 1, 0, 1, planes * row, row,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int ulysses_attn_fwd_lse_slab(const ulysses_plan_t* plan, const void* heads, void* out_heads, void* lse,
                               float softmax_scale, void* stream) {
   if (!plan) return ULYSSES_ERR_ARG;

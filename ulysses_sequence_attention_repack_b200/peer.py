@@ -34,8 +34,8 @@ import functools
 import math
 import os
 
-from ._lib import (Plan, ulysses_attn_bwd_slab, ulysses_attn_fwd_lse_slab, ulysses_attn_fwd_push,
-                   ulysses_repack_bwd_push, ulysses_repack_fwd_push)
+from ._lib import (Plan, ulysses_a2a_pack, ulysses_a2a_unpack, ulysses_attn_bwd_slab, ulysses_attn_fwd_lse_slab,
+                   ulysses_attn_fwd_push, ulysses_repack_bwd_push, ulysses_repack_fwd_push)
 
 
 def plan_signature(plan: Plan) -> tuple:
@@ -138,13 +138,79 @@ class PeerLayer:
         return self.grad
 
 
+class CollectiveLayer:
+    """The same layer where ranks cannot map each other's memory: the bytes
+    cross in ``torch.distributed.all_to_all_single`` (NCCL) and this library's
+    kernels pack and unpack them (``ulysses_a2a_pack`` / ``ulysses_a2a_unpack``)
+    around the one-slab attention.  One exchange per plane, as the transport
+    page's fallback to a bulk all-to-all.  Same interface as ``PeerLayer``;
+    the output and gradients are its bit for bit.
+    """
+
+    def __init__(self, plan: Plan, group=None, device=None, softmax_scale: float | None = None,
+                 training: bool = False):
+        import torch
+        import torch.distributed as dist
+        agree_plan(plan, group)
+        self.plan = plan
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.device = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(plan.D)
+        self.training = bool(training)
+        C, Np, Nl, H, D = plan.planes, plan.padded_tokens, plan.rows_per_rank, plan.H, plan.D
+        Hl = H // plan.P
+        bf = dict(dtype=torch.bfloat16, device=self.device)
+        self.heads = torch.empty(C, Np, Hl, D, **bf)
+        self.send = torch.empty(Np, Hl, D, **bf)          # [P, Nl, Hl, D] in destination order
+        self.recv = torch.empty(Np, Hl, D, **bf)
+        self.out = torch.empty(Nl, H, D, **bf)
+        self.out_heads = torch.empty(Np, Hl, D, **bf)
+        self.lse = torch.empty(plan.slab_lse_bytes // 4, dtype=torch.float32, device=self.device)
+        if self.training:
+            self.dout_heads = torch.empty(1, Np, Hl, D, **bf)
+            self.dqkv_heads = torch.empty(3, Np, Hl, D, **bf)
+            self.grad = torch.empty(Nl, 3, H, D, **bf)
+            self.bwd_ws = torch.empty(plan.slab_attn_bwd_workspace_bytes, dtype=torch.uint8, device=self.device)
+
+    def _exchange(self, dst, src):
+        import torch.distributed as dist
+        dist.all_to_all_single(dst, src, group=self.group)
+
+    def forward(self, shard):
+        p, C = self.plan, self.plan.planes
+        for c in range(C):
+            ulysses_a2a_pack(p, shard, C, c, self.send)
+            self._exchange(self.heads[c], self.send)
+        ulysses_attn_fwd_lse_slab(p, self.heads, self.out_heads, self.lse, self.scale)
+        self._exchange(self.recv, self.out_heads)
+        ulysses_a2a_unpack(p, self.recv, self.out, 1, 0)
+        return self.out
+
+    __call__ = forward
+
+    def backward(self, dout_shard):
+        if not self.training:
+            raise RuntimeError("CollectiveLayer was built without training=True")
+        p = self.plan
+        ulysses_a2a_pack(p, dout_shard, 1, 0, self.send)
+        self._exchange(self.dout_heads[0], self.send)
+        ulysses_attn_bwd_slab(p, self.heads, self.out_heads, self.dout_heads, self.lse, self.dqkv_heads,
+                              self.bwd_ws, self.scale)
+        for c in range(3):
+            self._exchange(self.recv, self.dqkv_heads[c])
+            ulysses_a2a_unpack(p, self.recv, self.grad, 3, c)
+        return self.grad
+
+
 @functools.lru_cache(maxsize=None)
 def _autograd():
     import torch
 
     class PeerUlyssesAttention(torch.autograd.Function):
         """``out = PeerUlyssesAttention.apply(shard, layer)`` on every rank, with
-        ``layer`` a ``PeerLayer(..., training=True)``: the rank's output rows
+        ``layer`` a ``PeerLayer`` or ``CollectiveLayer`` built with
+        ``training=True``: the rank's output rows
         [Nl, H, D] (a fresh tensor), and in the backward the gradient of its
         input rows [Nl, C, H, D] (planes >= 3, a gate, get zeros)."""
 
@@ -167,6 +233,6 @@ def _autograd():
     return PeerUlyssesAttention
 
 
-def peer_ulysses_attention(shard, layer: PeerLayer):
+def peer_ulysses_attention(shard, layer):
     """Functional form: this rank's output rows, differentiable through ``layer``."""
     return _autograd().apply(shard, layer)

@@ -16,7 +16,9 @@
  *      cu_seqlens).
  *   3. repack_bwd  -- mode 1, the inverse map, applied to the attention output.
  *
- * All P "virtual ranks" are slabs of one GPU's memory; there is no collective.
+ * In the one-GPU calls all P "virtual ranks" are slabs of one GPU's memory
+ * and there is no collective; the "multi-GPU push" section below runs the
+ * same steps with one process per GPU.
  *
  * Notation: N real tokens, P virtual ranks, H heads, D = 128 head dim,
  * Hl = H / P, C planes (3 = Q,K,V; 4 = Q,K,V,G), Nl = ceil(N / P),

@@ -513,8 +513,10 @@ def run_fp8(args, rank, world, local_rank):
     if rank != 0:
         return None
     pk, pk_kind = peaks()
-    tpk, tpk_kind = tensor_peak(pk)
-    fp8_peak = 2.0 * tpk                      # measured bf16 x the nominal fp8/bf16 ratio (4.5 / 2.25)
+    # measured bf16 x the nominal fp8/bf16 ratio (4.5 / 2.25).  The burst figure:
+    # this kernel draws less power and holds 1.78-1.84 GHz under back-to-back
+    # launches (measured inside the kernel), the clock regime of the burst GEMM
+    fp8_peak = 2.0 * pk["bf16_tflops"]
     flops = attn_flops(N, H, cu)
     at_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     rf_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
@@ -538,9 +540,10 @@ def run_fp8(args, rank, world, local_rank):
         "repack_fwd_fp8_gbs": round(rf_bytes / (rf_ms * 1e-3) / 1e9, 1),
         "repack_bwd_us": round(rb_ms * 1000, 2), "repack_bwd_gbs": round(rb_bytes / (rb_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<fp8>", "achieved": round(attn_tflops, 1),
-                     "peak": round(fp8_peak, 1), "peak_kind": f"{pk_kind} {tpk_kind} x 2 (E4M3 dense)",
+                     "peak": round(fp8_peak, 1), "peak_kind": f"{pk_kind} bf16 burst x 2 (E4M3 dense)",
                      "unit": "TFLOP/s", "frac": round(attn_tflops / fp8_peak, 3),
-                     "frac_of_burst": round(attn_tflops / (2.0 * pk["bf16_tflops"]), 3),
+                     "frac_of_sustained": round(attn_tflops / (2.0 * pk.get("bf16_tflops_sustained",
+                                                                            pk["bf16_tflops"])), 3),
                      "traffic": recorded_traffic("attn_fwd_kernel_fp8", args.config),
                      "algorithmic_flops_per_launch": flops},
         "e2e": {"value": round(e2e_ms * 1000, 2), "unit": "us per layer",

@@ -258,7 +258,8 @@ int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void*
  * (ulysses_repack_bwd_push with planes = 3).
  *
  * Pointer tables are HOST arrays of P device pointers indexed by rank; each
- * must be 16-byte aligned, non-null, and must not overlap the call's source.
+ * must be 16-byte aligned, non-null, and must not overlap the call's source
+ * or another entry's buffer.
  * The calls only store: the caller orders the exchange, i.e. rank r reads T_r
  * (or O_r) only after every rank's push into it has completed, with a
  * stream-ordered barrier (an NCCL all-reduce of one word on the same stream,

@@ -157,6 +157,8 @@ def test_push_argument_checks_before_any_device_work():
     assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, table(0x40000000, 0), 3, None) == _lib.ULYSSES_ERR_ARG
     assert lib.ulysses_repack_fwd_push(h, 0, 0x10008, good, 3, None) == _lib.ULYSSES_ERR_ALIGN
     assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, table(0x40000000, 0x50000004), 3, None) == _lib.ULYSSES_ERR_ALIGN
+    # two ranks' destinations overlapping each other
+    assert lib.ulysses_repack_fwd_push(h, 0, 0x10000, table(0x40000000, 0x40000000 + 4096), 3, None) == _lib.ULYSSES_ERR_ARG
     # a destination slab overlapping the source shard
     assert lib.ulysses_repack_fwd_push(h, 1, 0x10000, table(0x40000000, 0x10000 + 4096), 3, None) == _lib.ULYSSES_ERR_ARG
     assert lib.ulysses_attn_fwd_push(h, 1, 0x10000, good, 0.1, None) in ok_codes

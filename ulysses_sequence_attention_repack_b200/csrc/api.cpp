@@ -326,7 +326,8 @@ bool push_layout_ok(const ulysses_plan_t* p) {
 }
 
 // Copies the caller's P destination pointers into a kernel table.  Each must
-// be non-null and 16-byte aligned, and none may overlap the source range.
+// be non-null and 16-byte aligned, and none may overlap the source range or
+// another destination.
 int push_table(const ulysses_plan_t* p, void* const* ptrs, int64_t dst_bytes, const void* src, int64_t src_bytes,
                ulysses::PushTable* t) {
   if (!ptrs) return ULYSSES_ERR_ARG;
@@ -335,6 +336,8 @@ int push_table(const ulysses_plan_t* p, void* const* ptrs, int64_t dst_bytes, co
     if (!ptrs[r]) return ULYSSES_ERR_ARG;
     if (!aligned16(ptrs[r])) return ULYSSES_ERR_ALIGN;
     if (overlap(src, src_bytes, ptrs[r], dst_bytes)) return ULYSSES_ERR_ARG;
+    for (int32_t q = 0; q < r; ++q)
+      if (overlap(ptrs[q], dst_bytes, ptrs[r], dst_bytes)) return ULYSSES_ERR_ARG;
     t->p[r] = ptrs[r];
   }
   return ULYSSES_OK;

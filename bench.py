@@ -554,6 +554,70 @@ def run_fp8(args, rank, world, local_rank):
     }
 
 
+def run_transport(args, rank, world, local_rank):
+    """Opt-in (--transport peer|nccl): the layer across the N GPUs of the
+    launch, one rank per GPU, rank q holding rows [q*Nl, (q+1)*Nl) of the
+    workload: PeerLayer (pushes over peer memory, the inverse exchange fused
+    into attention) or CollectiveLayer (NCCL all-to-all around this library's
+    pack/unpack kernels).  The plan's P is the number of GPUs; the total
+    problem is fixed (strong scaling)."""
+    import torch
+    import torch.distributed as dist
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs, peer
+
+    dev = torch.device("cuda", local_rank)
+    _, N, H, C, seed, cu = WORKLOADS[args.config]
+    P = world
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu)
+    Nl = plan.rows_per_rank
+    S = inputs.qkv_seq(N, H, P, C, seed, dev)
+    shard = S[rank * Nl:(rank + 1) * Nl].clone()
+    del S
+    layer = peer.PeerLayer(plan) if args.transport == "peer" else peer.CollectiveLayer(plan)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        layer(shard)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    sampler.begin()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        layer(shard)
+    b.record(stream)
+    torch.cuda.synchronize()
+    sampler.end()
+    dist.barrier()
+    clocks = sampler.stop()
+    if U.ulysses_last_device_error(plan) != 0:
+        raise RuntimeError("a kernel reported a device error in the multi-GPU layer")
+    ms = torch.tensor([a.elapsed_time(b) / args.steps], dtype=torch.float64, device=dev)
+    dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    ms = ms.item()
+    del layer
+    if rank != 0:
+        return None
+    flops = attn_flops(N, H, cu)
+    per_rank = 3 if args.transport == "peer" else 2 + 2 * C   # launches (+ collectives) per rank per step
+    return {
+        "metric": "Ulysses layer µs; attn TFLOP/s and repack GB/s vs B200 peak",
+        "value": round(ms * 1000.0, 2), "unit": "us per layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic N(0,1) bf16, seeded",
+        "config": {"workload": f"{WORKLOAD_TEXT[args.config]}; split over {world} GPU(s), P = {world}",
+                   "name": args.config, "P": P, "N": N, "Np": plan.padded_tokens,
+                   "H": H, "D": 128, "planes": C, "seed": seed, "cu_seqlens": cu, "transport": args.transport,
+                   "step": "one rank per GPU: push (or all-to-all) -> attention -> inverse exchange"},
+        "attn_tflops_whole_job": round(flops / (ms * 1e-3) / 1e12, 1),
+        "e2e": None, "gpu_launches": per_rank * args.steps, "clocks": clocks,
+    }
+
+
 def run_repack_stress(args, rank, world, local_rank):
     """Repack forward + backward at 250k tokens (QKVG), then a GB/s sweep over N."""
     import torch
@@ -719,6 +783,9 @@ def main():
     ap.add_argument("--config", default="dit19k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--transport", default="replicas", choices=["replicas", "peer", "nccl"],
+                    help="replicas (default): every GPU runs the whole one-GPU layer; peer / nccl: "
+                         "the layer split across the launched GPUs, one rank each")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -731,16 +798,30 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    if world > 1:
+    multi = args.transport != "replicas"
+    if multi and (args.config in FP8 or args.config in CAUSAL or args.config == "stress250k"):
+        ap.error("--transport peer|nccl runs the bf16 non-causal layer configs")
+    if world > 1 or multi:
         import datetime
 
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
+        if world == 1:   # a one-rank group of its own
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            if "MASTER_PORT" not in os.environ:
+                import socket
+                with socket.socket() as sk:
+                    sk.bind(("127.0.0.1", 0))
+                    os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        if args.config == "stress250k":
+        if multi:
+            line = run_transport(args, rank, world, local_rank)
+        elif args.config == "stress250k":
             line = run_repack_stress(args, rank, world, local_rank)
         elif args.config in FP8:
             line = run_fp8(args, rank, world, local_rank)
@@ -749,7 +830,7 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:
-        if world > 1:
+        if world > 1 or multi:
             import torch.distributed as dist
             dist.destroy_process_group()
 

@@ -118,3 +118,95 @@ def test_group_size_must_match_the_plan(tmp_path):
     mp.start_processes(_world_mismatch_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2, start_method="spawn")
     for r in range(2):
         assert (tmp_path / f"world{r}.txt").read_text() == "refused: the plan has P=4 ranks but the group has 2"
+
+
+# ---- CollectiveLayer's multi-rank orchestration on CPU processes (gloo).
+# The CUDA kernels are replaced by CPU stand-ins that compute what the C ABI
+# documents (pack / unpack index maps, fp64 attention and its gradient per
+# head), so the test checks the host side that only several ranks exercise:
+# buffer shapes, chunk order of the exchanges, the plane loops, and the
+# backward's sequence.  The stand-ins and the reference share the same
+# per-head arithmetic, so the exchanged results must match bit for bit.
+
+def _attn_heads_f64(q, k, v, N, scale):
+    """[Np, Hl, D] each -> [Np, Hl, D] fp64; keys >= N masked, pad rows zero."""
+    Np = q.shape[0]
+    s = torch.einsum("nhd,mhd->hnm", q, k) * scale
+    s[:, :, N:] = -float("inf")
+    p = torch.softmax(s, dim=-1)
+    o = torch.einsum("hnm,mhd->nhd", p, v)
+    o[N:] = 0
+    return o
+
+
+def _fake_kernels(N):
+    def pack(plan, src, planes, plane, send, stream=None):
+        P, Nl, H = plan.P, plan.rows_per_rank, plan.H
+        Hl = H // P
+        send.view(P, Nl, Hl, 128).copy_(src.view(Nl, planes, P, Hl, 128)[:, plane].permute(1, 0, 2, 3))
+
+    def unpack(plan, recv, out, planes, plane, stream=None):
+        P, Nl, H = plan.P, plan.rows_per_rank, plan.H
+        Hl = H // P
+        out.view(Nl, planes, P, Hl, 128)[:, plane] = recv.view(P, Nl, Hl, 128).permute(1, 0, 2, 3)
+
+    def fwd(plan, heads, out_heads, lse, scale, stream=None):
+        q, k, v = (heads[c].double() for c in range(3))
+        out_heads.copy_(_attn_heads_f64(q, k, v, N, scale).to(torch.bfloat16))
+
+    def bwd(plan, heads, out_heads, dout_heads, lse, dqkv, ws, scale, stream=None):
+        q, k, v = (heads[c].double().requires_grad_(True) for c in range(3))
+        o = _attn_heads_f64(q, k, v, N, scale)
+        o.backward(dout_heads[0].double())
+        for c, t in enumerate((q, k, v)):
+            dqkv[c].copy_(t.grad.to(torch.bfloat16))
+
+    return pack, unpack, fwd, bwd
+
+
+def _collective_worker(rank, world, port, N, H, C, result_dir):
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import peer
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        plan = U.ulysses_plan(N, H, 128, world, C)
+        pack, unpack, fwd, bwd = _fake_kernels(N)
+        peer.ulysses_a2a_pack, peer.ulysses_a2a_unpack = pack, unpack
+        peer.ulysses_attn_fwd_lse_slab, peer.ulysses_attn_bwd_slab = fwd, bwd
+        S, dO = torch.load(os.path.join(result_dir, "inputs.pt"))
+        Nl = plan.rows_per_rank
+        layer = peer.CollectiveLayer(plan, device=torch.device("cpu"), training=True)
+        out = layer(S[rank * Nl:(rank + 1) * Nl].contiguous()).clone()
+        grad = layer.backward(dO[rank * Nl:(rank + 1) * Nl].contiguous()).clone()
+        torch.save((out, grad), os.path.join(result_dir, f"rank{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,N,H,C", [(2, 300, 4, 3), (4, 257, 8, 4)])
+def test_collective_layer_orchestration(tmp_path, world, N, H, C):
+    """CollectiveLayer over `world` CPU processes: every rank's output rows and
+    Q/K/V gradient rows equal the whole layer computed in one process."""
+    Np = -(-N // world) * world
+    g = torch.Generator().manual_seed(world * 100 + N)
+    S = torch.randn((Np, C, H, 128), generator=g).to(torch.bfloat16)
+    S[N:] = 0
+    dO = torch.randn((Np, H, 128), generator=g).to(torch.bfloat16)
+    dO[N:] = 0
+    torch.save((S, dO), tmp_path / "inputs.pt")
+    mp.start_processes(_collective_worker, args=(world, _free_port(), N, H, C, str(tmp_path)), nprocs=world,
+                       start_method="spawn")
+    # the reference: all heads over the whole sequence in one process
+    scale = 1.0 / np.sqrt(128)
+    q, k, v = (S[:, c].double().requires_grad_(True) for c in range(3))
+    o = _attn_heads_f64(q, k, v, N, scale)
+    o.backward(dO.double())
+    out_ref = o.detach().to(torch.bfloat16)
+    grad_ref = torch.stack([t.grad.to(torch.bfloat16) for t in (q, k, v)], 1)    # [Np, 3, H, D]
+    Nl = Np // world
+    for r in range(world):
+        out, grad = torch.load(tmp_path / f"rank{r}.pt")
+        assert torch.equal(out.view(torch.int16), out_ref[r * Nl:(r + 1) * Nl].view(torch.int16)), f"rank {r} output"
+        assert torch.equal(grad.view(torch.int16), grad_ref[r * Nl:(r + 1) * Nl].view(torch.int16)), f"rank {r} grad"

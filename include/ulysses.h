@@ -229,6 +229,17 @@ size_t ulysses_workspace_bytes_fp8(const ulysses_plan_t* plan);
 int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/*
+ * ulysses_layer_fwd_fp8 from HOST buffers, streamed by head groups exactly as
+ * ulysses_layer_fwd_host (same groups, streams, events and ordering against
+ * `stream`); the workspace is ulysses_workspace_bytes_fp8() long and holds
+ * the groups' E4M3 head slabs, then their outputs.  The result equals
+ * ulysses_layer_fwd_fp8's bit for bit.  Errors: as ulysses_layer_fwd_host.
+ */
+int ulysses_layer_fwd_fp8_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
+                               void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 /* ---------------------------------------------------------------- multi-GPU push
  * Steps 1 and 3 across P real GPUs, one process per GPU: rank q owns the
  * sequence rows [q*Nl, (q+1)*Nl).  These are the all-to-all exchanges of

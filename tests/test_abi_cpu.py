@@ -124,6 +124,10 @@ def test_launch_argument_checks_before_any_device_work():
     assert lib.ulysses_attn_fwd_fp8(h, 0x10000, 0x10000, 0.1, None) == _lib.ULYSSES_ERR_ARG
     assert lib.ulysses_attn_fwd_fp8(h, 0x10000, 0x90000000, 0.0, None) == _lib.ULYSSES_ERR_ARG
     assert lib.ulysses_layer_fwd_fp8(h, 0x10000, 0x90000000, None, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
+    fh = lib.ulysses_layer_fwd_fp8_host
+    assert fh(h, 0x30000000, 0x20000000, 0x10000, 0x90000000, None, 0, None) == _lib.ULYSSES_ERR_WORKSPACE
+    assert fh(h, 0x30000000, 0x20000000, 0x10008, 0x90000000, None, 0, None) == _lib.ULYSSES_ERR_ALIGN
+    assert fh(h, None, 0x20000000, 0x10000, 0x90000000, None, 0, None) == _lib.ULYSSES_ERR_ARG
     assert lib.ulysses_workspace_bytes_fp8(h) == ((1024 * 3 * 8 * 128 + 255) // 256 * 256 + 1024 * 8 * 128 * 2)
     # a gate-less plan cannot run attention
     p2 = U.ulysses_plan(1024, 8, 128, 2, 2)

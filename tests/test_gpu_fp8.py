@@ -122,3 +122,37 @@ def test_fp8_saturates_and_keeps_sign(gpu):
     want = orc.repack_fwd_fp8(_bits(S), P)
     np.testing.assert_array_equal(_u8(T8), want)
     assert {0x7E, 0xFE, 0x80}.issubset(set(np.unique(want).tolist()))
+
+
+@pytest.mark.parametrize("P,N,H,C,cu,seed", [pytest.param(2, 1024, 8, 3, None, 80, id="tiny"),
+                                             pytest.param(4, 1001, 8, 4, None, 81, id="ragged-qkvg"),
+                                             pytest.param(8, 2048, 16, 3, [0, 1024, 1536, 2048], 82, id="varlen-P8"),
+                                             pytest.param(2, 57_001, 8, 3, None, 83, id="head-groups")])
+def test_fp8_host_layer_equals_device_layer(gpu, P, N, H, C, cu, seed):
+    """ulysses_layer_fwd_fp8_host (copies and kernels streamed by head groups)
+    equals ulysses_layer_fwd_fp8 bit for bit, twice in a row on a non-default
+    stream that is the only thing synchronised."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu)
+    Np = plan.padded_tokens
+    S = inputs.qkv_seq(N, H, P, C, seed, gpu)
+    ws = torch.empty(plan.workspace_bytes_fp8, dtype=torch.uint8, device=gpu)
+    want = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_layer_fwd_fp8(plan, S, want, ws)
+    torch.cuda.synchronize()
+    want_bits = _bits(want)
+    host_in = S.cpu().pin_memory()
+    dev_in = torch.empty_like(S)
+    dev_out = torch.empty_like(want)
+    stream = torch.cuda.Stream(device=gpu)
+    for _ in range(2):
+        host_out = torch.full(want.shape, float("nan"), dtype=torch.bfloat16).pin_memory()
+        dev_in.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            U.ulysses_layer_fwd_fp8_host(plan, host_in, host_out, dev_in, dev_out, ws, stream=stream)
+        stream.synchronize()
+        assert U.ulysses_last_device_error(plan, stream) == 0
+        assert np.array_equal(host_out.view(torch.int16).numpy().view("uint16"), want_bits)

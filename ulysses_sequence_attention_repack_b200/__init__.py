@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     ulysses_layer_bwd,
     ulysses_layer_fwd,
     ulysses_layer_fwd_fp8,
+    ulysses_layer_fwd_fp8_host,
     ulysses_layer_fwd_fused_noalloc,
     ulysses_layer_fwd_host,
     ulysses_plan,

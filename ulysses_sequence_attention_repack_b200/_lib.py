@@ -38,7 +38,7 @@ EXPORTS = (
     "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd", "ulysses_repack_fwd_fp8", "ulysses_attn_fwd_fp8",
     "ulysses_workspace_bytes_fp8", "ulysses_layer_fwd_fp8", "ulysses_repack_fwd_push", "ulysses_attn_fwd_push",
     "ulysses_repack_bwd_push", "ulysses_attn_fwd_lse_slab", "ulysses_attn_bwd_slab", "ulysses_a2a_pack",
-    "ulysses_a2a_unpack",
+    "ulysses_a2a_unpack", "ulysses_layer_fwd_fp8_host",
 )
 
 
@@ -131,6 +131,8 @@ def load() -> ctypes.CDLL:
         lib.ulysses_attn_fwd_push.restype = ctypes.c_int
         lib.ulysses_repack_bwd_push.argtypes = [vp, i32, vp, ctypes.POINTER(vp), i32, vp]
         lib.ulysses_repack_bwd_push.restype = ctypes.c_int
+        lib.ulysses_layer_fwd_fp8_host.argtypes = [vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.ulysses_layer_fwd_fp8_host.restype = ctypes.c_int
         lib.ulysses_a2a_pack.argtypes = [vp, vp, i32, i32, vp, vp]
         lib.ulysses_a2a_pack.restype = ctypes.c_int
         lib.ulysses_a2a_unpack.argtypes = [vp, vp, vp, i32, i32, vp]
@@ -416,6 +418,16 @@ def ulysses_layer_fwd_host(plan: Plan, host_qkv_seq, host_out_seq, dev_qkv_seq, 
     _check(load().ulysses_layer_fwd_host(plan.handle, _ptr(host_qkv_seq), _ptr(host_out_seq), _ptr(dev_qkv_seq),
                                          _ptr(dev_out_seq), _ptr(workspace), int(workspace_bytes), int(fused),
                                          _stream(stream)), "ulysses_layer_fwd_host")
+
+
+def ulysses_layer_fwd_fp8_host(plan: Plan, host_qkv_seq, host_out_seq, dev_qkv_seq, dev_out_seq, workspace,
+                               workspace_bytes: int | None = None, stream=None) -> None:
+    """The FP8 layer from host buffers, streamed by head groups (workspace_bytes_fp8)."""
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().ulysses_layer_fwd_fp8_host(plan.handle, _ptr(host_qkv_seq), _ptr(host_out_seq), _ptr(dev_qkv_seq),
+                                             _ptr(dev_out_seq), _ptr(workspace), int(workspace_bytes),
+                                             _stream(stream)), "ulysses_layer_fwd_fp8_host")
 
 
 def ulysses_last_device_error(plan: Plan, stream=None) -> int:

@@ -277,8 +277,12 @@ cudaError_t copy_heads_in(const ulysses_plan_t* p, int32_t h0, int32_t hg, const
 // of S in, their columns of O_S out.  The kernels see the group as a one-rank
 // problem (P = 1, H = hg) at offset pointers; with fused = 0 its head slab and
 // attention output live in the caller's workspace at Tg / OTg.
+// mode: 0 = unfused bf16, 1 = fused bf16, 2 = unfused with the E4M3 cast
+// (Tg then holds one byte per element)
 int group_layer_impl(const ulysses_plan_t* p, int32_t h0, int32_t hg, const uint8_t* S, uint8_t* OS, uint8_t* Tg,
-                     uint8_t* OTg, int32_t fused, float scale, cudaStream_t st) {
+                     uint8_t* OTg, int32_t mode, float scale, cudaStream_t st) {
+  const int32_t fused = mode == 1;
+  const int32_t fp8 = mode == 2;
   const int64_t cols = static_cast<int64_t>(hg) * p->D;   // elements of the group's heads in a row
   const int64_t row = static_cast<int64_t>(p->H) * p->D;
   const uint8_t* Sg = S + static_cast<int64_t>(h0) * p->D * 2;
@@ -305,10 +309,13 @@ int group_layer_impl(const ulysses_plan_t* p, int32_t h0, int32_t hg, const uint
   }
   for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
     const int32_t cc = std::min(p->plane_chunk, p->C - c0);
-    int s = status_of(ulysses::launch_repack(0, Sg, Tg, p->Np, hg, 1, p->C, c0, cc, p->token_stride,
-                                             p->plane_stride, st));
+    int s = status_of(fp8 ? ulysses::launch_repack_fp8(Sg, Tg, p->Np, hg, 1, p->C, c0, cc, p->token_stride,
+                                                       p->plane_stride, st)
+                          : ulysses::launch_repack(0, Sg, Tg, p->Np, hg, 1, p->C, c0, cc, p->token_stride,
+                                                   p->plane_stride, st));
     if (s != ULYSSES_OK) return s;
   }
+  a.fp8 = fp8;
   a.base = Tg;
   a.out = OTg;
   a.o_stride_r = p->Np * cols;
@@ -731,11 +738,16 @@ int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out
   return repack_bwd_impl(plan, OT, out_seq, 1, st);
 }
 
-int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
-                           void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
-                           int32_t fused, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The host-buffer layer for the three modes of group_layer_impl.
+int layer_host_impl(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq, void* dev_qkv_seq,
+                    void* dev_out_seq, void* workspace, size_t workspace_bytes, int32_t mode, void* stream) {
   if (!plan || !host_qkv_seq || !host_out_seq || !dev_qkv_seq || !dev_out_seq) return ULYSSES_ERR_ARG;
-  if (plan->C < 3 || (fused != 0 && fused != 1)) return ULYSSES_ERR_ARG;
+  const int32_t fused = mode == 1;
+  if (plan->C < 3 || mode < 0 || mode > 2) return ULYSSES_ERR_ARG;
   if (!aligned16(dev_qkv_seq) || !aligned16(dev_out_seq)) return ULYSSES_ERR_ALIGN;
   const int64_t in_bytes = seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride);
   if (overlap(dev_qkv_seq, in_bytes, dev_out_seq, out_seq_bytes(plan)) ||
@@ -744,13 +756,14 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
   uint8_t* T = nullptr;
   uint8_t* OT = nullptr;
   if (!fused) {
-    if (!workspace || workspace_bytes < ulysses_workspace_bytes(plan)) return ULYSSES_ERR_WORKSPACE;
+    const size_t need = mode == 2 ? ulysses_workspace_bytes_fp8(plan) : ulysses_workspace_bytes(plan);
+    if (!workspace || workspace_bytes < need) return ULYSSES_ERR_WORKSPACE;
     if (!aligned16(workspace)) return ULYSSES_ERR_ALIGN;
-    const int64_t ws = static_cast<int64_t>(ulysses_workspace_bytes(plan));
+    const int64_t ws = static_cast<int64_t>(need);
     if (overlap(workspace, ws, dev_qkv_seq, in_bytes) || overlap(workspace, ws, dev_out_seq, out_seq_bytes(plan)))
       return ULYSSES_ERR_ARG;
     T = static_cast<uint8_t*>(workspace);
-    OT = T + align_up(heads_bytes(plan, plan->C), 256);
+    OT = T + align_up(mode == 2 ? heads_bytes_fp8(plan, plan->C) : heads_bytes(plan, plan->C), 256);
   }
   int s = device_ready(plan);
   if (s != ULYSSES_OK) return s;
@@ -783,9 +796,9 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
     if (cudaStreamWaitEvent(st, h->in[g], 0) != cudaSuccess) return status_of(cudaErrorUnknown);
     uint8_t* Tg = fused ? nullptr : T + t_off;
     uint8_t* OTg = fused ? nullptr : OT + o_off;
-    t_off += static_cast<int64_t>(plan->C) * plan->Np * static_cast<int64_t>(width);
+    t_off += static_cast<int64_t>(plan->C) * plan->Np * static_cast<int64_t>(width) / (mode == 2 ? 2 : 1);
     o_off += plan->Np * static_cast<int64_t>(width);
-    if ((s = group_layer_impl(plan, h0, hg, din, dout, Tg, OTg, fused, scale, st)) != ULYSSES_OK) return s;
+    if ((s = group_layer_impl(plan, h0, hg, din, dout, Tg, OTg, mode, scale, st)) != ULYSSES_OK) return s;
     if (cudaEventRecord(h->out[g], st) != cudaSuccess || cudaStreamWaitEvent(h->d2h, h->out[g], 0) != cudaSuccess ||
         cudaMemcpy2DAsync(hout + off, pitch, dout + off, pitch, width, static_cast<size_t>(plan->Np),
                           cudaMemcpyDeviceToHost, h->d2h) != cudaSuccess)
@@ -795,6 +808,25 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
   if (cudaEventRecord(h->done, h->d2h) != cudaSuccess || cudaStreamWaitEvent(st, h->done, 0) != cudaSuccess)
     return status_of(cudaErrorUnknown);
   return ULYSSES_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
+                           void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
+                           int32_t fused, void* stream) {
+  if (fused != 0 && fused != 1) return ULYSSES_ERR_ARG;
+  return layer_host_impl(plan, host_qkv_seq, host_out_seq, dev_qkv_seq, dev_out_seq, workspace, workspace_bytes,
+                         fused, stream);
+}
+
+int ulysses_layer_fwd_fp8_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
+                               void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return layer_host_impl(plan, host_qkv_seq, host_out_seq, dev_qkv_seq, dev_out_seq, workspace, workspace_bytes, 2,
+                         stream);
 }
 
 int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_shard,

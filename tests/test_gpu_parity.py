@@ -28,6 +28,8 @@ CASES = [
     pytest.param(2, 1000, 4, 3, "token", [0, 300, 300, 777, 1000, 1000], 37, id="varlen-empty-segments"),
     pytest.param(1, 1, 1, 3, "token", None, 11, id="N1"),
     pytest.param(4, 5, 4, 3, "token", None, 12, id="N5-P4"),
+    # one head per rank across 56 ranks (the Video-DiT head count): 56 runs per row
+    pytest.param(56, 1000, 56, 3, "token", None, 38, id="P56-Hl1"),
 ]
 
 

@@ -28,6 +28,7 @@ CASES = [
     pytest.param(2, 1000, 4, 3, [0, 300, 300, 777, 1000], True, 64, id="causal-varlen-P2"),
     pytest.param(4, 5, 4, 3, None, False, 65, id="N5-P4"),
     pytest.param(1, 300, 2, 3, None, False, 66, id="P1"),
+    pytest.param(56, 1000, 56, 3, None, False, 76, id="P56-Hl1"),
 ]
 
 

@@ -1,0 +1,112 @@
+"""Host-side logic of bench.py that the reported numbers rest on (no GPU)."""
+import importlib.util
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    argv = sys.argv
+    sys.argv = ["bench.py"]
+    try:
+        spec.loader.exec_module(mod)
+    finally:
+        sys.argv = argv
+    return mod
+
+
+class _FakeProc:
+    def __init__(self, text):
+        self.text = text
+
+    def terminate(self):
+        pass
+
+    def communicate(self, timeout=None):
+        return self.text, ""
+
+
+def _line(stamp, mhz, watts, cap):
+    return f"{stamp}, {mhz}, 1965, {watts}, Not Active, Not Active, Not Active, {cap}"
+
+
+def test_clock_samples_are_taken_inside_the_timed_region(bench, monkeypatch):
+    """Idle samples before and after the timed region do not enter the median,
+    and throttle reasons count only inside it."""
+    s = bench.ClockSampler(0)
+    base = bench.ClockSampler._stamp("2026/12/02 10:00:00.000")
+    lines = [_line("2026/12/02 10:00:00.000", 1965, 240, "Not Active"),    # idle, before
+             _line("2026/12/02 10:00:00.500", 1600, 990, "Active"),        # loaded
+             _line("2026/12/02 10:00:00.700", 1580, 1000, "Active"),
+             _line("2026/12/02 10:00:00.900", 1620, 980, "Active"),
+             _line("2026/12/02 10:00:01.500", 1965, 250, "Not Active")]    # idle, after
+    s.proc = _FakeProc("\n".join(lines))
+    s.t0, s.t1 = base + 0.4, base + 1.0
+    monkeypatch.setattr(bench.time, "sleep", lambda _: None)
+    c = s.stop()
+    assert c["samples"] == 3 and c["window"] == "timed region"
+    assert c["sm_mhz"] == 1600 and c["power_w"] == 990
+    assert c["reasons"] == ["sw_power_cap"] and c["sm_max_mhz"] == 1965
+
+
+def test_short_region_falls_back_to_the_loaded_samples(bench, monkeypatch):
+    s = bench.ClockSampler(0)
+    base = bench.ClockSampler._stamp("2026/12/02 10:00:00.000")
+    lines = [_line("2026/12/02 10:00:00.000", 1965, 240, "Not Active"),
+             _line("2026/12/02 10:00:00.100", 1700, 900, "Active"),
+             _line("2026/12/02 10:00:00.200", 1965, 245, "Not Active")]
+    s.proc = _FakeProc("\n".join(lines))
+    s.t0, s.t1 = base + 0.12, base + 0.15      # no sample falls inside
+    monkeypatch.setattr(bench.time, "sleep", lambda _: None)
+    c = s.stop()
+    assert c["samples"] == 1 and c["sm_mhz"] == 1700 and c["window"].startswith("samples at")
+    assert c["reasons"] == ["sw_power_cap"]
+
+
+def test_without_nvidia_smi_the_clock_is_reported_missing(bench):
+    s = bench.ClockSampler(0)
+    s.proc = None
+    assert s.stop()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_percentiles_are_nearest_rank(bench):
+    xs = [5.0, 1.0, 4.0, 2.0, 3.0]
+    assert bench.pct(xs, 50) == 3.0
+    assert bench.pct(xs, 95) == 5.0
+    assert bench.pct(xs, 0) == 1.0
+    assert bench.pct([7.0], 95) == 7.0
+
+
+def test_attention_denominator_is_the_sustained_peak(bench):
+    pk = {"hbm_gbs": 6549.4, "bf16_tflops": 1642.9, "bf16_tflops_sustained": 1392.3}
+    assert bench.tensor_peak(pk) == (1392.3, "bf16 sustained")
+    assert bench.tensor_peak({"bf16_tflops": 1590.0})[0] == 1590.0
+
+
+def test_algorithmic_flops(bench):
+    # 4 N^2 H D for one sequence; varlen sums the segments; causal counts n + 1 keys per row
+    assert bench.attn_flops(1024, 8, None) == 4 * 1024 ** 2 * 8 * 128
+    assert bench.attn_flops(100, 2, [0, 60, 100]) == 4 * (60 ** 2 + 40 ** 2) * 2 * 128
+    assert bench.attn_flops(4, 1, None, causal=True) == 4 * 128 * (4 * 5 // 2)
+
+
+def test_traffic_record_is_void_once_the_source_changes(bench, tmp_path, monkeypatch):
+    import json
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    src = tmp_path / "ulysses_sequence_attention_repack_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k.cu").write_text("kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"k": {"w": {"source": "k.cu", "source_sha256_16": bench.source_hash("k.cu"), "dram_bytes_per_launch": 42}}}
+    (prof / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("k", "w") == 42
+    (src / "k.cu").write_text("kernel v2")
+    assert bench.recorded_traffic("k", "w") is None
+    assert bench.recorded_traffic("k", "other") is None

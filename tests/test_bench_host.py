@@ -110,3 +110,20 @@ def test_traffic_record_is_void_once_the_source_changes(bench, tmp_path, monkeyp
     (src / "k.cu").write_text("kernel v2")
     assert bench.recorded_traffic("k", "w") is None
     assert bench.recorded_traffic("k", "other") is None
+
+
+def test_peer_pointer_table_keeps_the_tensor_offset():
+    """PeerLayer maps its tensor's address on every rank from the symmetric
+    allocation's base addresses plus the tensor's offset inside its own."""
+    from ulysses_sequence_attention_repack_b200 import peer
+
+    class Handle:
+        buffer_ptrs = [0x7000_0000_0000, 0x7100_0000_0000, 0x7200_0000_0000]
+
+    class Local:
+        def data_ptr(self):
+            return 0x7100_0000_0000 + 4096
+
+    layer = peer.PeerLayer.__new__(peer.PeerLayer)
+    layer.rank = 1
+    assert layer._peer_ptrs(Handle(), Local()) == [0x7000_0000_1000, 0x7100_0000_1000, 0x7200_0000_1000]

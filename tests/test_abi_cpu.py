@@ -208,3 +208,41 @@ def test_strerror_covers_every_code():
     for code in range(9):
         assert U.strerror(code) != "unknown error code"
     assert U.strerror(99) == "unknown error code"
+
+
+def test_a_plain_c_program_links_the_library(tmp_path):
+    """The boundary is a C ABI: a C99 program that includes only
+    include/ulysses.h links libulysses.so, creates a plan and reads its sizes
+    (no GPU needed: launches would return ULYSSES_ERR_CUDA)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib = U.library_path()
+    U.load()   # builds the library if the sources are newer
+    src = tmp_path / "probe.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "ulysses.h"
+int main(void) {
+  ulysses_plan_t* p = NULL;
+  int s = ulysses_plan(&p, 19394, 56, 128, 4, 3, 0, 0, 0, NULL, 0);
+  if (s != ULYSSES_OK) return 10 + s;
+  printf("%lld %lld %zu %s\n", (long long)ulysses_plan_padded_tokens(p),
+         (long long)ulysses_plan_window_bytes_per_plane(p), ulysses_workspace_bytes(p), ulysses_strerror(ULYSSES_ERR_ALIGN));
+  int bad = ulysses_repack_fwd(p, NULL, NULL, NULL);
+  ulysses_plan_destroy(p);
+  return bad == ULYSSES_ERR_ARG ? 0 : 20;
+}
+''')
+    exe = tmp_path / "probe"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-L", os.path.dirname(lib), "-l:" + os.path.basename(lib),
+                    "-Wl,-rpath," + os.path.dirname(lib), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out
+    Np, window, ws = out.stdout.split()[:3]
+    assert int(Np) == 19396
+    assert int(window) == 4849 * 56 * 128 * 2
+    assert int(ws) > 0 and "16-byte" in out.stdout

@@ -27,3 +27,16 @@ def gpu():
         pytest.fail("a gpu-marked test ran without a CUDA device")
     import torch
     return torch.device("cuda", 0)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print the rel-L2 of every attention comparison made against the oracle."""
+    try:
+        import _parity
+    except ImportError:
+        return
+    if not _parity.RECORDS:
+        return
+    terminalreporter.write_sep("-", "attention parity against the fp64 oracle")
+    for label, r, mx, mn, gate in _parity.RECORDS:
+        terminalreporter.write_line(f"{label}: rel-L2 {r:.3e} (gate {gate:g}), max-abs {mx:.2e}, mean-abs {mn:.2e}")

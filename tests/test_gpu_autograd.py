@@ -9,6 +9,7 @@ import math
 
 import numpy as np
 import pytest
+from _parity import check_attention
 
 from oracle import ulysses_oracle as orc
 
@@ -19,6 +20,7 @@ def _close(got, ref, what, max_rel=2e-2, mean_rel=5e-3):
     err = np.abs(got - ref)
     assert err.max() <= max_rel * np.abs(ref).max(), (what, float(err.max()))
     assert err.mean() <= mean_rel * np.abs(ref).mean(), (what, float(err.mean()))
+    check_attention(f"autograd {what}", got, ref, max_abs=None, mean_abs=None)
 
 
 @pytest.mark.parametrize("P,N,H,C,layout,cu,causal", [

@@ -18,6 +18,7 @@ import math
 
 import numpy as np
 import pytest
+from _parity import REL_L2_FP8, check_attention
 
 from oracle import ulysses_oracle as orc
 
@@ -83,10 +84,11 @@ def test_fp8_layer_against_oracle(gpu, P, N, H, C, layout, cu, causal, seed):
     bound = 2.0 ** -4 * A[:, :N] + 2.0 ** -8 * np.abs(ref[:, :N]) + 2e-3
     assert np.all(err <= bound), float((err / bound).max())
     segs = orc.segments_from_cu_seqlens(cu, N)
-    if not causal and min(b - a for a, b in segs if b > a) >= 512:
-        # every row averages over at least 512 keys: the statistical bound of
-        # the layer holds (causal rows near a segment start see few keys)
-        assert err.mean() <= MEAN_ABS, err.mean()
+    # every row averages over at least 512 keys: the statistical bound of the
+    # layer holds for mean-abs (causal rows near a segment start see few keys)
+    many_keys = not causal and min(b - a for a, b in segs if b > a) >= 512
+    check_attention(f"FP8 P={P} N={N} H={H} C={C} {layout} cu={cu} causal={causal}", got[:, :N], ref[:, :N],
+                    max_abs=None, mean_abs=MEAN_ABS if many_keys else None, rel_gate=REL_L2_FP8)
     # the layer is step 3 applied to that output, bit for bit
     np.testing.assert_array_equal(_bits(OS), orc.repack_bwd(_bits(OT)[:, None])[:, 0])
 

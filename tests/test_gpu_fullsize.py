@@ -12,13 +12,12 @@ import os
 
 import numpy as np
 import pytest
+from _parity import MEAN_ABS, REL_L2_FP8, check_attention
 
 from oracle import ulysses_oracle as orc
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-MAX_ABS = 2e-2
-MEAN_ABS = 2e-3
 ROWS_PER_HEAD = 4096
 
 # name: (P, N, H, C, seed, cu_seqlens)
@@ -89,9 +88,7 @@ def test_full_layer(gpu, name):
     del T_bits
     idx = torch.from_numpy(rows).to(gpu)
     got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
-    err = np.abs(got - ref)
-    assert err.max() <= MAX_ABS, err.max()
-    assert err.mean() <= MEAN_ABS, err.mean()
+    check_attention(f"full size {name}, {rows.size} rows x {H} heads", got, ref)
     # step 3: the layer output rows are the attention rows, heads regrouped
     lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
     assert np.array_equal(lay, orc.output_repack_bwd(got))
@@ -144,8 +141,42 @@ def test_full_layer_causal_dit19k(gpu):
     ref = orc.attention_heads(inputs.host_bits(T[:, :3]), N, 1.0 / math.sqrt(128), rows=rows, causal=True)
     idx = torch.from_numpy(rows).to(gpu)
     got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
-    err = np.abs(got - ref)
-    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    check_attention(f"full size dit19k causal, {rows.size} rows x {H} heads", got, ref)
+    lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(lay, orc.output_repack_bwd(got))
+
+
+def test_full_layer_sharp_softmax_dit19k(gpu):
+    """Q scaled by 8 at the Video-DiT size (logits of standard deviation 8):
+    the weight of each row sits on a handful of its 19,394 keys, and the
+    running max moves many times per row, so the O rescale in TMEM runs at
+    full size.  4096 seeded rows per head against fp64, in the benchmark's
+    call sequence; the fused layer equal to the unfused one bit for bit."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    P, N, H, C, seed = 4, 19_394, 56, 3, 1
+    plan = U.ulysses_plan(N, H, 128, P, C)
+    Np, Hl = plan.padded_tokens, H // P
+    S = inputs.qkv_seq(N, H, P, C, seed, gpu)
+    S[:, 0] *= 8                     # exact in bf16 (a power of two)
+    T = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    OS = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    OSf = torch.empty_like(OS)
+    scale = 1.0 / math.sqrt(128)
+    U.ulysses_repack_fwd(plan, S, T)
+    U.ulysses_attn_fwd(plan, T, OT, scale)
+    U.ulysses_repack_bwd(plan, OT, OS, 1)
+    U.ulysses_layer_fwd(plan, S, OSf, None, fused=1)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    assert torch.equal(OS, OSf)
+    rows = orc.sample_rows(N, ROWS_PER_HEAD, seed)
+    ref = orc.attention_heads(inputs.host_bits(T[:, :3]), N, scale, rows=rows, workers=_cores())
+    idx = torch.from_numpy(rows).to(gpu)
+    got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
+    check_attention(f"full size dit19k sharp softmax (Q x 8), {rows.size} rows x {H} heads", got, ref)
     lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
     assert np.array_equal(lay, orc.output_repack_bwd(got))
 
@@ -184,7 +215,8 @@ def test_full_layer_fp8_dit19k(gpu):
     got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
     err = np.abs(got - ref)
     assert np.all(err <= 2.0 ** -4 * A + 2.0 ** -8 * np.abs(ref) + 2e-3), float(err.max())
-    assert err.mean() <= MEAN_ABS, err.mean()
+    check_attention(f"full size dit19k FP8, {rows.size} rows x {H} heads", got, ref, max_abs=None,
+                    mean_abs=MEAN_ABS, rel_gate=REL_L2_FP8)
     lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
     assert np.array_equal(lay, orc.output_repack_bwd(got))
     assert not OS[N:].any()

@@ -8,13 +8,11 @@ import math
 
 import numpy as np
 import pytest
+from _parity import MAX_ABS, MEAN_ABS, check_attention
 
 from oracle import ulysses_oracle as orc
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS = 2e-2
-MEAN_ABS = 2e-3
 
 # (P, N, H, C, layout, cu_seqlens, seed)
 CASES = [
@@ -98,15 +96,11 @@ def test_repack_attention_layer_against_oracle(gpu, P, N, H, C, layout, cu, seed
     scale = 1.0 / math.sqrt(128)
     O_ref = orc.attention_heads(T_ref, N, scale, cu_seqlens=cu)
     O_gpu = _f32(OT)
-    err = np.abs(O_gpu - O_ref)
-    assert err.max() <= MAX_ABS, err.max()
-    assert err.mean() <= MEAN_ABS, err.mean()
+    check_attention(f"attn P={P} N={N} H={H} C={C} {layout} cu={cu}", O_gpu, O_ref)
     assert np.all(O_gpu[:, N:] == 0)
     # the whole layer: oracle composition, and fused == unfused bit for bit
     L_ref = orc.output_repack_bwd(O_ref)
-    L_gpu = _f32(OS)
-    errl = np.abs(L_gpu - L_ref)
-    assert errl.max() <= MAX_ABS and errl.mean() <= MEAN_ABS
+    check_attention(f"layer P={P} N={N} H={H} C={C} {layout} cu={cu}", _f32(OS), L_ref)
     assert np.array_equal(_bits(OS), _bits(OSf))
     # step 3 on the attention output equals the layer output bit for bit
     assert np.array_equal(_bits(OS), orc.repack_bwd(_bits(OT)[:, None])[:, 0])
@@ -142,8 +136,7 @@ def test_causal_attention_against_oracle(gpu, P, N, H, cu, seed):
     torch.cuda.synchronize()
     assert U.ulysses_last_device_error(plan) == 0
     ref = orc.attention_heads(_bits(T), N, 1.0 / math.sqrt(128), cu_seqlens=cu, causal=True)
-    err = np.abs(_f32(OT) - ref)
-    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    check_attention(f"causal P={P} N={N} H={H} cu={cu}", _f32(OT), ref)
     assert np.all(_f32(OT)[:, N:] == 0)
     assert np.array_equal(_bits(OS), _bits(OSf))
     assert np.array_equal(_bits(OS), orc.repack_bwd(_bits(OT)[:, None])[:, 0])
@@ -168,8 +161,7 @@ def test_sharp_softmax_diagnostic(gpu):
     U.ulysses_layer_fwd(plan, S, OS, None, fused=1)
     torch.cuda.synchronize()
     ref = orc.layer_fwd(_bits(S), P, N, 1.0 / math.sqrt(128))
-    err = np.abs(_f32(OS) - ref)
-    assert err.max() <= 4 * MAX_ABS and err.mean() <= MEAN_ABS
+    check_attention("sharp softmax (Q x 8) P=2 N=1024 H=4", _f32(OS), ref, max_abs=4 * MAX_ABS)
 
 
 def test_uniform_keys_give_mean_of_v(gpu):
@@ -186,8 +178,7 @@ def test_uniform_keys_give_mean_of_v(gpu):
     torch.cuda.synchronize()
     v = _f32(S[:N, 2])                                 # [N, H, D]
     want = np.broadcast_to(v.mean(axis=0, keepdims=True), v.shape)
-    err = np.abs(_f32(OS) - want)
-    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+    check_attention("uniform keys P=2 N=700 H=4", _f32(OS), want)
 
 
 HOST_CASES = [
@@ -238,5 +229,4 @@ def test_host_layer_streams_ranks_exactly(gpu, P, N, H, C, layout, cu, causal, s
     if N <= 4096:   # the device layer at larger N is checked against the oracle in the full-size tests
         ref = orc.layer_fwd(_seq_as_token_major(_bits(S), layout), P, N, 1.0 / math.sqrt(128), cu_seqlens=cu,
                             causal=causal)
-        err = np.abs(_f32(want) - ref)
-        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+        check_attention(f"host layer P={P} N={N} H={H} causal={causal}", _f32(want), ref)

@@ -8,6 +8,7 @@ norm and rotation (bounded here by 1e-5 of the terms' magnitude), i.e.
 """
 import numpy as np
 import pytest
+from _parity import check_attention
 
 from oracle import ulysses_oracle as orc
 
@@ -97,8 +98,7 @@ def test_prologue_feeds_attention(gpu):
     U.ulysses_attn_fwd(plan, T, OT, 1.0 / math.sqrt(128))
     torch.cuda.synchronize()
     ref = orc.attention_heads(inputs.host_bits(T), N, 1.0 / math.sqrt(128))
-    err = np.abs(OT.float().cpu().numpy() - ref)
-    assert err.max() <= 2e-2 and err.mean() <= 2e-3
+    check_attention(f"prologue -> attention P={P} N={N} H={H}", OT.float().cpu().numpy(), ref)
 
 
 def test_prologue_argument_checks(gpu):

@@ -14,6 +14,7 @@ import math
 
 import numpy as np
 import pytest
+from _parity import check_attention
 
 from oracle import ulysses_oracle as orc
 
@@ -124,8 +125,7 @@ def test_push_attention_against_oracle(gpu):
     torch.cuda.synchronize()
     got = torch.cat(O, 0).float().cpu().numpy().astype(np.float64)
     ref = orc.layer_fwd(_bits(S), P, N, scale)
-    err = np.abs(got - ref)[:N]
-    assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+    check_attention(f"push layer P={P} N={N} H={H}", got[:N], ref[:N])
     assert np.all(got[N:] == 0)
 
 

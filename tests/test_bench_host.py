@@ -83,10 +83,37 @@ def test_percentiles_are_nearest_rank(bench):
     assert bench.pct([7.0], 95) == 7.0
 
 
-def test_attention_denominator_is_the_sustained_peak(bench):
+def test_attention_denominator_is_the_burst_peak(bench):
+    """The roofline divides by the larger (burst) GEMM figure; the sustained
+    one is only reported beside it."""
     pk = {"hbm_gbs": 6549.4, "bf16_tflops": 1642.9, "bf16_tflops_sustained": 1392.3}
-    assert bench.tensor_peak(pk) == (1392.3, "bf16 sustained")
+    assert bench.tensor_peak(pk) == (1642.9, "bf16 burst")
+    assert bench.sustained_peak(pk) == 1392.3
     assert bench.tensor_peak({"bf16_tflops": 1590.0})[0] == 1590.0
+    assert bench.sustained_peak({"bf16_tflops": 1590.0}) == 1590.0
+
+
+def test_default_workload_is_the_largest_single_gpu_layer(bench):
+    P, N, H, C, seed, cu = bench.WORKLOADS["long104k"]
+    assert (P, N, H, C, seed, cu) == (8, 104_448, 56, 3, 3, None)
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    assert 'default="long104k"' in src
+
+
+def test_both_oracle_legs_use_one_sample_definition(bench):
+    """cpu_baseline and --impl reference call oracle_sample with the same
+    defaults: 4096 rows per head of two heads, extrapolated x N/rows x H/heads."""
+    import numpy as np
+    from ulysses_sequence_attention_repack_b200 import inputs
+    assert bench.ORACLE_ROWS_PER_HEAD == 4096 and bench.ORACLE_HEADS == 2
+    S = inputs.qkv_seq(1024, 8, 2, 3, 0, "cpu")
+    us, sample = bench.oracle_sample("tiny", inputs.host_bits(S))
+    assert us > 0
+    # N = 1024 <= 4096: every row of every head of rank 0, x 2 for rank 1's heads
+    assert "1024 query rows x 4 heads" in sample and "x1.00 rows x 2.0 heads" in sample
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    assert "oracle_sample(args.config, S_bits)" in src and "oracle_sample(config, S_bits)" in src
+    assert np.isfinite(us)
 
 
 def test_algorithmic_flops(bench):

@@ -441,7 +441,10 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
  * Synchronise `stream`, then read and clear the plan's device error word.
  * Returns 0 when no kernel reported an error, otherwise the error bits
  * (1 = a pipeline wait timed out and the kernel gave up; 2 = a work unit
- * decoded outside the problem), or -1 if the synchronisation itself failed.
+ * decoded outside the problem; 4 = in the bounds-checked build
+ * libulysses_debug.so only, a computed global offset fell outside its
+ * buffer and the access was skipped), or -1 if the synchronisation itself
+ * failed.
  */
 int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream);
 
@@ -460,19 +463,23 @@ int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream);
  * library holds until the process exits.  Each call clears the word on
  * `stream` before launching.  All calls share that array, so calls that
  * overlap on the GPU (other streams, other threads) race on it.  The first
- * call on each device looks up the array's device address (and may trigger
- * the library's lazy module load): make that first call before any stream
- * capture.  A call never needs more than the 4 bytes, whatever N, H or P; a
- * scratch requirement above the 256-byte maximum would be refused with
+ * call in each CUDA context (a device's primary context, and again after a
+ * cudaDeviceReset or with another driver-API context current) looks up the
+ * array's device address in that context (and may trigger the library's
+ * lazy module load): make that first call before any stream capture.  A call
+ * never needs more than the 4 bytes, whatever N, H or P; a scratch
+ * requirement above the 256-byte maximum would be refused with
  * ULYSSES_ERR_UNSUPPORTED.
  *
  * Arguments as ulysses_plan() (planes must be >= 3) and ulysses_layer_fwd():
  * qkv_seq / out_seq are device buffers ([Np, C, H, D] by default strides,
- * [Np, H, D] out).  host_status: NULL for a fully asynchronous call;
- * otherwise the call synchronises `stream` after the launch and stores the
- * kernel's error bits there (0 = none; ULYSSES_ERR_DEVICE is returned when
- * they are non-zero).  Errors: ARG, DIVISIBILITY, ALIGN, UNSUPPORTED, CUDA,
- * DEVICE.
+ * [Np, H, D] out).  host_status: NULL for a fully asynchronous call, which
+ * then reports no device-side errors (a timed-out wait or a bad work unit
+ * leaves a wrong output that nothing reports, and the next call clears the
+ * word); otherwise the call synchronises `stream` after the launch and
+ * stores the kernel's error bits there (0 = none; ULYSSES_ERR_DEVICE is
+ * returned when they are non-zero).  Errors: ARG, DIVISIBILITY, ALIGN,
+ * UNSUPPORTED, CUDA, DEVICE.
  */
 int ulysses_layer_fwd_fused_noalloc(const void* qkv_seq, void* out_seq, int64_t N, int32_t H, int32_t D,
                                     int32_t P, int32_t planes, int64_t token_stride, int64_t plane_stride,

@@ -1,5 +1,6 @@
 /*
- * ulysses_selftest.h -- test hooks of libulysses.so (not part of the layer).
+ * ulysses_selftest.h -- test hooks, exported by libulysses_selftest.so (a
+ * library of its own, built beside libulysses.so; not part of the layer).
  *
  * These entry points run single device helpers of the kernels on their own,
  * so tests can compare them with reference values.
@@ -33,6 +34,16 @@ int ulysses_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream
  * Returns 0, 1 for a bad argument, 6 for a CUDA launch error.
  */
 int ulysses_selftest_wait_timeout(unsigned int* dev_err, int64_t limit_us, void* stream);
+
+/*
+ * The range check of the bounds-checked build (-DULYSSES_DEBUG), forced on
+ * in this hook: offsets 0, -8 and 96 of 8 elements against an extent of 100.
+ * The first is inside and sets 0x10 in *dev_err; the other two are refused,
+ * each setting bit 4 (out of bounds) and 0x20 / 0x40 respectively.  No memory
+ * but *dev_err is touched.  Returns 0, 1 for a bad argument, 6 for a CUDA
+ * launch error.
+ */
+int ulysses_selftest_bounds_check(unsigned int* dev_err, void* stream);
 
 #ifdef __cplusplus
 }

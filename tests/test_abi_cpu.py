@@ -11,9 +11,8 @@ from ulysses_sequence_attention_repack_b200 import _lib
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def declared_symbols():
-    import glob
-    text = "".join(open(h).read() for h in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
+def declared_symbols(header="ulysses.h"):
+    text = open(os.path.join(ROOT, "include", header)).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(ulysses_\w+)\s*\(", text)))
 
@@ -25,6 +24,23 @@ def test_library_exports_every_declared_symbol():
     for name in syms:
         assert hasattr(lib, name), name
     assert set(syms) == set(U.EXPORTS)
+
+
+def test_test_hooks_live_outside_the_product_library():
+    """include/ulysses_selftest.h is served by libulysses_selftest.so alone."""
+    import ctypes
+
+    import _selftest_lib
+    hooks = declared_symbols("ulysses_selftest.h")
+    assert set(hooks) == set(_selftest_lib.SELFTEST_EXPORTS)
+    lib = U.load()
+    test_lib = _selftest_lib.load()
+    for name in hooks:
+        assert hasattr(test_lib, name), name
+        with pytest.raises(AttributeError):
+            getattr(ctypes.CDLL(U.library_path()), name)
+    assert not set(hooks) & set(U.EXPORTS)
+    assert lib is not None
 
 
 def test_library_built_for_sm100a():

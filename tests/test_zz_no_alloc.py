@@ -11,11 +11,9 @@ import ctypes
 
 import numpy as np
 import pytest
+from _parity import check_attention
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS = 2e-2
-MEAN_ABS = 2e-3
 
 
 def _call(lib, S, out, N, H, P, C, cu):
@@ -47,9 +45,34 @@ def test_no_alloc_matches_fused_layer_on_two_calls(gpu):
         code, status = _call(lib, S, out, N, H, P, C, cu)
         torch.cuda.synchronize()
         assert code == 0 and status == 0, (code, status)
-        err = np.abs(out.float().cpu().numpy() - ref.float().cpu().numpy())
-        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+        check_attention(f"no-alloc vs fused layer P={P} N={N}", out.float().cpu().numpy(),
+                        ref.float().cpu().numpy())
         assert torch.equal(out, ref)      # same kernel, same tile order: identical bits
+
+
+def test_no_alloc_leaves_device_memory_untouched(gpu):
+    """After a first call (which looks up the scratch address in this
+    context), further calls change neither the device's free memory nor
+    torch's allocation counters."""
+    import torch
+    from ulysses_sequence_attention_repack_b200 import inputs
+    lib = __import__("ulysses_sequence_attention_repack_b200").load()
+    P, N, H, C = 2, 1000, 8, 3
+    S = inputs.qkv_seq(N, H, P, C, 33, gpu)
+    out = torch.empty((S.shape[0], H, 128), dtype=torch.bfloat16, device=gpu)
+    first = _call(lib, S, out, N, H, P, C, None)
+    torch.cuda.synchronize()
+    assert first == (0, 0)
+    free0, _ = torch.cuda.mem_get_info(gpu)
+    stats0 = torch.cuda.memory_stats(gpu)
+    for _ in range(2):
+        assert _call(lib, S, out, N, H, P, C, None) == (0, 0)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info(gpu)
+    stats1 = torch.cuda.memory_stats(gpu)
+    assert free1 == free0
+    for key in ("allocation.all.allocated", "segment.all.allocated", "reserved_bytes.all.current"):
+        assert stats1.get(key, 0) == stats0.get(key, 0), key
 
 
 def test_no_alloc_rejects_bad_arguments(gpu):

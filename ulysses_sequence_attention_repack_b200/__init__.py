@@ -36,5 +36,4 @@ from ._lib import (  # noqa: F401
     ulysses_repack_fwd,
     ulysses_repack_fwd_fp8,
     ulysses_repack_fwd_push,
-    ulysses_selftest_exp2_poly,
 )

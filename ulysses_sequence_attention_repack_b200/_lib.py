@@ -32,8 +32,8 @@ EXPORTS = (
     "ulysses_plan", "ulysses_plan_ex", "ulysses_plan_destroy", "ulysses_plan_padded_tokens", "ulysses_plan_plane_chunk",
     "ulysses_plan_window_bytes_per_plane", "ulysses_workspace_bytes", "ulysses_repack_fwd",
     "ulysses_repack_bwd", "ulysses_attn_fwd", "ulysses_layer_fwd", "ulysses_layer_fwd_host",
-    "ulysses_last_device_error", "ulysses_strerror", "ulysses_selftest_exp2_poly",
-    "ulysses_layer_fwd_fused_noalloc", "ulysses_selftest_wait_timeout", "ulysses_prologue_repack_fwd",
+    "ulysses_last_device_error", "ulysses_strerror",
+    "ulysses_layer_fwd_fused_noalloc", "ulysses_prologue_repack_fwd",
     "ulysses_lse_bytes", "ulysses_attn_fwd_lse", "ulysses_attn_bwd_workspace_bytes", "ulysses_attn_bwd",
     "ulysses_layer_bwd_workspace_bytes", "ulysses_layer_bwd", "ulysses_repack_fwd_fp8", "ulysses_attn_fwd_fp8",
     "ulysses_workspace_bytes_fp8", "ulysses_layer_fwd_fp8", "ulysses_repack_fwd_push", "ulysses_attn_fwd_push",
@@ -53,7 +53,10 @@ _handle: ctypes.CDLL | None = None
 
 
 def library_path() -> str:
-    return _build.LIB
+    """The library this process loads: $ULYSSES_LIBRARY when set (for
+    example the bounds-checked libulysses_debug.so), else the in-tree
+    libulysses.so."""
+    return os.environ.get("ULYSSES_LIBRARY") or _build.LIB
 
 
 def load() -> ctypes.CDLL:
@@ -62,9 +65,9 @@ def load() -> ctypes.CDLL:
     with _lock:
         if _handle is not None:
             return _handle
-        path = _build.ensure_built()
+        path = os.environ.get("ULYSSES_LIBRARY") or _build.ensure_built()
         if not os.path.exists(path):
-            raise ImportError(f"libulysses.so missing at {path}")
+            raise ImportError(f"libulysses library missing at {path}")
         lib = ctypes.CDLL(path)
         vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         lib.ulysses_plan.argtypes = [ctypes.POINTER(vp), i64, i32, i32, i32, i32, i64, i64, i64,
@@ -115,8 +118,6 @@ def load() -> ctypes.CDLL:
                                                         ctypes.POINTER(ctypes.c_int32), i32,
                                                         ctypes.POINTER(ctypes.c_int32), vp]
         lib.ulysses_layer_fwd_fused_noalloc.restype = ctypes.c_int
-        lib.ulysses_selftest_wait_timeout.argtypes = [vp, i64, vp]
-        lib.ulysses_selftest_wait_timeout.restype = ctypes.c_int
         lib.ulysses_repack_fwd_fp8.argtypes = [vp, vp, vp, vp]
         lib.ulysses_repack_fwd_fp8.restype = ctypes.c_int
         lib.ulysses_attn_fwd_fp8.argtypes = [vp, vp, vp, ctypes.c_float, vp]
@@ -141,8 +142,6 @@ def load() -> ctypes.CDLL:
         lib.ulysses_attn_fwd_lse_slab.restype = ctypes.c_int
         lib.ulysses_attn_bwd_slab.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, ctypes.c_float, vp]
         lib.ulysses_attn_bwd_slab.restype = ctypes.c_int
-        lib.ulysses_selftest_exp2_poly.argtypes = [vp, vp, i64, vp]
-        lib.ulysses_selftest_exp2_poly.restype = ctypes.c_int
         _handle = lib
         return lib
 
@@ -434,19 +433,14 @@ def ulysses_last_device_error(plan: Plan, stream=None) -> int:
     return load().ulysses_last_device_error(plan.handle, _stream(stream))
 
 
-def ulysses_selftest_exp2_poly(x, y, stream=None) -> None:
-    """y = 2^x with the attention kernel's FMA-pipe exponential (float32 device tensors)."""
-    _check(load().ulysses_selftest_exp2_poly(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)),
-           "ulysses_selftest_exp2_poly")
-
-
 def ulysses_layer_fwd_fused_noalloc(qkv_seq, out_seq, N: int, H: int, D: int, P: int, planes: int,
                                     token_stride: int = 0, plane_stride: int = 0, cu_seqlens=None,
                                     check: bool = False, stream=None) -> int:
     """The fused layer without a plan and without any device allocation.
 
     Returns the kernel's error bits when ``check`` is true (the call then
-    synchronises the stream), else 0.
+    synchronises the stream; non-zero bits are returned, not raised), else 0.
+    Argument and CUDA errors raise UlyssesError.
     """
     if cu_seqlens is None:
         arr, ns = None, 0
@@ -458,5 +452,7 @@ def ulysses_layer_fwd_fused_noalloc(qkv_seq, out_seq, N: int, H: int, D: int, P:
     code = load().ulysses_layer_fwd_fused_noalloc(_ptr(qkv_seq), _ptr(out_seq), int(N), int(H), int(D), int(P),
                                                   int(planes), int(token_stride), int(plane_stride), arr, ns,
                                                   ctypes.byref(status) if check else None, _stream(stream))
+    if check and code == ULYSSES_ERR_DEVICE:
+        return status.value
     _check(code, "ulysses_layer_fwd_fused_noalloc")
     return status.value

@@ -2,6 +2,7 @@
 // launch sequence of the three steps.  Declarations and argument contracts
 // are in include/ulysses.h.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -13,6 +14,31 @@
 #include "internal.h"
 
 namespace {
+
+// NVTX ranges (domain "ulysses") around every launching entry point and
+// around the three steps inside the layer calls, so a timeline profiler
+// shows repack -> attention -> inverse repack.  Without a profiler attached
+// a range costs one function-pointer check.
+nvtxDomainHandle_t nvtx_domain() {
+  static const nvtxDomainHandle_t d = nvtxDomainCreateA("ulysses");
+  return d;
+}
+
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) {
+    nvtxEventAttributes_t a;
+    std::memset(&a, 0, sizeof(a));
+    a.version = NVTX_VERSION;
+    a.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+    a.messageType = NVTX_MESSAGE_TYPE_ASCII;
+    a.message.ascii = name;
+    nvtxDomainRangePushEx(nvtx_domain(), &a);
+  }
+  ~NvtxRange() { nvtxDomainRangePop(nvtx_domain()); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int32_t kHeadDim = 128;
 constexpr int32_t kMaxHeads = 1024;
@@ -59,7 +85,7 @@ int repack_fwd_impl(const ulysses_plan_t* p, const void* src, void* dst, cudaStr
   for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
     const int32_t cc = std::min(p->plane_chunk, p->C - c0);
     int s = status_of(ulysses::launch_repack(0, src, dst, p->Np, p->H, p->P, p->C, c0, cc, p->token_stride,
-                                             p->plane_stride, st));
+                                             p->plane_stride, st, p->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   return ULYSSES_OK;
@@ -82,7 +108,8 @@ int repack_bwd_impl(const ulysses_plan_t* p, const void* src, void* dst, int32_t
   // same window rule as the forward direction: at most plane_chunk planes per launch
   for (int32_t c0 = 0; c0 < planes; c0 += p->plane_chunk) {
     const int32_t cc = std::min(p->plane_chunk, planes - c0);
-    int s = status_of(ulysses::launch_repack(1, src, dst, p->Np, p->H, p->P, planes, c0, cc, tok, pl, st));
+    int s = status_of(
+        ulysses::launch_repack(1, src, dst, p->Np, p->H, p->P, planes, c0, cc, tok, pl, st, p->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   return ULYSSES_OK;
@@ -126,7 +153,7 @@ int repack_fwd_fp8_impl(const ulysses_plan_t* p, const void* src, void* dst, cud
   for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
     const int32_t cc = std::min(p->plane_chunk, p->C - c0);
     int s = status_of(ulysses::launch_repack_fp8(src, dst, p->Np, p->H, p->P, p->C, c0, cc, p->token_stride,
-                                                 p->plane_stride, st));
+                                                 p->plane_stride, st, p->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   return ULYSSES_OK;
@@ -310,9 +337,9 @@ int group_layer_impl(const ulysses_plan_t* p, int32_t h0, int32_t hg, const uint
   for (int32_t c0 = 0; c0 < p->C; c0 += p->plane_chunk) {
     const int32_t cc = std::min(p->plane_chunk, p->C - c0);
     int s = status_of(fp8 ? ulysses::launch_repack_fp8(Sg, Tg, p->Np, hg, 1, p->C, c0, cc, p->token_stride,
-                                                       p->plane_stride, st)
+                                                       p->plane_stride, st, p->dev_err)
                           : ulysses::launch_repack(0, Sg, Tg, p->Np, hg, 1, p->C, c0, cc, p->token_stride,
-                                                   p->plane_stride, st));
+                                                   p->plane_stride, st, p->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   a.fp8 = fp8;
@@ -322,7 +349,8 @@ int group_layer_impl(const ulysses_plan_t* p, int32_t h0, int32_t hg, const uint
   a.o_stride_n = cols;
   int s = status_of(ulysses::launch_attn(a, st));
   if (s != ULYSSES_OK) return s;
-  return status_of(ulysses::launch_repack(1, OTg, OSg, p->Np, hg, 1, 1, 0, 1, row, row, st));
+  return status_of(
+      ulysses::launch_repack(1, OTg, OSg, p->Np, hg, 1, 1, 0, 1, row, row, st, p->dev_err));
 }
 
 // Multi-GPU push: the plan must describe the default token-interleaved
@@ -493,6 +521,7 @@ size_t ulysses_workspace_bytes(const ulysses_plan_t* plan) {
 }
 
 int ulysses_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads, void* stream) {
+  NvtxRange range("ulysses_repack_fwd");
   if (!plan || !src_seq || !dst_heads) return ULYSSES_ERR_ARG;
   if (!aligned16(src_seq) || !aligned16(dst_heads)) return ULYSSES_ERR_ALIGN;
   if (overlap(src_seq, seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride), dst_heads,
@@ -505,6 +534,7 @@ int ulysses_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* ds
 
 int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* dst_seq, int32_t planes,
                        void* stream) {
+  NvtxRange range("ulysses_repack_bwd");
   if (!plan || !src_heads || !dst_seq) return ULYSSES_ERR_ARG;
   if (planes < 1 || planes > plan->C) return ULYSSES_ERR_ARG;
   if (!aligned16(src_heads) || !aligned16(dst_seq)) return ULYSSES_ERR_ALIGN;
@@ -520,6 +550,7 @@ int ulysses_repack_bwd(const ulysses_plan_t* plan, const void* src_heads, void* 
 int ulysses_prologue_repack_fwd(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads,
                                 const void* norm_q_weight, const void* norm_k_weight, const void* cos_table,
                                 const void* sin_table, int32_t rotary_dim, float eps, void* stream) {
+  NvtxRange range("ulysses_prologue_repack_fwd");
   if (!plan || !src_seq || !dst_heads || !norm_q_weight || !norm_k_weight) return ULYSSES_ERR_ARG;
   if (plan->C < 2 || !(eps > 0.f) || !std::isfinite(eps)) return ULYSSES_ERR_ARG;
   if (rotary_dim < 0 || rotary_dim > plan->D) return ULYSSES_ERR_ARG;
@@ -539,7 +570,7 @@ int ulysses_prologue_repack_fwd(const ulysses_plan_t* plan, const void* src_seq,
     const int32_t cc = std::min(plan->plane_chunk, plan->C - c0);
     s = status_of(ulysses::launch_prologue_repack(src_seq, dst_heads, norm_q_weight, norm_k_weight, cos_table,
                                                   sin_table, rotary_dim, eps, plan->Np, plan->H, plan->P, plan->C,
-                                                  c0, cc, plan->token_stride, plan->plane_stride, st));
+                                                  c0, cc, plan->token_stride, plan->plane_stride, st, plan->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   return ULYSSES_OK;
@@ -547,6 +578,7 @@ int ulysses_prologue_repack_fwd(const ulysses_plan_t* plan, const void* src_seq,
 
 int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, float softmax_scale,
                      void* stream) {
+  NvtxRange range("ulysses_attn_fwd");
   if (!plan || !qkv_heads || !out_heads) return ULYSSES_ERR_ARG;
   if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
   if (!aligned16(qkv_heads) || !aligned16(out_heads)) return ULYSSES_ERR_ALIGN;
@@ -557,6 +589,7 @@ int ulysses_attn_fwd(const ulysses_plan_t* plan, const void* qkv_heads, void* ou
 }
 
 int ulysses_repack_fwd_fp8(const ulysses_plan_t* plan, const void* src_seq, void* dst_heads_fp8, void* stream) {
+  NvtxRange range("ulysses_repack_fwd_fp8");
   if (!plan || !src_seq || !dst_heads_fp8) return ULYSSES_ERR_ARG;
   if (!aligned16(src_seq) || !aligned16(dst_heads_fp8)) return ULYSSES_ERR_ALIGN;
   if (overlap(src_seq, seq_extent_bytes(plan, plan->C, plan->token_stride, plan->plane_stride), dst_heads_fp8,
@@ -569,6 +602,7 @@ int ulysses_repack_fwd_fp8(const ulysses_plan_t* plan, const void* src_seq, void
 
 int ulysses_attn_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_heads_fp8, void* out_heads, float softmax_scale,
                          void* stream) {
+  NvtxRange range("ulysses_attn_fwd_fp8");
   if (!plan || !qkv_heads_fp8 || !out_heads) return ULYSSES_ERR_ARG;
   if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
   if (!aligned16(qkv_heads_fp8) || !aligned16(out_heads)) return ULYSSES_ERR_ALIGN;
@@ -585,6 +619,7 @@ size_t ulysses_workspace_bytes_fp8(const ulysses_plan_t* plan) {
 
 int ulysses_layer_fwd_fp8(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
                           size_t workspace_bytes, void* stream) {
+  NvtxRange range("ulysses_layer_fwd_fp8");
   if (!plan || !qkv_seq || !out_seq) return ULYSSES_ERR_ARG;
   if (plan->C < 3) return ULYSSES_ERR_ARG;
   if (!aligned16(qkv_seq) || !aligned16(out_seq)) return ULYSSES_ERR_ALIGN;
@@ -610,6 +645,7 @@ size_t ulysses_lse_bytes(const ulysses_plan_t* plan) { return plan ? static_cast
 
 int ulysses_attn_fwd_lse(const ulysses_plan_t* plan, const void* qkv_heads, void* out_heads, void* lse,
                          float softmax_scale, void* stream) {
+  NvtxRange range("ulysses_attn_fwd_lse");
   if (!plan || !qkv_heads || !out_heads || !lse) return ULYSSES_ERR_ARG;
   if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
   if (!aligned16(qkv_heads) || !aligned16(out_heads) || !aligned16(lse)) return ULYSSES_ERR_ALIGN;
@@ -630,6 +666,7 @@ size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan) {
 int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads,
                      const void* dout_heads, const void* lse, void* dqkv_heads, void* workspace,
                      size_t workspace_bytes, float softmax_scale, void* stream) {
+  NvtxRange range("ulysses_attn_bwd");
   if (!plan || !qkv_heads || !out_heads || !dout_heads || !lse || !dqkv_heads) return ULYSSES_ERR_ARG;
   if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
   if (!workspace || workspace_bytes < ulysses_attn_bwd_workspace_bytes(plan)) return ULYSSES_ERR_WORKSPACE;
@@ -665,6 +702,7 @@ size_t ulysses_layer_bwd_workspace_bytes(const ulysses_plan_t* plan) {
 
 int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads, const void* lse,
                       const void* dout_seq, void* dqkv_seq, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange range("ulysses_layer_bwd");
   if (!plan || !qkv_heads || !out_heads || !lse || !dout_seq || !dqkv_seq) return ULYSSES_ERR_ARG;
   if (plan->C < 3) return ULYSSES_ERR_ARG;
   if (!workspace || workspace_bytes < ulysses_layer_bwd_workspace_bytes(plan)) return ULYSSES_ERR_WORKSPACE;
@@ -686,7 +724,8 @@ int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const v
   float* delta = reinterpret_cast<float*>(dT + align_up(heads_bytes(plan, 3), 256));
   // mode 0 on the output gradient (one dense plane [Np, H, D])
   const int64_t row = static_cast<int64_t>(plan->H) * plan->D;
-  s = status_of(ulysses::launch_repack(0, dout_seq, dOT, plan->Np, plan->H, plan->P, 1, 0, 1, row, row, st));
+  s = status_of(
+      ulysses::launch_repack(0, dout_seq, dOT, plan->Np, plan->H, plan->P, 1, 0, 1, row, row, st, plan->dev_err));
   if (s != ULYSSES_OK) return s;
   ulysses::AttnBwdLaunch a;
   a.qkv = qkv_heads;
@@ -703,7 +742,7 @@ int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const v
   for (int32_t c0 = 0; c0 < 3; c0 += plan->plane_chunk) {
     const int32_t cc = std::min(plan->plane_chunk, 3 - c0);
     s = status_of(ulysses::launch_repack(1, dT, dqkv_seq, plan->Np, plan->H, plan->P, 3, c0, cc, plan->token_stride,
-                                         plan->plane_stride, st));
+                                         plan->plane_stride, st, plan->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   return ULYSSES_OK;
@@ -711,6 +750,7 @@ int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const v
 
 int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out_seq, void* workspace,
                       size_t workspace_bytes, int32_t fused, void* stream) {
+  NvtxRange range("ulysses_layer_fwd");
   if (!plan || !qkv_seq || !out_seq) return ULYSSES_ERR_ARG;
   if (plan->C < 3 || (fused != 0 && fused != 1)) return ULYSSES_ERR_ARG;
   if (!aligned16(qkv_seq) || !aligned16(out_seq)) return ULYSSES_ERR_ALIGN;
@@ -721,6 +761,7 @@ int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out
   if (fused) {
     int s = device_ready(plan);
     if (s != ULYSSES_OK) return s;
+    NvtxRange step("fused attention");
     return attn_impl(plan, qkv_seq, 1, out_seq, scale, st);
   }
   if (!workspace) return ULYSSES_ERR_WORKSPACE;
@@ -733,8 +774,15 @@ int ulysses_layer_fwd(const ulysses_plan_t* plan, const void* qkv_seq, void* out
   if (s != ULYSSES_OK) return s;
   uint8_t* T = static_cast<uint8_t*>(workspace);
   uint8_t* OT = T + align_up(heads_bytes(plan, plan->C), 256);
-  if ((s = repack_fwd_impl(plan, qkv_seq, T, st)) != ULYSSES_OK) return s;
-  if ((s = attn_impl(plan, T, 0, OT, scale, st)) != ULYSSES_OK) return s;
+  {
+    NvtxRange step("repack_fwd");
+    if ((s = repack_fwd_impl(plan, qkv_seq, T, st)) != ULYSSES_OK) return s;
+  }
+  {
+    NvtxRange step("attention");
+    if ((s = attn_impl(plan, T, 0, OT, scale, st)) != ULYSSES_OK) return s;
+  }
+  NvtxRange step("repack_bwd");
   return repack_bwd_impl(plan, OT, out_seq, 1, st);
 }
 
@@ -817,6 +865,7 @@ extern "C" {
 int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
                            void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
                            int32_t fused, void* stream) {
+  NvtxRange range("ulysses_layer_fwd_host");
   if (fused != 0 && fused != 1) return ULYSSES_ERR_ARG;
   return layer_host_impl(plan, host_qkv_seq, host_out_seq, dev_qkv_seq, dev_out_seq, workspace, workspace_bytes,
                          fused, stream);
@@ -825,12 +874,14 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
 int ulysses_layer_fwd_fp8_host(const ulysses_plan_t* plan, const void* host_qkv_seq, void* host_out_seq,
                                void* dev_qkv_seq, void* dev_out_seq, void* workspace, size_t workspace_bytes,
                                void* stream) {
+  NvtxRange range("ulysses_layer_fwd_fp8_host");
   return layer_host_impl(plan, host_qkv_seq, host_out_seq, dev_qkv_seq, dev_out_seq, workspace, workspace_bytes, 2,
                          stream);
 }
 
 int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_shard,
                             void* const* dst_heads, int32_t planes, void* stream) {
+  NvtxRange range("ulysses_repack_fwd_push");
   if (!plan || !src_shard || !dst_heads || rank < 0 || rank >= plan->P || planes < 1 || planes > plan->C)
     return ULYSSES_ERR_ARG;
   if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
@@ -845,7 +896,7 @@ int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void
   for (int32_t c0 = 0; c0 < planes; c0 += plan->plane_chunk) {
     const int32_t cc = std::min(plan->plane_chunk, planes - c0);
     s = status_of(ulysses::launch_push(0, src_shard, t, plan->Nl, plan->Np, plan->H, plan->P, planes, c0, cc, rank,
-                                       st));
+                                       st, plan->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   return ULYSSES_OK;
@@ -853,6 +904,7 @@ int ulysses_repack_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void
 
 int ulysses_repack_bwd_push(const ulysses_plan_t* plan, int32_t rank, const void* src_heads, void* const* dst_seq,
                             int32_t planes, void* stream) {
+  NvtxRange range("ulysses_repack_bwd_push");
   if (!plan || !src_heads || !dst_seq || rank < 0 || rank >= plan->P || planes < 1 || planes > plan->C)
     return ULYSSES_ERR_ARG;
   if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
@@ -867,7 +919,7 @@ int ulysses_repack_bwd_push(const ulysses_plan_t* plan, int32_t rank, const void
   for (int32_t c0 = 0; c0 < planes; c0 += plan->plane_chunk) {
     const int32_t cc = std::min(plan->plane_chunk, planes - c0);
     s = status_of(ulysses::launch_push(1, src_heads, t, plan->Nl, plan->Np, plan->H, plan->P, planes, c0, cc, rank,
-                                       st));
+                                       st, plan->dev_err));
     if (s != ULYSSES_OK) return s;
   }
   return ULYSSES_OK;
@@ -875,6 +927,7 @@ int ulysses_repack_bwd_push(const ulysses_plan_t* plan, int32_t rank, const void
 
 int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* heads, void* const* dst_seq,
                           float softmax_scale, void* stream) {
+  NvtxRange range("ulysses_attn_fwd_push");
   if (!plan || !heads || !dst_seq || rank < 0 || rank >= plan->P) return ULYSSES_ERR_ARG;
   if (plan->C < 3 || !(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return ULYSSES_ERR_ARG;
   if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
@@ -913,6 +966,7 @@ int ulysses_attn_fwd_push(const ulysses_plan_t* plan, int32_t rank, const void* 
 
 int ulysses_a2a_pack(const ulysses_plan_t* plan, const void* src_shard, int32_t planes, int32_t plane, void* send,
                      void* stream) {
+  NvtxRange range("ulysses_a2a_pack");
   if (!plan || !src_shard || !send || planes < 1 || planes > kMaxPlanes || plane < 0 || plane >= planes)
     return ULYSSES_ERR_ARG;
   if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
@@ -926,11 +980,12 @@ int ulysses_a2a_pack(const ulysses_plan_t* plan, const void* src_shard, int32_t 
   // mode 0 over the shard's Nl rows, one plane: send [P, 1, Nl, Hl, D]
   const uint8_t* src = static_cast<const uint8_t*>(src_shard) + static_cast<int64_t>(plane) * row * 2;
   return status_of(ulysses::launch_repack(0, src, send, plan->Nl, plan->H, plan->P, 1, 0, 1, planes * row, row,
-                                          static_cast<cudaStream_t>(stream)));
+                                          static_cast<cudaStream_t>(stream), plan->dev_err));
 }
 
 int ulysses_a2a_unpack(const ulysses_plan_t* plan, const void* recv, void* out_shard, int32_t planes, int32_t plane,
                        void* stream) {
+  NvtxRange range("ulysses_a2a_unpack");
   if (!plan || !recv || !out_shard || planes < 1 || planes > kMaxPlanes || plane < 0 || plane >= planes)
     return ULYSSES_ERR_ARG;
   if (!push_layout_ok(plan)) return ULYSSES_ERR_UNSUPPORTED;
@@ -942,11 +997,12 @@ int ulysses_a2a_unpack(const ulysses_plan_t* plan, const void* recv, void* out_s
   // mode 1 over Nl rows, one plane: recv [P, 1, Nl, Hl, D] -> plane `plane` of [Nl, planes, H, D]
   uint8_t* dst = static_cast<uint8_t*>(out_shard) + static_cast<int64_t>(plane) * row * 2;
   return status_of(ulysses::launch_repack(1, recv, dst, plan->Nl, plan->H, plan->P, 1, 0, 1, planes * row, row,
-                                          static_cast<cudaStream_t>(stream)));
+                                          static_cast<cudaStream_t>(stream), plan->dev_err));
 }
 
 int ulysses_attn_fwd_lse_slab(const ulysses_plan_t* plan, const void* heads, void* out_heads, void* lse,
                               float softmax_scale, void* stream) {
+  NvtxRange range("ulysses_attn_fwd_lse_slab");
   if (!plan) return ULYSSES_ERR_ARG;
   const ulysses_plan_t v = slab_view(plan);
   return ulysses_attn_fwd_lse(&v, heads, out_heads, lse, softmax_scale, stream);
@@ -955,6 +1011,7 @@ int ulysses_attn_fwd_lse_slab(const ulysses_plan_t* plan, const void* heads, voi
 int ulysses_attn_bwd_slab(const ulysses_plan_t* plan, const void* heads, const void* out_heads,
                           const void* dout_heads, const void* lse, void* dqkv_heads, void* workspace,
                           size_t workspace_bytes, float softmax_scale, void* stream) {
+  NvtxRange range("ulysses_attn_bwd_slab");
   if (!plan) return ULYSSES_ERR_ARG;
   const ulysses_plan_t v = slab_view(plan);
   return ulysses_attn_bwd(&v, heads, out_heads, dout_heads, lse, dqkv_heads, workspace, workspace_bytes,

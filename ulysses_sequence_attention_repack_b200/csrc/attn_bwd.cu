@@ -627,14 +627,15 @@ using EncodeTiledFnB = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFnB encode_fn() {
-  static EncodeTiledFnB fn = nullptr;
-  if (!fn) {
+  static const EncodeTiledFnB fn = [] {   // initialised once, thread-safe
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFnB>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFnB>(ptr);
+    cudaGetLastError();
+    return static_cast<EncodeTiledFnB>(nullptr);
+  }();
   return fn;
 }
 
@@ -656,15 +657,13 @@ bool head_map(CUtensorMap* m, const void* base, int64_t P, int64_t C, int64_t Np
 template <bool kPassA>
 cudaError_t launch_pass(const CUtensorMap& tq, const CUtensorMap& td, const BwdParams& p, int sms,
                         cudaStream_t stream) {
-  static bool attr_set[2][64] = {{false}};
+  static PerDeviceOnce setup;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[kPassA][dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<kPassA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[kPassA][dev] = true;
-  }
+  cudaError_t e = setup.run(dev, [] {
+    return cudaFuncSetAttribute(attn_bwd_kernel<kPassA>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   const int grid = std::min(p.num_units, sms);
   attn_bwd_kernel<kPassA><<<grid, kThreads, kSmemBytes, stream>>>(tq, td, p);
   return cudaGetLastError();

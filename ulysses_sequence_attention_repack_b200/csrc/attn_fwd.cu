@@ -45,6 +45,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include "bounds.cuh"
 #include "exp2_poly.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
@@ -142,6 +143,8 @@ struct AttnParams {
   int32_t paired;                  // 1: the causal pair schedule (enough units for two per CTA)
   float scale_log2;
   int64_t push_rows;               // > 0: row n is stored to push.p[n / push_rows] (multi-GPU push)
+  int32_t push_ranks;              // table entries in use
+  int64_t out_ext, lse_ext;        // elements, for the bounds-checked build only (bounds.cuh)
   SegDesc seg[ULYSSES_MAX_SEQS];   // longest first
   PushTable push;
 };
@@ -606,17 +609,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(BAR(B_OEMPTY0 + wg));
       const int n = w.q0 + wg * BM + row;
-      if (p.lse && n < sd.q_end && n < p.Np)
-        p.lse[(static_cast<int64_t>(w.r) * p.Hl + w.j) * p.lse_stride + n] = m_used + log2f(l);
+      if (p.lse && n < sd.q_end && n < p.Np) {
+        const int64_t li = (static_cast<int64_t>(w.r) * p.Hl + w.j) * p.lse_stride + n;
+        if (in_bounds(li, 1, p.lse_ext, p.err)) p.lse[li] = m_used + log2f(l);
+      }
       if (n < sd.q_end && n < p.Np) {
-        __nv_bfloat16* obase = p.out + w.r * p.o_stride_r;
-        int64_t orow = n;
+        __nv_bfloat16* obase = p.out;
+        int64_t ooff = w.r * p.o_stride_r + n * p.o_stride_n + w.j * p.o_stride_j;
+        bool ok = true;
         if (p.push_rows > 0) {   // the owning rank's shard, through its peer pointer
           const int64_t q = n / p.push_rows;
-          obase = static_cast<__nv_bfloat16*>(p.push.p[q]);
-          orow = n - q * p.push_rows;
+          ok = in_bounds(q, 1, p.push_ranks, p.err);
+          obase = static_cast<__nv_bfloat16*>(p.push.p[ok ? q : 0]);
+          ooff = (n - q * p.push_rows) * p.o_stride_n + w.j * p.o_stride_j;
         }
-        uint4* dst = reinterpret_cast<uint4*>(obase + orow * p.o_stride_n + w.j * p.o_stride_j);
+        ok = ok && in_bounds(ooff, HD, p.out_ext, p.err);
+        uint4* dst = reinterpret_cast<uint4*>(obase + ooff);
         const bool pad = n >= p.N;   // pad rows are written as zeros
         const float inv = 1.0f / l;
         const float* o = reinterpret_cast<const float*>(&oraw[0][0]);
@@ -628,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           q.z = pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
           q.w = pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
           if (pad) q = make_uint4(0u, 0u, 0u, 0u);
-          dst[v] = q;
+          if (ok) dst[v] = q;
         }
       }
       ++uc;
@@ -648,30 +656,30 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static const EncodeTiledFn fn = [] {   // initialised once, thread-safe
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    cudaGetLastError();
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
   return fn;
 }
 
 template <bool kFp8>
 cudaError_t launch_kernel(const CUtensorMap& tmap, const AttnParams& p, int grid, int dev, cudaStream_t stream) {
-  static bool attr_set[64] = {false};
-  if (dev < 64 && !attr_set[dev]) {
+  static PerDeviceOnce setup;
+  cudaError_t e = setup.run(dev, [] {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_fwd_kernel<kFp8>);
-    if (e != cudaSuccess) return e;
+    cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_kernel<kFp8>);
+    if (r != cudaSuccess) return r;
     if (fa.numRegs != static_cast<int>(kLaunchRegs)) return cudaErrorInvalidConfiguration;   // see register split
-    e = cudaFuncSetAttribute(attn_fwd_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<kFp8>::kBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+    return cudaFuncSetAttribute(attn_fwd_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Smem<kFp8>::kBytes);
+  });
+  if (e != cudaSuccess) return e;
   attn_fwd_kernel<kFp8><<<grid, kThreads, Smem<kFp8>::kBytes, stream>>>(tmap, p);
   return cudaGetLastError();
 }
@@ -740,8 +748,14 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
     for (int q = 0; q < a.push_ranks; ++q)
       if (!a.push->p[q]) return cudaErrorInvalidValue;
     p.push_rows = a.push_rows;
+    p.push_ranks = a.push_ranks;
     p.push = *a.push;
   }
+  // extents of the output (per table entry when pushing) and of the lse rows
+  p.out_ext = (a.push_rows > 0 ? (a.push_rows - 1) * a.o_stride_n
+                               : (a.P - 1) * a.o_stride_r + (a.Np - 1) * a.o_stride_n) +
+              (a.Hl - 1) * a.o_stride_j + HD;
+  p.lse_ext = static_cast<int64_t>(a.P) * a.Hl * a.lse_stride;
 
   // Non-empty segments, longest first.  The segment that ends at N also
   // covers the pad query rows [N, Np), which are written as zeros.

@@ -1,9 +1,11 @@
 // Host-side declarations shared by the C ABI (api.cpp) and the kernel files.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <mutex>
 
 #include "../../include/ulysses.h"
 
@@ -14,6 +16,28 @@ struct Segment {
 };
 
 struct HostPipe;   // copy streams and events of the host-buffer layer (api.cpp)
+
+// One-time setup per device (kernel attributes), safe to call from several
+// host threads at once.  run(dev, f) calls f() until it has succeeded once
+// for dev; devices past kMaxDevices run f() on every call.
+class PerDeviceOnce {
+ public:
+  template <class F>
+  cudaError_t run(int dev, F&& f) {
+    const bool tracked = dev >= 0 && dev < kMaxDevices;
+    if (tracked && done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (tracked && done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    const cudaError_t e = f();
+    if (e == cudaSuccess && tracked) done_[dev].store(true, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  static constexpr int kMaxDevices = 256;
+  std::mutex mu_;
+  std::atomic<bool> done_[kMaxDevices] = {};
+};
 
 }  // namespace ulysses
 
@@ -36,21 +60,23 @@ namespace ulysses {
 //   dir = 0: seq -> heads (mode 0), dir = 1: heads -> seq (mode 1).
 //   seq side: element (n, c, h, d) at n*tok_stride + c*plane_stride + h*D + d
 //   head side: [P, Ctot, Np, Hl, D]
+// err: device error word for the bounds-checked build (bounds.cuh); may be null.
 cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
-                          int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream);
+                          int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream,
+                          unsigned int* err = nullptr);
 
 // Mode 0 with the E4M3 cast (FP8 attention variant) over planes [c0, c0 + cc):
 // head side [P, Ctot, Np, Hl, D] of one-byte codes.
 cudaError_t launch_repack_fp8(const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
                               int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
-                              cudaStream_t stream);
+                              cudaStream_t stream, unsigned int* err = nullptr);
 
 // Prologue (per-head RMSNorm + partial RoPE on planes 0 and 1) fused with one
 // mode-0 repack launch over planes [c0, c0 + cc).
 cudaError_t launch_prologue_repack(const void* src, void* dst, const void* wq, const void* wk, const void* cos,
                                    const void* sin, int32_t rd, float eps, int64_t Np, int32_t H, int32_t P,
                                    int32_t Ctot, int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, unsigned int* err = nullptr);
 
 // Destination table of the multi-GPU push (a kernel parameter): entry r is
 // rank r's buffer (a peer mapping, or a local buffer when ranks are emulated).
@@ -62,7 +88,8 @@ struct PushTable {
 //   dir = 0: shard [Nl, C, H, D] -> dst.p[r] = T_r [C, Np, Hl, D], rows rank*Nl + i
 //   dir = 1: head rows [C, Np, Hl, D] -> dst.p[q] = [Nl, C, H, D], heads rank*Hl + j
 cudaError_t launch_push(int dir, const void* src, const PushTable& dst, int64_t Nl, int64_t Np, int32_t H,
-                        int32_t P, int32_t C, int32_t c0, int32_t cc, int32_t rank, cudaStream_t stream);
+                        int32_t P, int32_t C, int32_t c0, int32_t cc, int32_t rank, cudaStream_t stream,
+                        unsigned int* err = nullptr);
 
 // Attention launch description (filled by api.cpp).
 struct AttnLaunch {

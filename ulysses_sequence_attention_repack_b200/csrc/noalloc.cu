@@ -11,6 +11,7 @@
 // The only scratch the attention kernel uses is its 4-byte device error word
 // (set when a bounded wait gives up).  Here it lives in g_noalloc_scratch,
 // which every GPU that loads the library holds until the process exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -24,34 +25,82 @@ namespace {
 
 constexpr size_t kScratchBytes = 256;         // stated maximum: 64 words
 constexpr size_t kScratchNeededBytes = 4;     // one error word per call, any problem size
-constexpr int kMaxDevices = 64;
+constexpr int kCacheSlots = 64;
 
 // File-scope scratch.  Host code must not use this name as an address: in
 // host code it is only a stand-in for the symbol; the device address comes
 // from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned int g_noalloc_scratch[kScratchBytes / sizeof(unsigned int)];
 
+// The array's device address is valid only in the CUDA context it was looked
+// up in, so the lookups are cached per context: by the driver's context ID,
+// which is never reused within a process.  A cudaDeviceReset, or a different
+// driver-API context made current on the same device, gives a new ID and a
+// fresh lookup instead of a stale address.
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  unsigned int* addr;
+};
 std::mutex g_setup_mutex;
-unsigned int* g_scratch_addr[kMaxDevices] = {nullptr};
+ScratchSlot g_slots[kCacheSlots] = {};
+int g_next_slot = 0;
 
-// Device address of g_noalloc_scratch on the current device (looked up once
-// per device, with that device current).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_get_current = nullptr;
+CtxGetIdFn g_get_id = nullptr;
+bool g_api_looked_up = false;
+
+// 1: *id is the current context's ID; 0: no context is current yet;
+// -1: the driver offers no context IDs.  Called with g_setup_mutex held.
+int current_context_id(unsigned long long* id) {
+  if (!g_api_looked_up) {
+    g_api_looked_up = true;
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      g_get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      g_get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+    cudaGetLastError();
+  }
+  if (!g_get_current || !g_get_id) return -1;
+  CUcontext ctx = nullptr;
+  if (g_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  return g_get_id(ctx, id) == CUDA_SUCCESS ? 1 : -1;
+}
+
+// Device address of g_noalloc_scratch in the current context, looked up once
+// per context with its device current.  Without context IDs from the driver
+// the address is looked up on every call (a lookup, no allocation).
 int scratch_address(unsigned int** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  unsigned long long id = 0;
+  int have = current_context_id(&id);
+  if (have == 1) {
+    for (const ScratchSlot& sl : g_slots)
+      if (sl.addr && sl.ctx_id == id) {
+        *out = sl.addr;
+        return ULYSSES_OK;
+      }
+  }
+  // with no context current yet, this first runtime call makes the device's
+  // primary context current (and may load the library's device code)
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
     cudaGetLastError();
     return ULYSSES_ERR_CUDA;
   }
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
-      cudaGetLastError();
-      return ULYSSES_ERR_CUDA;
-    }
-    g_scratch_addr[dev] = static_cast<unsigned int*>(ptr);
+  if (have == 0) have = current_context_id(&id);
+  if (have == 1) {
+    g_slots[g_next_slot] = {id, static_cast<unsigned int*>(ptr)};
+    g_next_slot = (g_next_slot + 1) % kCacheSlots;
   }
-  *out = g_scratch_addr[dev];
+  *out = static_cast<unsigned int*>(ptr);
   return ULYSSES_OK;
 }
 

@@ -25,6 +25,7 @@
 
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
 
 namespace ulysses {
@@ -75,6 +76,10 @@ struct PrologueArgs {
   int32_t H, Hl, Ctot, c0, cc;
   int32_t rd;                         // rotary dims (multiple of 16, <= 128)
   float eps;
+  // extents in elements, for the bounds-checked build only (bounds.cuh):
+  // sequence side, head side, and the cos / sin tables [Np, rd]
+  int64_t src_ext, dst_ext, table_ext;
+  unsigned int* err;
 };
 
 __global__ void __launch_bounds__(kThreads) prologue_repack_kernel(const PrologueArgs a) {
@@ -111,12 +116,19 @@ __global__ void __launch_bounds__(kThreads) prologue_repack_kernel(const Prologu
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int k = k0 + u * 32 + lane;
-          if (k < vec_per_row) v[u] = ld_stream(a.src + ((seq_base + static_cast<int64_t>(k) * 8) >> 3));
+          if (k < vec_per_row) {
+            const int64_t s_el = seq_base + static_cast<int64_t>(k) * 8;
+            v[u] = make_int4(0, 0, 0, 0);
+            if (in_bounds(s_el, 8, a.src_ext, a.err)) v[u] = ld_stream(a.src + (s_el >> 3));
+          }
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int k = k0 + u * 32 + lane;
-          if (k < vec_per_row) st_stream(a.dst + ((head_base + head_off[k >> 4] + (k & 15) * 8) >> 3), v[u]);
+          if (k < vec_per_row) {
+            const int64_t d_el = head_base + head_off[k >> 4] + (k & 15) * 8;
+            if (in_bounds(d_el, 8, a.dst_ext, a.err)) st_stream(a.dst + (d_el >> 3), v[u]);
+          }
         }
       }
       continue;
@@ -128,8 +140,10 @@ __global__ void __launch_bounds__(kThreads) prologue_repack_kernel(const Prologu
       const uint16_t* wp = (c == 0 ? a.wq : a.wk) + ch * 8;
       unpack8(*reinterpret_cast<const int4*>(wp), w);
       if (ch < rd8) {
-        unpack8(*reinterpret_cast<const int4*>(a.cos + n * a.rd + ch * 8), cs);
-        unpack8(*reinterpret_cast<const int4*>(a.sin + n * a.rd + ch * 8), sn);
+        const int64_t t_el = n * a.rd + ch * 8;
+        const bool ok = in_bounds(t_el, 8, a.table_ext, a.err);
+        unpack8(ok ? *reinterpret_cast<const int4*>(a.cos + t_el) : make_int4(0, 0, 0, 0), cs);
+        unpack8(ok ? *reinterpret_cast<const int4*>(a.sin + t_el) : make_int4(0, 0, 0, 0), sn);
         if (rot_lo) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) sn[e] = -sn[e];   // y[i] cos - y[i + rd/2] sin
@@ -149,7 +163,8 @@ __global__ void __launch_bounds__(kThreads) prologue_repack_kernel(const Prologu
       for (int u = 0; u < kPairs; ++u) {
         const int h = hp0 + 2 * u + half;
         v[u] = make_int4(0, 0, 0, 0);
-        if (h < a.H) v[u] = ld_stream(a.src + ((seq_base + static_cast<int64_t>(h) * HD + ch * 8) >> 3));
+        const int64_t s_el = seq_base + static_cast<int64_t>(h) * HD + ch * 8;
+        if (h < a.H && in_bounds(s_el, 8, a.src_ext, a.err)) v[u] = ld_stream(a.src + (s_el >> 3));
       }
 #pragma unroll
       for (int u = 0; u < kPairs; ++u) {
@@ -174,7 +189,10 @@ __global__ void __launch_bounds__(kThreads) prologue_repack_kernel(const Prologu
         o.y = static_cast<int>(pack2(fmaf(pr[2], sn[2], y[2] * cs[2]), fmaf(pr[3], sn[3], y[3] * cs[3])));
         o.z = static_cast<int>(pack2(fmaf(pr[4], sn[4], y[4] * cs[4]), fmaf(pr[5], sn[5], y[5] * cs[5])));
         o.w = static_cast<int>(pack2(fmaf(pr[6], sn[6], y[6] * cs[6]), fmaf(pr[7], sn[7], y[7] * cs[7])));
-        if (h < a.H) st_stream(a.dst + ((head_base + head_off[h] + ch * 8) >> 3), o);
+        if (h < a.H) {
+          const int64_t d_el = head_base + head_off[h] + ch * 8;
+          if (in_bounds(d_el, 8, a.dst_ext, a.err)) st_stream(a.dst + (d_el >> 3), o);
+        }
       }
     }
   }
@@ -185,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) prologue_repack_kernel(const Prologu
 cudaError_t launch_prologue_repack(const void* src, void* dst, const void* wq, const void* wk, const void* cos,
                                    const void* sin, int32_t rd, float eps, int64_t Np, int32_t H, int32_t P,
                                    int32_t Ctot, int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, unsigned int* err) {
   if (H > kMaxHeads || P < 1 || H % P != 0) return cudaErrorInvalidValue;
   const int64_t rows = Np * cc;
   if (rows == 0) return cudaSuccess;
@@ -212,6 +230,10 @@ cudaError_t launch_prologue_repack(const void* src, void* dst, const void* wq, c
   a.cc = cc;
   a.rd = rd;
   a.eps = eps;
+  a.src_ext = (Np - 1) * tok_stride + static_cast<int64_t>(Ctot - 1) * plane_stride + static_cast<int64_t>(H) * HD;
+  a.dst_ext = static_cast<int64_t>(Ctot) * Np * H * HD;
+  a.table_ext = Np * rd;
+  a.err = err;
   prologue_repack_kernel<<<grid, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }

@@ -20,6 +20,7 @@
 
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
 
 namespace ulysses {
@@ -45,12 +46,15 @@ __device__ __forceinline__ void st_stream(int4* p, int4 v) {
 }
 
 // Element offsets are int64 throughout: the largest head-sharded buffer holds
-// 7.2e9 elements.
+// 7.2e9 elements.  src_ext / dst_ext are the buffers' extents in elements,
+// used by the bounds-checked build only (bounds.cuh).
 template <int DIR>
 __global__ void __launch_bounds__(kRepackThreads) repack_kernel(const int4* __restrict__ src,
                                                                 int4* __restrict__ dst, int64_t Np, int32_t H,
                                                                 int32_t Hl, int32_t Ctot, int32_t c0, int32_t cc,
-                                                                int64_t tok_stride, int64_t plane_stride) {
+                                                                int64_t tok_stride, int64_t plane_stride,
+                                                                int64_t src_ext, int64_t dst_ext,
+                                                                unsigned int* err) {
   // head_off[h]: element offset of head h's run inside a head-sharded row,
   // relative to T[0, c, n, 0, 0]: r*Ctot*Np*Hl*D + j*D with r = h / Hl, j = h % Hl.
   __shared__ int64_t head_off[kMaxHeads];
@@ -83,7 +87,9 @@ __global__ void __launch_bounds__(kRepackThreads) repack_kernel(const int4* __re
           const int h = k >> 4;
           const int64_t seq_off = seq_base + static_cast<int64_t>(k) * 8;
           const int64_t head_el = head_base + head_off[h] + (k & 15) * 8;
-          v[u] = ld_stream(src + ((DIR == 0 ? seq_off : head_el) >> 3));
+          const int64_t s_el = DIR == 0 ? seq_off : head_el;
+          v[u] = make_int4(0, 0, 0, 0);
+          if (in_bounds(s_el, 8, src_ext, err)) v[u] = ld_stream(src + (s_el >> 3));
         }
       }
 #pragma unroll
@@ -93,7 +99,8 @@ __global__ void __launch_bounds__(kRepackThreads) repack_kernel(const int4* __re
           const int h = k >> 4;
           const int64_t seq_off = seq_base + static_cast<int64_t>(k) * 8;
           const int64_t head_el = head_base + head_off[h] + (k & 15) * 8;
-          st_stream(dst + ((DIR == 0 ? head_el : seq_off) >> 3), v[u]);
+          const int64_t d_el = DIR == 0 ? head_el : seq_off;
+          if (in_bounds(d_el, 8, dst_ext, err)) st_stream(dst + (d_el >> 3), v[u]);
         }
       }
     }
@@ -122,7 +129,8 @@ __global__ void __launch_bounds__(kRepackThreads) repack_fp8_kernel(const int4* 
                                                                     uint2* __restrict__ dst, int64_t Np,
                                                                     int32_t H, int32_t Hl, int32_t Ctot,
                                                                     int32_t c0, int32_t cc, int64_t tok_stride,
-                                                                    int64_t plane_stride) {
+                                                                    int64_t plane_stride, int64_t src_ext,
+                                                                    int64_t dst_ext, unsigned int* err) {
   __shared__ int64_t head_off[kMaxHeads];
   constexpr int D = 128;
   const int64_t rank_stride = static_cast<int64_t>(Ctot) * Np * Hl * D;
@@ -148,7 +156,11 @@ __global__ void __launch_bounds__(kRepackThreads) repack_fp8_kernel(const int4* 
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int k = k0 + u * 32 + lane;
-        if (k < vec_per_row) v[u] = ld_stream(src + ((seq_base + static_cast<int64_t>(k) * 8) >> 3));
+        if (k < vec_per_row) {
+          const int64_t s_el = seq_base + static_cast<int64_t>(k) * 8;
+          v[u] = make_int4(0, 0, 0, 0);
+          if (in_bounds(s_el, 8, src_ext, err)) v[u] = ld_stream(src + (s_el >> 3));
+        }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
@@ -158,18 +170,28 @@ __global__ void __launch_bounds__(kRepackThreads) repack_fp8_kernel(const int4* 
           uint2 o;
           o.x = e4m3x4(static_cast<uint32_t>(v[u].x), static_cast<uint32_t>(v[u].y));
           o.y = e4m3x4(static_cast<uint32_t>(v[u].z), static_cast<uint32_t>(v[u].w));
-          dst[head_el >> 3] = o;
+          if (in_bounds(head_el, 8, dst_ext, err)) dst[head_el >> 3] = o;
         }
       }
     }
   }
 }
 
+// Extents (elements) of the two sides of one repack launch: the
+// sequence-sharded buffer as its strides span it over Ctot planes, and the
+// head-sharded [P, Ctot, Np, Hl, D] buffer.
+inline int64_t seq_extent(int64_t Np, int32_t H, int32_t Ctot, int64_t tok_stride, int64_t plane_stride) {
+  return (Np - 1) * tok_stride + static_cast<int64_t>(Ctot - 1) * plane_stride + static_cast<int64_t>(H) * 128;
+}
+inline int64_t head_extent(int64_t Np, int32_t H, int32_t Ctot) {
+  return static_cast<int64_t>(Ctot) * Np * H * 128;
+}
+
 }  // namespace
 
 cudaError_t launch_repack_fp8(const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
                               int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, unsigned int* err) {
   if (H > kMaxHeads || P < 1 || H % P != 0) return cudaErrorInvalidValue;
   const int64_t rows = Np * cc;
   if (rows == 0) return cudaSuccess;
@@ -180,12 +202,15 @@ cudaError_t launch_repack_fp8(const void* src, void* dst, int64_t Np, int32_t H,
   const int64_t want = (rows + warps_per_cta - 1) / warps_per_cta;
   const int grid = static_cast<int>(want < static_cast<int64_t>(sms) * 8 ? want : static_cast<int64_t>(sms) * 8);
   repack_fp8_kernel<<<grid, kRepackThreads, 0, stream>>>(static_cast<const int4*>(src), static_cast<uint2*>(dst),
-                                                         Np, H, H / P, Ctot, c0, cc, tok_stride, plane_stride);
+                                                         Np, H, H / P, Ctot, c0, cc, tok_stride, plane_stride,
+                                                         seq_extent(Np, H, Ctot, tok_stride, plane_stride),
+                                                         head_extent(Np, H, Ctot), err);
   return cudaGetLastError();
 }
 
 cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32_t H, int32_t P, int32_t Ctot,
-                          int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream) {
+                          int32_t c0, int32_t cc, int64_t tok_stride, int64_t plane_stride, cudaStream_t stream,
+                          unsigned int* err) {
   if (H > kMaxHeads || P < 1 || H % P != 0) return cudaErrorInvalidValue;
   const int64_t rows = Np * cc;
   if (rows == 0) return cudaSuccess;
@@ -197,12 +222,16 @@ cudaError_t launch_repack(int dir, const void* src, void* dst, int64_t Np, int32
   const int64_t want = (rows + warps_per_cta - 1) / warps_per_cta;
   const int grid = static_cast<int>(want < static_cast<int64_t>(sms) * 8 ? want : static_cast<int64_t>(sms) * 8);
   const int Hl = H / P;
+  const int64_t seq_ext = seq_extent(Np, H, Ctot, tok_stride, plane_stride);
+  const int64_t head_ext = head_extent(Np, H, Ctot);
   if (dir == 0) {
     repack_kernel<0><<<grid, kRepackThreads, 0, stream>>>(static_cast<const int4*>(src), static_cast<int4*>(dst),
-                                                          Np, H, Hl, Ctot, c0, cc, tok_stride, plane_stride);
+                                                          Np, H, Hl, Ctot, c0, cc, tok_stride, plane_stride,
+                                                          seq_ext, head_ext, err);
   } else {
     repack_kernel<1><<<grid, kRepackThreads, 0, stream>>>(static_cast<const int4*>(src), static_cast<int4*>(dst),
-                                                          Np, H, Hl, Ctot, c0, cc, tok_stride, plane_stride);
+                                                          Np, H, Hl, Ctot, c0, cc, tok_stride, plane_stride,
+                                                          head_ext, seq_ext, err);
   }
   return cudaGetLastError();
 }

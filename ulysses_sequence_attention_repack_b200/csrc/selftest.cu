@@ -5,6 +5,7 @@
 #include <cstdint>
 
 #include "../../include/ulysses_selftest.h"
+#include "bounds.cuh"
 #include "exp2_poly.cuh"
 
 namespace {
@@ -58,5 +59,25 @@ extern "C" int ulysses_selftest_exp2_poly(const float* x, float* y, int64_t n, v
   const int64_t blocks = (pairs + threads - 1) / threads;
   if (blocks > 0x7fffffff) return 1;
   exp2_poly_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? 0 : 6;
+}
+
+namespace {
+
+// The range check of the bounds-checked build, forced on: three offsets
+// against an extent of 100 elements, of which only the first is inside.  No
+// memory is touched; the results land in *err next to kErrBounds.
+__global__ void bounds_check_kernel(unsigned int* err) {
+  if (threadIdx.x != 0) return;
+  if (ulysses::in_bounds<true>(0, 8, 100, err)) atomicOr(err, 0x10u);
+  if (!ulysses::in_bounds<true>(-8, 8, 100, err)) atomicOr(err, 0x20u);
+  if (!ulysses::in_bounds<true>(96, 8, 100, err)) atomicOr(err, 0x40u);
+}
+
+}  // namespace
+
+extern "C" int ulysses_selftest_bounds_check(unsigned int* dev_err, void* stream) {
+  if (!dev_err) return 1;
+  bounds_check_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev_err);
   return cudaGetLastError() == cudaSuccess ? 0 : 6;
 }

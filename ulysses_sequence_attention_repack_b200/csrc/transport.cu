@@ -18,6 +18,7 @@
 
 #include <cstdint>
 
+#include "bounds.cuh"
 #include "internal.h"
 
 namespace ulysses {
@@ -41,10 +42,13 @@ __device__ __forceinline__ void st_vec(int4* p, int4 v) {
 }
 
 // mode 0: rows = Nl * cc runs of H*D elements; head h of (i, c) goes to
-// rank h / Hl at element ((c*Np + q*Nl + i)*Hl + h % Hl)*D.
+// rank h / Hl at element ((c*Np + q*Nl + i)*Hl + h % Hl)*D.  src_vecs /
+// dst_vecs: extents in 16-byte vectors of the shard and of each rank's
+// destination, for the bounds-checked build only (bounds.cuh).
 __global__ void __launch_bounds__(kThreads) push_fwd_kernel(const int4* __restrict__ src, PushTable dst,
                                                             int64_t Nl, int64_t Np, int32_t H, int32_t Hl,
-                                                            int32_t C, int32_t c0, int32_t cc, int32_t rank) {
+                                                            int32_t C, int32_t c0, int32_t cc, int32_t rank,
+                                                            int64_t src_vecs, int64_t dst_vecs, unsigned int* err) {
   __shared__ int4* head_base[kMaxHeads];   // rank r's buffer + j*D (16-byte units)
   constexpr int D = 128;
   for (int h = threadIdx.x; h < H; h += blockDim.x) {
@@ -67,12 +71,19 @@ __global__ void __launch_bounds__(kThreads) push_fwd_kernel(const int4* __restri
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int k = k0 + u * 32 + lane;
-        if (k < vec_per_row) v[u] = ld_stream(src + src_vec + k);
+        if (k < vec_per_row) {
+          v[u] = make_int4(0, 0, 0, 0);
+          if (in_bounds(src_vec + k, 1, src_vecs, err)) v[u] = ld_stream(src + src_vec + k);
+        }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int k = k0 + u * 32 + lane;
-        if (k < vec_per_row) st_vec(head_base[k >> 4] + dst_vec + (k & 15), v[u]);
+        if (k < vec_per_row) {
+          const int h = k >> 4;
+          const int64_t rel = static_cast<int64_t>(h - (h / Hl) * Hl) * (D / 8) + dst_vec + (k & 15);
+          if (in_bounds(rel, 1, dst_vecs, err)) st_vec(head_base[h] + dst_vec + (k & 15), v[u]);
+        }
       }
     }
   }
@@ -82,7 +93,9 @@ __global__ void __launch_bounds__(kThreads) push_fwd_kernel(const int4* __restri
 // of plane c goes to rank q = n / Nl at element (((n - q*Nl)*Cp + c)*H + r*Hl)*D.
 __global__ void __launch_bounds__(kThreads) push_bwd_kernel(const int4* __restrict__ src, PushTable dst,
                                                             int64_t Nl, int64_t Np, int32_t H, int32_t Hl,
-                                                            int32_t Cp, int32_t c0, int32_t cc, int32_t rank) {
+                                                            int32_t Cp, int32_t c0, int32_t cc, int32_t rank,
+                                                            int32_t nranks, int64_t src_vecs, int64_t dst_vecs,
+                                                            unsigned int* err) {
   constexpr int D = 128;
   const int lane = threadIdx.x & 31;
   const int64_t rows = Np * cc;
@@ -95,18 +108,23 @@ __global__ void __launch_bounds__(kThreads) push_bwd_kernel(const int4* __restri
     const int q = static_cast<int>(n / Nl);
     const int64_t i = n - q * Nl;
     const int64_t src_vec = (static_cast<int64_t>(c) * Np + n) * vec_per_row;
-    int4* out = static_cast<int4*>(dst.p[q]) + ((i * Cp + c) * H + static_cast<int64_t>(rank) * Hl) * (D / 8);
+    const int64_t out_vec = ((i * Cp + c) * H + static_cast<int64_t>(rank) * Hl) * (D / 8);
+    if (!in_bounds(q, 1, nranks, err)) continue;   // a table entry past the ranks in use
+    int4* out = static_cast<int4*>(dst.p[q]) + out_vec;
     for (int k0 = 0; k0 < vec_per_row; k0 += 32 * kUnroll) {
       int4 v[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int k = k0 + u * 32 + lane;
-        if (k < vec_per_row) v[u] = ld_stream(src + src_vec + k);
+        if (k < vec_per_row) {
+          v[u] = make_int4(0, 0, 0, 0);
+          if (in_bounds(src_vec + k, 1, src_vecs, err)) v[u] = ld_stream(src + src_vec + k);
+        }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int k = k0 + u * 32 + lane;
-        if (k < vec_per_row) st_vec(out + k, v[u]);
+        if (k < vec_per_row && in_bounds(out_vec + k, 1, dst_vecs, err)) st_vec(out + k, v[u]);
       }
     }
   }
@@ -124,18 +142,22 @@ int grid_for(int64_t rows) {
 }  // namespace
 
 cudaError_t launch_push(int dir, const void* src, const PushTable& dst, int64_t Nl, int64_t Np, int32_t H,
-                        int32_t P, int32_t C, int32_t c0, int32_t cc, int32_t rank, cudaStream_t stream) {
+                        int32_t P, int32_t C, int32_t c0, int32_t cc, int32_t rank, cudaStream_t stream,
+                        unsigned int* err) {
   if (H > kMaxHeads || P < 1 || P > ULYSSES_MAX_PUSH_RANKS || H % P != 0 || rank < 0 || rank >= P)
     return cudaErrorInvalidValue;
   const int64_t rows = (dir == 0 ? Nl : Np) * cc;
   if (rows == 0) return cudaSuccess;
   const int grid = grid_for(rows);
+  const int64_t Hl = H / P;
+  // extents in 16-byte vectors: shard [Nl, C, H, D] and head slab [C, Np, Hl, D]
+  const int64_t shard_vecs = Nl * C * H * 16, slab_vecs = static_cast<int64_t>(C) * Np * Hl * 16;
   if (dir == 0)
     push_fwd_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const int4*>(src), dst, Nl, Np, H, H / P, C, c0,
-                                                   cc, rank);
+                                                   cc, rank, shard_vecs, slab_vecs, err);
   else
     push_bwd_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const int4*>(src), dst, Nl, Np, H, H / P, C, c0,
-                                                   cc, rank);
+                                                   cc, rank, P, slab_vecs, shard_vecs, err);
   return cudaGetLastError();
 }
 

@@ -12,7 +12,7 @@ import os
 
 import numpy as np
 import pytest
-from _parity import MEAN_ABS, REL_L2_FP8, check_attention
+from _parity import MAX_ABS, MEAN_ABS, REL_L2_FP8, check_attention
 
 from oracle import ulysses_oracle as orc
 
@@ -176,7 +176,13 @@ def test_full_layer_sharp_softmax_dit19k(gpu):
     ref = orc.attention_heads(inputs.host_bits(T[:, :3]), N, scale, rows=rows, workers=_cores())
     idx = torch.from_numpy(rows).to(gpu)
     got = OT.index_select(1, idx).float().cpu().numpy().astype(np.float64)
-    check_attention(f"full size dit19k sharp softmax (Q x 8), {rows.size} rows x {H} heads", got, ref)
+    # |O| reaches ~4 here (the weight sits on a few N(0,1) value rows), where
+    # the bf16 rounding of O alone is up to 2^-8 |O| ~ 0.016 and that of P adds
+    # as much again: the absolute max-abs gate of the N(0,1) workloads (|O| ~
+    # 0.01) does not apply, and the tiny diagnostic's 4 x allowance is used;
+    # rel-L2 and mean-abs keep their gates
+    check_attention(f"full size dit19k sharp softmax (Q x 8), {rows.size} rows x {H} heads", got, ref,
+                    max_abs=4 * MAX_ABS)
     lay = OS.index_select(0, idx).float().cpu().numpy().astype(np.float64)
     assert np.array_equal(lay, orc.output_repack_bwd(got))
 

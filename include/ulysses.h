@@ -77,6 +77,13 @@ enum {
  * segment), as in the causal flash wrapper of the prime-rl Ulysses context
  * parallelism pull request. */
 #define ULYSSES_PLAN_CAUSAL 1u
+/* ulysses_plan_ex flag: run the bf16 attention forward on CTA pairs
+ * (clusters of two SMs; one cta_group::2 MMA of 256 query rows per tile, each
+ * SM loading half of every K and V tile) instead of the default one CTA per
+ * SM.  Both give the same bits; on B200 the pair kernel measured 19-22%
+ * slower (the cross-SM hand-offs lengthen the S -> softmax -> P V chain that
+ * bounds the loop), so it is opt-in. */
+#define ULYSSES_PLAN_PAIR_ATTENTION 2u
 /* Most ranks the multi-GPU push calls address (one NVLink domain). */
 #define ULYSSES_MAX_PUSH_RANKS 64
 
@@ -111,7 +118,8 @@ int ulysses_plan(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t 
                  int64_t token_stride, int64_t plane_stride, int64_t plane_chunk,
                  const int32_t* cu_seqlens_host, int32_t num_seqs);
 
-/* ulysses_plan with option flags (ULYSSES_PLAN_CAUSAL); ulysses_plan is
+/* ulysses_plan with option flags (ULYSSES_PLAN_CAUSAL,
+ * ULYSSES_PLAN_PAIR_ATTENTION); ulysses_plan is
  * ulysses_plan_ex with flags = 0.  Unknown flag bits -> ULYSSES_ERR_ARG. */
 int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
                     int64_t token_stride, int64_t plane_stride, int64_t plane_chunk,

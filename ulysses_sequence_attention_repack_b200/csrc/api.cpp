@@ -406,7 +406,7 @@ int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32
                     int32_t num_seqs, uint32_t flags) {
   if (!out) return ULYSSES_ERR_ARG;
   *out = nullptr;
-  if (flags & ~ULYSSES_PLAN_CAUSAL) return ULYSSES_ERR_ARG;
+  if (flags & ~(ULYSSES_PLAN_CAUSAL | ULYSSES_PLAN_PAIR_ATTENTION)) return ULYSSES_ERR_ARG;
   if (D != kHeadDim) return ULYSSES_ERR_UNSUPPORTED;
   if (N < 1 || H < 1 || P < 1 || planes < 1 || planes > kMaxPlanes) return ULYSSES_ERR_ARG;
   if (H > kMaxHeads) return ULYSSES_ERR_UNSUPPORTED;
@@ -470,6 +470,7 @@ int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32
   p->plane_chunk = static_cast<int32_t>(chunk);
   p->num_seqs = nseq;
   p->causal = (flags & ULYSSES_PLAN_CAUSAL) ? 1 : 0;
+  p->pair_cta = (flags & ULYSSES_PLAN_PAIR_ATTENTION) ? 1 : 0;
   std::memcpy(p->segs, segs, sizeof(ulysses::Segment) * nseq);
   p->device = -1;
   p->dev_err = nullptr;

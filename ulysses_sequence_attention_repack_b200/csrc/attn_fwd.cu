@@ -64,6 +64,7 @@ namespace {
 constexpr int kThreads = 384;      // 3 warpgroups
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
+constexpr int kFwdWarp = 10;        // CTA pairs: forwards the odd CTA's completed fills
 // Register split: the kernel is launched with kLaunchRegs per thread
 // (384 x 168 = 64512); warpgroup 2 (TMA, MMA, two spare warps) drops to
 // kProducerRegs and the two softmax warpgroups rise to kSoftmaxRegs:
@@ -78,21 +79,26 @@ constexpr int BM = 128;            // query rows per tile
 constexpr int BN = 128;            // keys per tile
 constexpr int HD = 128;            // head dim
 constexpr int kUnitRows = 2 * BM;  // query rows per work unit (two tiles)
+constexpr int kPairUnitRows = 4 * BM;   // CTA pairs: two tiles of 256 rows (128 in each CTA)
 constexpr uint32_t kBoxBytes = BM * 128;  // one TMA box: 128 rows x 128 bytes, 128B-swizzled (16 KB)
 constexpr int kStages = 2;
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s per wait
 
 // Tile geometry per element type.  A 128 x 128 tile is two boxes of 64 bf16
-// columns (32 KB) or one box of 128 E4M3 columns (16 KB).
-template <bool kFp8>
+// columns (32 KB) or one box of 128 E4M3 columns (16 KB).  In a CTA pair each
+// CTA holds half of every K tile (64 keys, two boxes of 64 rows) and half of
+// every V tile (64 head-dim columns, one box of 128 rows): 16 KB each.
+template <bool kFp8, bool kPair = false>
 struct Geo {
   static constexpr int kBoxes = kFp8 ? 1 : 2;
-  static constexpr uint32_t kTileBytes = kBoxes * kBoxBytes;
+  static constexpr uint32_t kTileBytes = kBoxes * kBoxBytes;              // one CTA's Q tile
+  static constexpr uint32_t kKBytes = kPair ? kTileBytes / 2 : kTileBytes;   // one K stage
+  static constexpr uint32_t kVBytes = kPair ? kTileBytes / 2 : kTileBytes;   // one V stage
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr uint32_t kOffQ = 0;                                  // [2 tiles]
   static constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;             // [stages]
-  static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;       // [stages]
-  static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr uint32_t kOffV = kOffK + kStages * kKBytes;          // [stages]
+  static constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
 };
 // barrier indices
 enum {
@@ -104,9 +110,9 @@ enum {
   B_PHALF0, B_PHALF1,
   B_DONE, B_COUNT
 };
-template <bool kFp8>
+template <bool kFp8, bool kPair = false>
 struct Smem {
-  static constexpr uint32_t kOffBar = Geo<kFp8>::kOffBar;
+  static constexpr uint32_t kOffBar = Geo<kFp8, kPair>::kOffBar;
   static constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;     // TMEM base address
   static constexpr uint32_t kOffAbort = kOffSlot + 4;
   static constexpr uint32_t kBytes = kOffAbort + 4 + 1024;        // + alignment slack
@@ -119,12 +125,14 @@ constexpr uint32_t kIdescS = idesc_bf16_f32(BM, BN, 0, 0);    // Q, K both K-maj
 constexpr uint32_t kIdescPV = idesc_bf16_f32(BM, HD, 0, 1);   // P from TMEM, V MN-major (head dim contiguous)
 constexpr uint32_t kIdescS8 = idesc_e4m3_f32(BM, BN, 0, 0);   // the same for E4M3 operands
 constexpr uint32_t kIdescPV8 = idesc_e4m3_f32(BM, HD, 0, 1);
+constexpr uint32_t kIdescS2 = idesc_bf16_f32(2 * BM, BN, 0, 0);   // CTA pairs: M = 256
+constexpr uint32_t kIdescPV2 = idesc_bf16_f32(2 * BM, HD, 0, 1);
 
 struct SegDesc {
   int32_t start;       // first query row and first key
   int32_t kv_end;      // one past the last key
   int32_t q_end;       // one past the last query row this segment writes (Np for the last segment)
-  int32_t nqb;         // 256-row query blocks
+  int32_t nqb;         // query blocks of one work unit's rows (256, or 512 for CTA pairs)
   int32_t unit_base;   // first work unit of this segment
   int32_t pair_base;   // causal schedule: first pair of query blocks of this segment
 };
@@ -153,6 +161,7 @@ struct Unit {
   int seg, r, j, q0;
 };
 
+template <int kRows>
 __device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& w) {
   int s = 0;
   while (s + 1 < p.nseg && u >= p.seg[s + 1].unit_base) ++s;
@@ -163,7 +172,7 @@ __device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& w)
   w.seg = s;
   w.r = rh / p.Hl;
   w.j = rh - w.r * p.Hl;
-  w.q0 = p.seg[s].start + qb * kUnitRows;
+  w.q0 = p.seg[s].start + qb * kRows;
   return local >= 0 && w.r < p.P;
 }
 
@@ -180,13 +189,16 @@ __device__ __forceinline__ bool decode_unit(const AttnParams& p, int u, Unit& w)
 //   round robin would leave the busiest CTA with ~1.2x the average work at
 //   the Video-DiT size.  With fewer than two units per SM the pairs would
 //   idle half the SMs, so small causal problems keep the plain schedule.
-__device__ __forceinline__ int unit_of_cta(const AttnParams& p, int k, Unit& w) {
+//   cta / ncta: this CTA's index and the grid size, or the pair's index and
+//   the number of pairs.
+template <int kRows>
+__device__ __forceinline__ int unit_of_cta(const AttnParams& p, int k, Unit& w, int cta, int ncta) {
   if (!p.paired) {
-    const int u = blockIdx.x + k * gridDim.x;
+    const int u = cta + k * ncta;
     if (u >= p.num_units) return 0;
-    return decode_unit(p, u, w) ? 1 : -1;
+    return decode_unit<kRows>(p, u, w) ? 1 : -1;
   }
-  const int pp = blockIdx.x + (k >> 1) * gridDim.x;
+  const int pp = cta + (k >> 1) * ncta;
   if (pp >= p.num_pairs) return 0;
   int s = 0;
   while (s + 1 < p.nseg && pp >= p.seg[s + 1].pair_base) ++s;
@@ -197,7 +209,7 @@ __device__ __forceinline__ int unit_of_cta(const AttnParams& p, int k, Unit& w) 
   const int i = local - rh * half;
   const int qb = (k & 1) ? i : nqb - 1 - i;
   if ((k & 1) && qb >= nqb - 1 - i) return 2;   // the unpaired middle block
-  return decode_unit(p, p.seg[s].unit_base + rh * nqb + qb, w) ? 1 : -1;
+  return decode_unit<kRows>(p, p.seg[s].unit_base + rh * nqb + qb, w) ? 1 : -1;
 }
 
 // P = exp2(s * scale_log2 - m) for columns [64 half, 64 half + 64) of one row,
@@ -262,8 +274,9 @@ __device__ __forceinline__ void exp_store_half_fp8(const float* s, int half, f2 
 
 // Number of 128-key tiles a unit visits: the whole segment, or (causal) the
 // keys up to the unit's last query row.
+template <int kRows>
 __device__ __forceinline__ int unit_kv_tiles(const AttnParams& p, const SegDesc& sd, const Unit& w) {
-  const int hi = p.causal ? min(sd.kv_end, w.q0 + kUnitRows) : sd.kv_end;
+  const int hi = p.causal ? min(sd.kv_end, w.q0 + kRows) : sd.kv_end;
   return (hi - sd.start + BN - 1) / BN;
 }
 
@@ -278,13 +291,29 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
 
 // kFp8: Q, K, V are E4M3 codes (one byte per element) and P is stored as
 // E4M3 for the P V product; otherwise everything is bf16.
-template <bool kFp8>
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ AttnParams p) {
-  using G = Geo<kFp8>;
+//
+// kPair: the kernel runs as clusters of two CTAs on neighbouring SMs.  A work
+// unit is 512 query rows of one (rank, head, sequence); tile i (i = 0, 1) of
+// the pair is rows q0 + 256 i .. q0 + 256 i + 255, the even CTA holding the
+// first 128 of them in its shared memory and TMEM and the odd CTA the other
+// 128.  One thread of the even CTA issues every MMA as a cta_group::2
+// operation of M = 256: S_i = Q_i K^T reads each CTA's 64 keys of the K tile
+// (B split by N) and O_i += P_i V each CTA's 64 head-dim columns of V.  So
+// each SM copies into shared memory half of every K and V tile, and the
+// B-operand reads of both products are split between the two SMs.  Each
+// CTA's softmax warps work on their own TMEM rows exactly as in the
+// single-CTA kernel; their P and O hand-offs arrive (one arrival per warp)
+// on the even CTA's barriers, and the MMA thread's commits arrive on the
+// barriers of both CTAs.  Every CTA's copies complete on its own barriers,
+// and warp 10 of the odd CTA forwards each completed fill to the even CTA's
+// barrier, so each producer can wait for its own copies before its CTA exits.
+template <bool kFp8, bool kPair>
+__device__ __forceinline__ void attn_body(const CUtensorMap* tmap, const CUtensorMap* tmapK, const AttnParams& p) {
+  using G = Geo<kFp8, kPair>;
+  constexpr int kRows = kPair ? kPairUnitRows : kUnitRows;
   constexpr uint32_t kTileBytes = G::kTileBytes;
   constexpr uint32_t kOffQ = G::kOffQ, kOffK = G::kOffK, kOffV = G::kOffV, kOffBar = G::kOffBar;
-  constexpr uint32_t kOffSlot = Smem<kFp8>::kOffSlot, kOffAbort = Smem<kFp8>::kOffAbort;
+  constexpr uint32_t kOffSlot = Smem<kFp8, kPair>::kOffSlot, kOffAbort = Smem<kFp8, kPair>::kOffAbort;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -296,35 +325,76 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   WaitGuard g{abort_flag, p.err, kWaitLimitNs};
+  // the CTA (or pair) index and count the work units are dealt over
+  const uint32_t cr = kPair ? cluster_ctarank() : 0u;   // 0: the CTA whose thread issues the MMAs
+  const bool leader = cr == 0;
+  const int cta = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int ncta = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // shared::cluster addresses of barrier 0 in the even (L) and the odd (O) CTA of a pair
+  const uint32_t lbar0 = kPair ? mapa_shared(bar0, 0) : bar0;
+  const uint32_t obar0 = kPair ? mapa_shared(bar0, 1) : bar0;
+  auto LBAR = [&](int i) { return lbar0 + 8u * static_cast<uint32_t>(i); };
+  auto OBAR = [&](int i) { return obar0 + 8u * static_cast<uint32_t>(i); };
+  // tcgen05 completion of everything this thread issued, on barrier i of both CTAs
+  auto commit = [&](int i) {
+    if constexpr (kPair) {
+      mma_commit_pair(LBAR(i));
+      mma_commit_pair(OBAR(i));
+    } else {
+      mma_commit(BAR(i));
+    }
+  };
+  // a P or O hand-off of this softmax thread: per thread, or per warp of both
+  // CTAs onto the even CTA's barrier
+  auto hand_off = [&](int i) {
+    if constexpr (kPair) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(LBAR(i));
+    } else {
+      mbar_arrive(BAR(i));
+    }
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(BAR(B_QFULL0), 1);
-    mbar_init(BAR(B_QFULL1), 1);
+    // the even CTA's fill barriers also take the odd CTA's forwarded arrival
+    const uint32_t fills = (kPair && leader) ? 2 : 1;
+    const uint32_t hands = kPair ? 8 : BM;   // 4 warps x 2 CTAs, or 128 threads
+    mbar_init(BAR(B_QFULL0), fills);
+    mbar_init(BAR(B_QFULL1), fills);
     mbar_init(BAR(B_QEMPTY), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(BAR(B_KFULL0 + s), 1);
+      mbar_init(BAR(B_KFULL0 + s), fills);
       mbar_init(BAR(B_KEMPTY0 + s), 1);
-      mbar_init(BAR(B_VFULL0 + s), 1);
+      mbar_init(BAR(B_VFULL0 + s), fills);
       mbar_init(BAR(B_VEMPTY0 + s), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(B_SFULL0 + i), 1);
-      mbar_init(BAR(B_PFULL0 + i), BM);
+      mbar_init(BAR(B_PFULL0 + i), hands);
       mbar_init(BAR(B_OFULL0 + i), 1);
-      mbar_init(BAR(B_OEMPTY0 + i), BM);
-      mbar_init(BAR(B_PHALF0 + i), BM);
+      mbar_init(BAR(B_OEMPTY0 + i), hands);
+      mbar_init(BAR(B_PHALF0 + i), hands);
     }
     mbar_init(BAR(B_DONE), 1);
     fence_mbar_init();
   }
-  if (warp == kTmaWarp && lane == 0) prefetch_tmap(&tmap);
+  if (warp == kTmaWarp && lane == 0) {
+    prefetch_tmap(tmap);
+    if (kPair) prefetch_tmap(tmapK);
+  }
   if (warp == kMmaWarp) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();   // both CTAs' barriers initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
@@ -336,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         Unit w;
-        const int st = unit_of_cta(p, k, w);
+        const int st = unit_of_cta<kRows>(p, k, w, cta, ncta);
         if (st == 0) break;
         if (st == 2) continue;
         if (st < 0) {
@@ -346,32 +416,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const SegDesc& sd = p.seg[w.seg];
         const int hc = p.fused ? w.r * p.Hl + w.j : w.j;   // head coordinate
         const int rc = p.fused ? 0 : w.r;                  // rank coordinate
-        if (uc > 0 && !(ok = mbar_wait(BAR(B_QEMPTY), (uc - 1) & 1, g))) break;
+        if (uc > 0 && !(ok = mbar_wait<kPair>(BAR(B_QEMPTY), (uc - 1) & 1, g))) break;
         for (int i = 0; i < 2; ++i) {
+          const int q_row = w.q0 + (kPair ? i * 2 * BM + static_cast<int>(cr) * BM : i * BM);
           mbar_arrive_expect_tx(BAR(B_QFULL0 + i), kTileBytes);
           for (int h = 0; h < G::kBoxes; ++h)
-            tma_load_5d(sbase + kOffQ + i * kTileBytes + h * kBoxBytes, &tmap, BAR(B_QFULL0 + i), 64 * h, hc,
-                        w.q0 + i * BM, 0, rc);
+            tma_load_5d(sbase + kOffQ + i * kTileBytes + h * kBoxBytes, tmap, BAR(B_QFULL0 + i), 64 * h, hc, q_row,
+                        0, rc);
         }
-        const int nkv = unit_kv_tiles(p, sd, w);
+        const int nkv = unit_kv_tiles<kRows>(p, sd, w);
         for (int t = 0; t < nkv; ++t) {
           const int kv0 = sd.start + t * BN;
           {
             const uint32_t s = kc % kStages, ph = (kc / kStages) & 1;
             if (kc >= kStages && !(ok = mbar_wait(BAR(B_KEMPTY0 + s), ph ^ 1, g))) break;
-            mbar_arrive_expect_tx(BAR(B_KFULL0 + s), kTileBytes);
-            for (int h = 0; h < G::kBoxes; ++h)
-              tma_load_5d(sbase + kOffK + s * kTileBytes + h * kBoxBytes, &tmap, BAR(B_KFULL0 + s), 64 * h, hc,
-                          kv0, 1, rc);
+            mbar_arrive_expect_tx(BAR(B_KFULL0 + s), G::kKBytes);
+            if constexpr (kPair) {   // this CTA's 64 keys, both 64-column boxes (64 rows each)
+              for (int h = 0; h < 2; ++h)
+                tma_load_5d(sbase + kOffK + s * G::kKBytes + h * (G::kKBytes / 2), tmapK, BAR(B_KFULL0 + s),
+                            64 * h, hc, kv0 + 64 * static_cast<int>(cr), 1, rc);
+            } else {
+              for (int h = 0; h < G::kBoxes; ++h)
+                tma_load_5d(sbase + kOffK + s * G::kKBytes + h * kBoxBytes, tmap, BAR(B_KFULL0 + s), 64 * h, hc,
+                            kv0, 1, rc);
+            }
             ++kc;
           }
           {
             const uint32_t s = vc % kStages, ph = (vc / kStages) & 1;
             if (vc >= kStages && !(ok = mbar_wait(BAR(B_VEMPTY0 + s), ph ^ 1, g))) break;
-            mbar_arrive_expect_tx(BAR(B_VFULL0 + s), kTileBytes);
-            for (int h = 0; h < G::kBoxes; ++h)
-              tma_load_5d(sbase + kOffV + s * kTileBytes + h * kBoxBytes, &tmap, BAR(B_VFULL0 + s), 64 * h, hc,
+            mbar_arrive_expect_tx(BAR(B_VFULL0 + s), G::kVBytes);
+            if constexpr (kPair) {   // this CTA's 64 head-dim columns of all 128 keys: one box
+              tma_load_5d(sbase + kOffV + s * G::kVBytes, tmap, BAR(B_VFULL0 + s), 64 * static_cast<int>(cr), hc,
                           kv0, 2, rc);
+            } else {
+              for (int h = 0; h < G::kBoxes; ++h)
+                tma_load_5d(sbase + kOffV + s * G::kVBytes + h * kBoxBytes, tmap, BAR(B_VFULL0 + s), 64 * h, hc,
+                            kv0, 2, rc);
+            }
             ++vc;
           }
         }
@@ -387,22 +469,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t n = (vc > kStages ? vc - kStages : 0); n < vc; ++n)
         drain_wait(BAR(B_VFULL0 + n % kStages), (n / kStages) & 1);
     }
+   } else if (kPair && warp == kFwdWarp) {
+    // ------------------------------------------------------------ fill forwarder (odd CTA of a pair)
+    // Follows the producer's fills in order: once this CTA's half of a fill
+    // has landed, arrive on the even CTA's barrier of that fill.
+    if (!leader && lane == 0) {
+      uint32_t kc = 0, vc = 0, uc = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        Unit w;
+        const int st = unit_of_cta<kRows>(p, k, w, cta, ncta);
+        if (st == 0 || st < 0) break;
+        if (st == 2) continue;
+        const int nkv = unit_kv_tiles<kRows>(p, p.seg[w.seg], w);
+        for (int i = 0; ok && i < 2; ++i) {
+          if (!(ok = mbar_wait(BAR(B_QFULL0 + i), uc & 1, g))) break;
+          mbar_arrive_cluster(LBAR(B_QFULL0 + i));
+        }
+        for (int t = 0; ok && t < nkv; ++t) {
+          if (!(ok = mbar_wait(BAR(B_KFULL0 + kc % kStages), (kc / kStages) & 1, g))) break;
+          mbar_arrive_cluster(LBAR(B_KFULL0 + kc % kStages));
+          ++kc;
+          if (!(ok = mbar_wait(BAR(B_VFULL0 + vc % kStages), (vc / kStages) & 1, g))) break;
+          mbar_arrive_cluster(LBAR(B_VFULL0 + vc % kStages));
+          ++vc;
+        }
+        ++uc;
+      }
+    }
    } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ tcgen05 issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       uint32_t kc = 0, vc = 0, uc = 0, pc = 0;
       bool ok = true;
-      // descriptors computed once; each group of 8 MMAs is one asm block
+      // descriptors computed once; each group of 8 MMAs is one asm block.  In
+      // a pair the same shared-memory offsets hold the odd CTA's halves.
       const uint64_t dQ0 = desc_sw128(sbase + kOffQ, 16, 1024);
       const uint64_t dQ1 = desc_sw128(sbase + kOffQ + kTileBytes, 16, 1024);
       const uint64_t dK0 = desc_sw128(sbase + kOffK, 16, 1024);
-      const uint64_t dK1 = desc_sw128(sbase + kOffK + kTileBytes, 16, 1024);
+      const uint64_t dK1 = desc_sw128(sbase + kOffK + G::kKBytes, 16, 1024);
       // V is read MN-major: the leading byte offset steps to the second
-      // 64-column box of a bf16 tile (an E4M3 tile's 128 columns are one box)
+      // 64-column box of a bf16 tile (an E4M3 tile's 128 columns are one box;
+      // a pair's CTA holds one 64-column box)
       const uint64_t dV0 = desc_sw128(sbase + kOffV, kBoxBytes, 1024);
-      const uint64_t dV1 = desc_sw128(sbase + kOffV + kTileBytes, kBoxBytes, 1024);
+      const uint64_t dV1 = desc_sw128(sbase + kOffV + G::kVBytes, kBoxBytes, 1024);
       auto issue_s = [&](int i, uint32_t ks) {
-        if (kFp8)
+        if (kPair)
+          mma_ss_k128_pair(tmem + kColS0 + 128 * i, i ? dQ1 : dQ0, ks ? dK1 : dK0, kIdescS2, 0);
+        else if (kFp8)
           mma_ss_f8_k128(tmem + kColS0 + 128 * i, i ? dQ1 : dQ0, ks ? dK1 : dK0, kIdescS8, 0);
         else
           mma_ss_k128(tmem + kColS0 + 128 * i, i ? dQ1 : dQ0, ks ? dK1 : dK0, kIdescS, 0);
@@ -411,7 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (bf16 pairs) or [16 h, 16 h + 16) (E4M3 quads), V rows 64 h.. (8 KB
       // further in each 128-byte-wide box: +512 descriptor units)
       auto issue_pv_half = [&](int i, uint32_t vs, int h, uint32_t acc) {
-        if (kFp8)
+        if (kPair)
+          mma_ts_k64_pair(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 32 * h, (vs ? dV1 : dV0) + 512 * h,
+                          kIdescPV2, acc);
+        else if (kFp8)
           mma_ts_f8_k64(tmem + kColO0 + 128 * i, tmem + kColS0 + 128 * i + 16 * h, (vs ? dV1 : dV0) + 512 * h,
                         kIdescPV8, acc);
         else
@@ -420,46 +537,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int k = 0; ok; ++k) {
         Unit w;
-        const int st = unit_of_cta(p, k, w);
+        const int st = unit_of_cta<kRows>(p, k, w, cta, ncta);
         if (st == 0 || st < 0) break;
         if (st == 2) continue;
         const SegDesc& sd = p.seg[w.seg];
-        const int nkv = unit_kv_tiles(p, sd, w);
-        if (!(ok = mbar_wait(BAR(B_QFULL0), uc & 1, g))) break;
-        if (!(ok = mbar_wait(BAR(B_QFULL1), uc & 1, g))) break;
+        const int nkv = unit_kv_tiles<kRows>(p, sd, w);
+        if (!(ok = mbar_wait<kPair>(BAR(B_QFULL0), uc & 1, g))) break;
+        if (!(ok = mbar_wait<kPair>(BAR(B_QFULL1), uc & 1, g))) break;
         uint32_t ks = kc % kStages;
-        if (!(ok = mbar_wait(BAR(B_KFULL0 + ks), (kc / kStages) & 1, g))) break;
+        if (!(ok = mbar_wait<kPair>(BAR(B_KFULL0 + ks), (kc / kStages) & 1, g))) break;
         tc_fence_after();
         issue_s(0, ks);
-        mma_commit(BAR(B_SFULL0));
+        commit(B_SFULL0);
         issue_s(1, ks);
-        mma_commit(BAR(B_SFULL1));
+        commit(B_SFULL1);
         ++kc;
-        if (nkv == 1) mma_commit(BAR(B_QEMPTY));
+        if (nkv == 1) commit(B_QEMPTY);
         for (int t = 0; ok && t < nkv; ++t) {
           const uint32_t vs = vc % kStages;
-          if (!(ok = mbar_wait(BAR(B_VFULL0 + vs), (vc / kStages) & 1, g))) break;
+          if (!(ok = mbar_wait<kPair>(BAR(B_VFULL0 + vs), (vc / kStages) & 1, g))) break;
           for (int i = 0; i < 2; ++i) {
-            if (t == 0 && uc > 0 && !(ok = mbar_wait(BAR(B_OEMPTY0 + i), (uc - 1) & 1, g))) break;
-            if (!(ok = mbar_wait(BAR(B_PHALF0 + i), pc & 1, g))) break;
+            if (t == 0 && uc > 0 && !(ok = mbar_wait<kPair>(BAR(B_OEMPTY0 + i), (uc - 1) & 1, g))) break;
+            if (!(ok = mbar_wait<kPair>(BAR(B_PHALF0 + i), pc & 1, g))) break;
             tc_fence_after();
             issue_pv_half(i, vs, 0, t > 0);
-            if (!(ok = mbar_wait(BAR(B_PFULL0 + i), pc & 1, g))) break;
+            if (!(ok = mbar_wait<kPair>(BAR(B_PFULL0 + i), pc & 1, g))) break;
             tc_fence_after();
             issue_pv_half(i, vs, 1, 1);
             if (t == nkv - 1) {
-              mma_commit(BAR(B_OFULL0 + i));
+              commit(B_OFULL0 + i);
             } else if (i == 0) {
               ks = kc % kStages;
-              if (!(ok = mbar_wait(BAR(B_KFULL0 + ks), (kc / kStages) & 1, g))) break;
+              if (!(ok = mbar_wait<kPair>(BAR(B_KFULL0 + ks), (kc / kStages) & 1, g))) break;
               tc_fence_after();
               issue_s(0, ks);
-              mma_commit(BAR(B_SFULL0));
+              commit(B_SFULL0);
             } else {
               issue_s(1, ks);
-              mma_commit(BAR(B_SFULL1));
+              commit(B_SFULL1);
               ++kc;
-              if (t + 1 == nkv - 1) mma_commit(BAR(B_QEMPTY));
+              if (t + 1 == nkv - 1) commit(B_QEMPTY);
             }
           }
           ++pc;
@@ -469,7 +586,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++uc;
       }
       // drain: all MMAs this thread issued are complete before TMEM is freed
-      mma_commit(BAR(B_DONE));
+      if constexpr (kPair)
+        mma_commit_pair(LBAR(B_DONE));
+      else
+        mma_commit(BAR(B_DONE));
       drain_wait(BAR(B_DONE), 0);
     }
    }
@@ -487,15 +607,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       Unit w;
-      const int st = unit_of_cta(p, k, w);
+      const int st = unit_of_cta<kRows>(p, k, w, cta, ncta);
       if (st == 0 || st < 0) break;
       if (st == 2) continue;
       const SegDesc& sd = p.seg[w.seg];
-      const int nkv = unit_kv_tiles(p, sd, w);
+      const int nkv = unit_kv_tiles<kRows>(p, sd, w);
+      // first query row of this thread's tile in this CTA
+      const int tile_row0 = w.q0 + (kPair ? wg * 2 * BM + static_cast<int>(cr) * BM : wg * BM);
       float m_used = -INFINITY;   // running max, log2 units (scaled)
       float l = 0.f;              // running sum of exp2(x - m_used)
       for (int t = 0; t < nkv; ++t) {
-        if (!(ok = mbar_wait_warp(BAR(B_SFULL0 + wg), sc & 1, g))) break;
+        if (!(ok = mbar_wait_warp<kPair>(BAR(B_SFULL0 + wg), sc & 1, g))) break;
         ++sc;
         if (wg == 1 && row == 0) {
           // S1(t) complete => S0(t) complete (same issuer, issued earlier):
@@ -515,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* s = reinterpret_cast<float*>(&sraw[0][0]);
         // keys past the segment end, and (causal) past this row, are masked
         const int kv0 = sd.start + t * BN;
-        const int row_n = w.q0 + wg * BM + row;
+        const int row_n = tile_row0 + row;
         const int valid = (p.causal ? min(sd.kv_end, row_n + 1) : sd.kv_end) - kv0;   // may be <= 0
         const bool masked = __any_sync(0xffffffffu, valid < BN);
         if (masked) {
@@ -577,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           exp_store_half<false>(s, 0, scale2, negm2, acc, tS);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(B_PHALF0 + wg));
+        hand_off(B_PHALF0 + wg);
         if (kFp8 && emu)
           exp_store_half_fp8<true>(s, 1, scale2, negm2, acc, tS);
         else if (kFp8)
@@ -593,11 +715,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(B_PFULL0 + wg));
+        hand_off(B_PFULL0 + wg);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 -> global
-      if (!(ok = mbar_wait_warp(BAR(B_OFULL0 + wg), uc & 1, g))) break;
+      if (!(ok = mbar_wait_warp<kPair>(BAR(B_OFULL0 + wg), uc & 1, g))) break;
       if (wg == 1 && row == 0) mbar_arrive(BAR(B_VEMPTY0 + vslot++ % kStages));   // last V of the unit
       tc_fence_after();
       uint32_t oraw[4][32];
@@ -607,8 +729,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_regs_ready(oraw[c]);
       tc_fence_before();
-      mbar_arrive(BAR(B_OEMPTY0 + wg));
-      const int n = w.q0 + wg * BM + row;
+      hand_off(B_OEMPTY0 + wg);
+      const int n = tile_row0 + row;
       if (p.lse && n < sd.q_end && n < p.Np) {
         const int64_t li = (static_cast<int64_t>(w.r) * p.Hl + w.j) * p.lse_stride + n;
         if (in_bounds(li, 1, p.lse_ext, p.err)) p.lse[li] = m_used + log2f(l);
@@ -645,8 +767,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // in a pair, neither CTA frees TMEM or exits while the other's MMAs,
+  // commits or hand-offs may still reach it
+  if constexpr (kPair) cluster_sync();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (warp == kMmaWarp) {
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ AttnParams p) {
+  attn_body<kFp8, false>(&tmap, &tmap, p);
+}
+
+// bf16 attention on CTA pairs (clusters of two); tmapK reads 64-key halves of
+// the K tiles.
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmapK,
+                         const __grid_constant__ AttnParams p) {
+  attn_body<false, true>(&tmap, &tmapK, p);
 }
 
 // ---------------------------------------------------------------- host side
@@ -666,6 +810,51 @@ EncodeTiledFn get_encode_fn() {
     return static_cast<EncodeTiledFn>(nullptr);
   }();
   return fn;
+}
+
+// Largest number of CTA pairs resident at once (one pair per two SMs of a
+// cluster-capable partition), cached per device.
+int g_pair_clusters[256] = {0};
+
+cudaError_t launch_pair_kernel(const CUtensorMap& tmap, const CUtensorMap& tmapK, const AttnParams& p, int grid,
+                               int dev, cudaStream_t stream) {
+  static PerDeviceOnce setup;
+  cudaError_t e = setup.run(dev, [] {
+    cudaFuncAttributes fa;
+    cudaError_t r = cudaFuncGetAttributes(&fa, attn_fwd_pair_kernel);
+    if (r != cudaSuccess) return r;
+    if (fa.numRegs != static_cast<int>(kLaunchRegs)) return cudaErrorInvalidConfiguration;   // see register split
+    return cudaFuncSetAttribute(attn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Smem<false, true>::kBytes);
+  });
+  if (e != cudaSuccess) return e;
+  attn_fwd_pair_kernel<<<grid, kThreads, Smem<false, true>::kBytes, stream>>>(tmap, tmapK, p);
+  return cudaGetLastError();
+}
+
+int pair_clusters(int dev, int sms) {
+  static PerDeviceOnce setup;
+  if (dev < 0 || dev >= 256) return sms / 2;
+  const cudaError_t e = setup.run(dev, [dev, sms] {
+    cudaError_t r = cudaFuncSetAttribute(attn_fwd_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Smem<false, true>::kBytes);
+    if (r != cudaSuccess) return r;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Smem<false, true>::kBytes;
+    int n = 0;
+    r = cudaOccupancyMaxActiveClusters(&n, attn_fwd_pair_kernel, &cfg);
+    if (r != cudaSuccess) return r;
+    g_pair_clusters[dev] = n;
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return g_pair_clusters[dev];
 }
 
 template <bool kFp8>
@@ -718,12 +907,23 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   // one box is 128 rows of 128 bytes: 64 bf16 or 128 E4M3 columns
   cuuint32_t box[5] = {a.fp8 ? 128u : 64u, 1, BM, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUtensorMap tmap;
+  CUtensorMap tmap, tmapK;
   CUresult cr = encode(&tmap, a.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
                        const_cast<void*>(a.base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // bf16 attention runs on CTA pairs when the plan asks for it; the pair
+  // kernel also reads 64-key halves of the K tiles (boxes of 64 rows)
+  const bool pair = !a.fp8 && pl->pair_cta;
+  if (pair) {
+    cuuint32_t boxK[5] = {64, 1, BM / 2, 1, 1};
+    cr = encode(&tmapK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(a.base), dims, strides, boxK, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
+  const int unit_rows = pair ? kPairUnitRows : kUnitRows;
 
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
@@ -773,7 +973,7 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
     d.start = sg.start;
     d.kv_end = sg.end;
     d.q_end = (sg.end == a.N) ? static_cast<int32_t>(a.Np) : sg.end;
-    d.nqb = (d.q_end - d.start + kUnitRows - 1) / kUnitRows;
+    d.nqb = (d.q_end - d.start + unit_rows - 1) / unit_rows;
     d.unit_base = units;
     d.pair_base = pairs;
     units += d.nqb * a.P * a.Hl;
@@ -787,6 +987,12 @@ cudaError_t launch_attn(const AttnLaunch& a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (pair) {
+    const int clusters = pair_clusters(dev, sms);
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    p.paired = (p.causal && units >= 2 * clusters) ? 1 : 0;
+    return launch_pair_kernel(tmap, tmapK, p, 2 * std::min(units, clusters), dev, stream);
+  }
   p.paired = (p.causal && units >= 2 * sms) ? 1 : 0;
   const int grid = std::min(units, sms);
   return a.fp8 ? launch_kernel<true>(tmap, p, grid, dev, stream) : launch_kernel<false>(tmap, p, grid, dev, stream);

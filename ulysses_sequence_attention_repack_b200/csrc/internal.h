@@ -48,6 +48,7 @@ struct ulysses_plan_s {
   int32_t plane_chunk;
   int32_t num_seqs;
   int32_t causal;                       // attention sees keys m <= n only
+  int32_t pair_cta;                     // bf16 attention on CTA pairs (clusters of two) instead of one CTA per SM
   ulysses::Segment segs[ULYSSES_MAX_SEQS];
   int32_t device;                       // device the plan's scratch lives on (-1: none)
   unsigned int* dev_err;                // device error word (16 bytes allocated)

@@ -153,4 +153,5 @@ def test_peer_pointer_table_keeps_the_tensor_offset():
 
     layer = peer.PeerLayer.__new__(peer.PeerLayer)
     layer.rank = 1
+    layer.exchange = "symmetric"
     assert layer._peer_ptrs(Handle(), Local()) == [0x7000_0000_1000, 0x7100_0000_1000, 0x7200_0000_1000]

@@ -27,6 +27,13 @@ every rank's allocation into every peer (NVLink over NVSwitch) and provides
 the barrier; every byte of the layer is moved and computed by this library's
 kernels.  All ranks must build the plan with the same arguments; the
 constructor checks that (``agree_plan``).
+
+``exchange="ipc"`` maps the peers' buffers through CUDA IPC handles instead
+(ordinary allocations; the handles cross in one all-gather over the group),
+and each barrier becomes a host barrier: the stream is synchronised, then
+``torch.distributed.barrier``.  It serves groups without symmetric memory,
+gloo groups included, and processes that share one GPU: no kernel of one
+rank then waits on another rank's kernel.
 """
 from __future__ import annotations
 
@@ -67,57 +74,96 @@ class PeerLayer:
     """
 
     def __init__(self, plan: Plan, group=None, device=None, softmax_scale: float | None = None,
-                 training: bool = False):
+                 training: bool = False, exchange: str = "symmetric"):
         import torch
         import torch.distributed as dist
-        from torch.distributed import _symmetric_memory as symm
-        # no NVLink multicast object is needed: the kernels use plain peer stores
-        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
+        if exchange not in ("symmetric", "ipc"):
+            raise ValueError("exchange must be 'symmetric' or 'ipc'")
         agree_plan(plan, group)
         self.plan = plan
         self.group = group if group is not None else dist.group.WORLD
         self.rank = dist.get_rank(self.group)
         self.device = device if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.scale = float(softmax_scale) if softmax_scale is not None else 1.0 / math.sqrt(plan.D)
+        self.exchange = exchange
+        self._ipc_keep = []   # peer tensors opened from IPC handles (keep the mappings alive)
         C, Np, Nl, H = plan.planes, plan.padded_tokens, plan.rows_per_rank, plan.H
         Hl = H // plan.P
-        self.heads = symm.empty(C, Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
-        self.out = symm.empty(Nl, H, plan.D, dtype=torch.bfloat16, device=self.device)
-        self._heads_h = symm.rendezvous(self.heads, self.group)
-        self._out_h = symm.rendezvous(self.out, self.group)
+        bf = dict(dtype=torch.bfloat16, device=self.device)
+        # buffers the peers store into: (tensor, handle) pairs
+        self.heads, self._heads_h = self._shared((C, Np, Hl, plan.D))
+        self.out, self._out_h = self._shared((Nl, H, plan.D))
         self.heads_ptrs = self._peer_ptrs(self._heads_h, self.heads)
         self.out_ptrs = self._peer_ptrs(self._out_h, self.out)
         self.training = bool(training)
         if self.training:
             # this rank's output and lse for the backward, the dO slab and the
             # gradient shard the peers push into, and the backward's scratch
-            self.out_heads = torch.empty(Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
+            self.out_heads = torch.empty(Np, Hl, plan.D, **bf)
             self.lse = torch.empty(plan.slab_lse_bytes // 4, dtype=torch.float32, device=self.device)
-            self.dout_heads = symm.empty(1, Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
-            self.dqkv_heads = torch.empty(3, Np, Hl, plan.D, dtype=torch.bfloat16, device=self.device)
-            self.grad = symm.empty(Nl, 3, H, plan.D, dtype=torch.bfloat16, device=self.device)
+            self.dout_heads, self._dout_h = self._shared((1, Np, Hl, plan.D))
+            self.dqkv_heads = torch.empty(3, Np, Hl, plan.D, **bf)
+            self.grad, self._grad_h = self._shared((Nl, 3, H, plan.D))
             self.bwd_ws = torch.empty(plan.slab_attn_bwd_workspace_bytes, dtype=torch.uint8, device=self.device)
-            self._dout_h = symm.rendezvous(self.dout_heads, self.group)
-            self._grad_h = symm.rendezvous(self.grad, self.group)
             self.dout_ptrs = self._peer_ptrs(self._dout_h, self.dout_heads)
             self.grad_ptrs = self._peer_ptrs(self._grad_h, self.grad)
 
+    def _shared(self, shape):
+        """A bf16 buffer the peers can store into, and its exchange handle."""
+        import torch
+        if self.exchange == "ipc":
+            return torch.empty(shape, dtype=torch.bfloat16, device=self.device), None
+        from torch.distributed import _symmetric_memory as symm
+        # no NVLink multicast object is needed: the kernels use plain peer stores
+        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
+        t = symm.empty(*shape, dtype=torch.bfloat16, device=self.device)
+        return t, symm.rendezvous(t, self.group)
+
     def _peer_ptrs(self, handle, local) -> list[int]:
         """Every rank's address of the same tensor, as mapped on this device."""
+        if self.exchange == "ipc":
+            return self._ipc_ptrs(local)
         ptrs = [int(p) for p in handle.buffer_ptrs]
         off = local.data_ptr() - ptrs[self.rank]
         return [p + off for p in ptrs]
 
+    def _ipc_ptrs(self, local) -> list[int]:
+        """The peers' addresses of their copy of `local`, opened from the CUDA
+        IPC handles every rank publishes in one all-gather (a collective)."""
+        import torch.distributed as dist
+        from torch.multiprocessing.reductions import reduce_tensor
+        shared = [None] * dist.get_world_size(self.group)
+        dist.all_gather_object(shared, reduce_tensor(local), group=self.group)
+        ptrs = []
+        for r, (rebuild, args) in enumerate(shared):
+            if r == self.rank:
+                ptrs.append(local.data_ptr())
+                continue
+            t = rebuild(*args)
+            self._ipc_keep.append(t)
+            ptrs.append(t.data_ptr())
+        return ptrs
+
+    def _barrier(self, handle, channel: int) -> None:
+        """Every rank's stores issued so far are complete before any rank goes on."""
+        if self.exchange == "ipc":
+            import torch
+            import torch.distributed as dist
+            torch.cuda.current_stream(self.device).synchronize()
+            dist.barrier(group=self.group)
+        else:
+            handle.barrier(channel=channel)
+
     def forward(self, shard):
         """shard: this rank's rows [Nl, C, H, D] (bf16, on this rank's device)."""
         ulysses_repack_fwd_push(self.plan, self.rank, shard, self.heads_ptrs)
-        self._heads_h.barrier(channel=0)
+        self._barrier(self._heads_h, 0)
         if self.training:
             ulysses_attn_fwd_lse_slab(self.plan, self.heads, self.out_heads, self.lse, self.scale)
             ulysses_repack_bwd_push(self.plan, self.rank, self.out_heads, self.out_ptrs, 1)
         else:
             ulysses_attn_fwd_push(self.plan, self.rank, self.heads, self.out_ptrs, self.scale)
-        self._out_h.barrier(channel=1)
+        self._barrier(self._out_h, 1)
         return self.out
 
     __call__ = forward
@@ -130,11 +176,11 @@ class PeerLayer:
         if not self.training:
             raise RuntimeError("PeerLayer was built without training=True")
         ulysses_repack_fwd_push(self.plan, self.rank, dout_shard, self.dout_ptrs, 1)
-        self._dout_h.barrier(channel=0)
+        self._barrier(self._dout_h, 0)
         ulysses_attn_bwd_slab(self.plan, self.heads, self.out_heads, self.dout_heads, self.lse, self.dqkv_heads,
                               self.bwd_ws, self.scale)
         ulysses_repack_bwd_push(self.plan, self.rank, self.dqkv_heads, self.grad_ptrs, 3)
-        self._grad_h.barrier(channel=1)
+        self._barrier(self._grad_h, 1)
         return self.grad
 
 

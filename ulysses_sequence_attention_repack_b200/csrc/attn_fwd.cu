@@ -65,6 +65,7 @@ constexpr int kThreads = 384;      // 3 warpgroups
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
 constexpr int kFwdWarp = 10;        // CTA pairs: forwards the odd CTA's completed fills
+constexpr int kHandWarp = 11;       // CTA pairs: forwards the odd CTA's P and O hand-offs
 // Register split: the kernel is launched with kLaunchRegs per thread
 // (384 x 168 = 64512); warpgroup 2 (TMA, MMA, two spare warps) drops to
 // kProducerRegs and the two softmax warpgroups rise to kSoftmaxRegs:
@@ -344,22 +345,18 @@ __device__ __forceinline__ void attn_body(const CUtensorMap* tmap, const CUtenso
       mma_commit(BAR(i));
     }
   };
-  // a P or O hand-off of this softmax thread: per thread, or per warp of both
-  // CTAs onto the even CTA's barrier
-  auto hand_off = [&](int i) {
-    if constexpr (kPair) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(LBAR(i));
-    } else {
-      mbar_arrive(BAR(i));
-    }
-  };
+  // a P or O hand-off of this softmax thread: a CTA-scope arrival on its own
+  // CTA's barrier (in a pair, the odd CTA's completed phases are forwarded to
+  // the even CTA by warp kHandWarp, so no softmax thread pays a cluster-scope
+  // release)
+  auto hand_off = [&](int i) { mbar_arrive(BAR(i)); };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    // the even CTA's fill barriers also take the odd CTA's forwarded arrival
+    // the even CTA's fill and hand-off barriers also take the odd CTA's
+    // forwarded arrival
     const uint32_t fills = (kPair && leader) ? 2 : 1;
-    const uint32_t hands = kPair ? 8 : BM;   // 4 warps x 2 CTAs, or 128 threads
+    const uint32_t hands = (kPair && leader) ? BM + 1 : BM;
     mbar_init(BAR(B_QFULL0), fills);
     mbar_init(BAR(B_QFULL1), fills);
     mbar_init(BAR(B_QEMPTY), 1);
@@ -493,6 +490,37 @@ __device__ __forceinline__ void attn_body(const CUtensorMap* tmap, const CUtenso
           if (!(ok = mbar_wait(BAR(B_VFULL0 + vc % kStages), (vc / kStages) & 1, g))) break;
           mbar_arrive_cluster(LBAR(B_VFULL0 + vc % kStages));
           ++vc;
+        }
+        ++uc;
+      }
+    }
+   } else if (kPair && warp == kHandWarp) {
+    // ------------------------------------------------------------ hand-off forwarder (odd CTA of a pair)
+    // Forwards this CTA's completed P and O hand-off phases to the even CTA,
+    // in the order the MMA thread consumes them (O of the previous unit, then
+    // P by halves, tile 0 before tile 1), so this CTA's barrier is never more
+    // than one phase ahead of the forwarder.
+    if (!leader && lane == 0) {
+      uint32_t pc = 0, uc = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        Unit w;
+        const int st = unit_of_cta<kRows>(p, k, w, cta, ncta);
+        if (st == 0 || st < 0) break;
+        if (st == 2) continue;
+        const int nkv = unit_kv_tiles<kRows>(p, p.seg[w.seg], w);
+        for (int t = 0; ok && t < nkv; ++t) {
+          for (int i = 0; ok && i < 2; ++i) {
+            if (t == 0 && uc > 0) {
+              if (!(ok = mbar_wait(BAR(B_OEMPTY0 + i), (uc - 1) & 1, g))) break;
+              mbar_arrive_cluster(LBAR(B_OEMPTY0 + i));
+            }
+            if (!(ok = mbar_wait(BAR(B_PHALF0 + i), pc & 1, g))) break;
+            mbar_arrive_cluster(LBAR(B_PHALF0 + i));
+            if (!(ok = mbar_wait(BAR(B_PFULL0 + i), pc & 1, g))) break;
+            mbar_arrive_cluster(LBAR(B_PFULL0 + i));
+          }
+          ++pc;
         }
         ++uc;
       }

@@ -245,7 +245,7 @@ def run_ours(args, rank, world, local_rank):
     P, N, H, C, seed, cu = WORKLOADS[args.config]
     causal = args.config in CAUSAL
     Hl = H // P
-    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu, causal=causal)
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu, causal=causal, pair_cta=args.pair_attention)
     Np = plan.padded_tokens
     S = inputs.qkv_seq(N, H, P, C, seed, dev)
     T = torch.empty((P, C, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
@@ -431,7 +431,7 @@ def run_ours(args, rank, world, local_rank):
     rb_gbs = rb_bytes / (rb_ms * 1e-3) / 1e9
     ms_per_step = total_ms / args.steps
     launches_per_step = math.ceil(C / plan.plane_chunk) + 1 + 1
-    traffic = recorded_traffic("attn_fwd_kernel", args.config)
+    traffic = recorded_traffic("attn_fwd_pair_kernel" if args.pair_attention else "attn_fwd_kernel", args.config)
     tpk, tpk_kind = tensor_peak(pk)
     spk = sustained_peak(pk)
     for w in others.values():
@@ -453,6 +453,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD_TEXT[args.config], "name": args.config, "P": P, "N": N, "Np": Np,
                    "H": H, "D": 128, "planes": C, "seed": seed, "cu_seqlens": cu, "causal": causal,
                    "step": "repack_fwd + attn_fwd + repack_bwd(output), one C-ABI call each",
+                   "attention_kernel": "CTA pairs" if args.pair_attention else "one CTA per SM",
                    "replicas": world, "l2": f"inputs larger than L2 ({S.numel() * 2 / 1e6:.0f} MB per step)"},
         "attn_us": round(at_ms * 1000, 2),
         "attn_tflops": round(attn_tflops, 1),
@@ -474,7 +475,8 @@ def run_ours(args, rank, world, local_rank):
         "attn_bwd_tflops": round(2.5 * flops / (bwd_ms * 1e-3) / 1e12, 1),
         "prologue_repack_fwd_us": round(prologue_ms * 1000, 2),
         "prologue_repack_fwd_gbs": round(rf_bytes / (prologue_ms * 1e-3) / 1e9, 1),
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": round(attn_tflops, 1),
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_pair_kernel" if args.pair_attention else "attn_fwd_kernel",
+                     "achieved": round(attn_tflops, 1),
                      "peak": tpk, "peak_kind": f"{pk_kind} {tpk_kind}", "unit": "TFLOP/s",
                      "frac": round(attn_tflops / tpk, 3),
                      "frac_of_sustained": round(attn_tflops / spk, 3), "traffic": traffic,
@@ -861,6 +863,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip the other layer workloads timed after the main one")
+    ap.add_argument("--pair-attention", action="store_true",
+                    help="run the bf16 attention on CTA pairs (ULYSSES_PLAN_PAIR_ATTENTION) instead of one CTA per SM")
     ap.add_argument("--transport", default="replicas", choices=["replicas", "peer", "nccl"],
                     help="replicas (default): every GPU runs the whole one-GPU layer; peer / nccl: "
                          "the layer split across the launched GPUs, one rank each")

@@ -84,6 +84,13 @@ enum {
  * slower (the cross-SM hand-offs lengthen the S -> softmax -> P V chain that
  * bounds the loop), so it is opt-in. */
 #define ULYSSES_PLAN_PAIR_ATTENTION 2u
+/* ulysses_plan_ex flag: run the attention backward in two passes without
+ * atomics (keys, then queries; S and dP are computed in both), so its output
+ * is the same bits on every run.  The default is one pass over the keys that
+ * adds dQ into an fp32 accumulator in the workspace with reductions performed
+ * in L2: faster, but the order of those additions varies between runs, and so
+ * can the last bit of a dQ value. */
+#define ULYSSES_PLAN_DETERMINISTIC 4u
 /* Most ranks the multi-GPU push calls address (one NVLink domain). */
 #define ULYSSES_MAX_PUSH_RANKS 64
 
@@ -119,7 +126,7 @@ int ulysses_plan(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t 
                  const int32_t* cu_seqlens_host, int32_t num_seqs);
 
 /* ulysses_plan with option flags (ULYSSES_PLAN_CAUSAL,
- * ULYSSES_PLAN_PAIR_ATTENTION); ulysses_plan is
+ * ULYSSES_PLAN_PAIR_ATTENTION, ULYSSES_PLAN_DETERMINISTIC); ulysses_plan is
  * ulysses_plan_ex with flags = 0.  Unknown flag bits -> ULYSSES_ERR_ARG. */
 int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32_t P, int32_t planes,
                     int64_t token_stride, int64_t plane_stride, int64_t plane_chunk,
@@ -370,7 +377,9 @@ int ulysses_attn_fwd_lse(const ulysses_plan_t* plan, const void* qkv_heads, void
                          float softmax_scale, void* stream);
 
 /* Workspace of ulysses_attn_bwd: the row terms -rowsum(dO o O) and a negated
- * copy of lse, each ulysses_lse_bytes() long. */
+ * copy of lse, each ulysses_lse_bytes() long, then (unless the plan has
+ * ULYSSES_PLAN_DETERMINISTIC) the fp32 dQ accumulator, P*Hl*Np*D*4 bytes
+ * from the next 256-byte boundary. */
 size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan);
 
 /*
@@ -378,8 +387,10 @@ size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan);
  * qkv_heads T [P, C, Np, Hl, D], its output out_heads O_T [P, Np, Hl, D], the
  * output gradient dout_heads [P, Np, Hl, D] and the forward's lse.  Honors the
  * plan's segments and causal flag; pad rows get zero gradients.  fp32
- * accumulation, bf16 output.  Two passes over the keys and the queries; no
- * atomics, deterministic.  Errors: ARG, ALIGN, WORKSPACE, CUDA.
+ * accumulation, bf16 output.  By default one pass over the keys: dK and dV
+ * accumulate in TMEM, dQ in the workspace's fp32 accumulator through L2
+ * reductions (run-to-run order varies; see ULYSSES_PLAN_DETERMINISTIC for the
+ * two-pass, bit-reproducible form).  Errors: ARG, ALIGN, WORKSPACE, CUDA.
  */
 int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads,
                      const void* dout_heads, const void* lse, void* dqkv_heads, void* workspace,
@@ -451,8 +462,9 @@ int ulysses_layer_fwd_host(const ulysses_plan_t* plan, const void* host_qkv_seq,
  * (1 = a pipeline wait timed out and the kernel gave up; 2 = a work unit
  * decoded outside the problem; 4 = in the bounds-checked build
  * libulysses_debug.so only, a computed global offset fell outside its
- * buffer and the access was skipped), or -1 if the synchronisation itself
- * failed.
+ * buffer and the access was skipped; 8 = the one-pass attention backward
+ * found its dynamic shared memory not 1024-byte aligned and did nothing), or
+ * -1 if the synchronisation itself failed.
  */
 int ulysses_last_device_error(const ulysses_plan_t* plan, void* stream);
 

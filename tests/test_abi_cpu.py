@@ -65,7 +65,8 @@ def test_plan_flags():
     lib = U.load()
     h = ctypes.c_void_p()
     for flags, want in ((0, 0), (_lib.ULYSSES_PLAN_CAUSAL, 0), (_lib.ULYSSES_PLAN_PAIR_ATTENTION, 0),
-                        (_lib.ULYSSES_PLAN_CAUSAL | _lib.ULYSSES_PLAN_PAIR_ATTENTION, 0), (4, _lib.ULYSSES_ERR_ARG)):
+                        (_lib.ULYSSES_PLAN_CAUSAL | _lib.ULYSSES_PLAN_PAIR_ATTENTION, 0),
+                        (_lib.ULYSSES_PLAN_DETERMINISTIC, 0), (7, 0), (8, _lib.ULYSSES_ERR_ARG)):
         code = lib.ulysses_plan_ex(ctypes.byref(h), 1024, 8, 128, 2, 3, 0, 0, 0, None, 0, flags)
         assert code == want, (flags, code)
         if code == 0:

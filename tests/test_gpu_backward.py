@@ -1,5 +1,9 @@
 """Attention backward and layer backward against the fp64 oracle.
 
+Both forms of the backward are checked: the default one pass over the keys
+(dQ added into an fp32 accumulator through L2 reductions) and the two-pass
+deterministic form (plan flag ULYSSES_PLAN_DETERMINISTIC).
+
 The GPU path rounds P and dS to bf16 for its tensor-core products (as the
 forward rounds P), accumulates in fp32 and rounds the gradients to bf16 once.
 Each bf16 rounding is a relative error of at most 2^-8 (RMS 1.66e-3, see
@@ -49,12 +53,16 @@ def _close(got, ref, what, record=True):
         check_attention(f"backward {what}", got, ref, max_abs=None, mean_abs=None)
 
 
+FORMS = [pytest.param(False, id="one-pass"), pytest.param(True, id="two-pass")]
+
+
+@pytest.mark.parametrize("deterministic", FORMS)
 @pytest.mark.parametrize("P,N,H,cu,causal,seed", CASES)
-def test_attention_backward_against_oracle(gpu, P, N, H, cu, causal, seed):
+def test_attention_backward_against_oracle(gpu, P, N, H, cu, causal, seed, deterministic):
     import torch
     import ulysses_sequence_attention_repack_b200 as U
     from ulysses_sequence_attention_repack_b200 import inputs
-    plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=causal)
+    plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=causal, deterministic=deterministic)
     Np, Hl = plan.padded_tokens, H // P
     scale = 1.0 / math.sqrt(128)
     S = inputs.qkv_seq(N, H, P, 3, 100 + seed, gpu)
@@ -77,8 +85,9 @@ def test_attention_backward_against_oracle(gpu, P, N, H, cu, causal, seed):
     ref = orc.attention_heads_bwd(T_bits, inputs.host_bits(dO), N, scale, cu, causal)
     got = dT.float().cpu().numpy().astype(np.float64)
     assert np.all(np.isfinite(got))
+    form = "two-pass" if deterministic else "one-pass"
     for c, name in enumerate(("dQ", "dK", "dV")):
-        _close(got[:, c, :N], ref[:, c, :N], name)
+        _close(got[:, c, :N], ref[:, c, :N], f"{name} {form}")
     assert np.all(got[:, :, N:] == 0)               # pad rows get no gradient
     # lse check: log2 of sum_m exp2(s log2e q.k) per row, fp64
     q = orc.bf16_bits_to_f64(T_bits[:, 0])
@@ -97,12 +106,13 @@ def test_attention_backward_against_oracle(gpu, P, N, H, cu, causal, seed):
                 assert np.abs(got_lse[r * Hl + j, a:b] - want).max() < 1e-3
 
 
+@pytest.mark.parametrize("deterministic", FORMS)
 @pytest.mark.parametrize("P,N,H,cu,causal", [(2, 1024, 8, None, False), (4, 1001, 8, [0, 500, 1001], True)])
-def test_layer_backward_against_oracle(gpu, P, N, H, cu, causal):
+def test_layer_backward_against_oracle(gpu, P, N, H, cu, causal, deterministic):
     import torch
     import ulysses_sequence_attention_repack_b200 as U
     from ulysses_sequence_attention_repack_b200 import inputs
-    plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=causal)
+    plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=causal, deterministic=deterministic)
     Np, Hl = plan.padded_tokens, H // P
     scale = 1.0 / math.sqrt(128)
     S = inputs.qkv_seq(N, H, P, 3, 300, gpu)
@@ -127,8 +137,9 @@ def test_layer_backward_against_oracle(gpu, P, N, H, cu, causal):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("deterministic", FORMS)
 @pytest.mark.parametrize("causal", [False, True])
-def test_attention_backward_dit19k(gpu, causal):
+def test_attention_backward_dit19k(gpu, causal, deterministic):
     """Video-DiT size (P=4, N=19,394, H=56), as the benchmark times it.
 
     Every head: sum_k dK[k] = 0 (each row of dS sums to zero) and
@@ -139,7 +150,7 @@ def test_attention_backward_dit19k(gpu, causal):
     import ulysses_sequence_attention_repack_b200 as U
     from ulysses_sequence_attention_repack_b200 import inputs
     P, N, H = 4, 19_394, 56
-    plan = U.ulysses_plan(N, H, 128, P, 3, causal=causal)
+    plan = U.ulysses_plan(N, H, 128, P, 3, causal=causal, deterministic=deterministic)
     Np, Hl = plan.padded_tokens, H // P
     scale = 1.0 / math.sqrt(128)
     S = inputs.qkv_seq(N, H, P, 3, 1, gpu)
@@ -193,5 +204,49 @@ def test_attention_backward_dit19k(gpu, causal):
                 pairs["dV"][0].append(got_v[r, :, j])
                 pairs["dV"][1].append(dv)
     for name, (g_l, r_l) in pairs.items():
-        check_attention(f"backward dit19k causal={causal} {name} (sampled rows)", np.stack(g_l), np.stack(r_l),
-                        max_abs=None, mean_abs=None)
+        form = "two-pass" if deterministic else "one-pass"
+        check_attention(f"backward dit19k causal={causal} {form} {name} (sampled rows)", np.stack(g_l),
+                        np.stack(r_l), max_abs=None, mean_abs=None)
+
+
+@pytest.mark.parametrize("P,N,H,cu,causal", [(2, 1024, 8, None, False), (4, 1001, 8, [0, 500, 1001], True)])
+def test_backward_repeatability(gpu, P, N, H, cu, causal):
+    """The two-pass form gives the same bits on every run.  The one-pass form
+    gives the same dK and dV bits (each key block's loop runs in one CTA in a
+    fixed order); its dQ is summed by L2 reductions in whatever order the CTAs
+    reach them, so two runs agree to within rounding: here within one bf16
+    step of the larger value, plus 1e-6 of the tensor's largest magnitude for
+    sums that cancel to near zero."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    scale = 1.0 / math.sqrt(128)
+    runs = {}
+    for det in (False, True):
+        plan = U.ulysses_plan(N, H, 128, P, 3, 0, 0, 0, cu, causal=causal, deterministic=det)
+        Np, Hl = plan.padded_tokens, H // P
+        S = inputs.qkv_seq(N, H, P, 3, 400, gpu)
+        T = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+        U.ulysses_repack_fwd(plan, S, T)
+        OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+        lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=gpu)
+        U.ulysses_attn_fwd_lse(plan, T, OT, lse, scale)
+        dO = _grad(gpu, (P, Np, Hl, 128), 401)
+        dO[:, N:] = 0
+        ws = torch.empty(plan.attn_bwd_workspace_bytes, dtype=torch.uint8, device=gpu)
+        outs = []
+        for _ in range(3):
+            dT = torch.full((P, 3, Np, Hl, 128), float("nan"), dtype=torch.bfloat16, device=gpu)
+            U.ulysses_attn_bwd(plan, T, OT, dO, lse, dT, ws, scale)
+            outs.append(dT)
+        torch.cuda.synchronize()
+        assert U.ulysses_last_device_error(plan) == 0
+        runs[det] = outs
+    for dT in runs[True][1:]:
+        assert torch.equal(dT.view(torch.int16), runs[True][0].view(torch.int16))
+    a = runs[False][0]
+    for b in runs[False][1:]:
+        assert torch.equal(b[:, 1:].view(torch.int16), a[:, 1:].view(torch.int16))
+        x, y = a[:, 0].double(), b[:, 0].double()
+        tol = 2.0 ** -7 * torch.maximum(x.abs(), y.abs()) + 1e-6 * x.abs().max()
+        assert ((x - y).abs() <= tol).all()

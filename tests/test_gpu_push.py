@@ -38,11 +38,11 @@ def _bits(t):
     return inputs.host_bits(t)
 
 
-def _setup(gpu, P, N, H, C, cu, causal, seed):
+def _setup(gpu, P, N, H, C, cu, causal, seed, deterministic=False):
     import torch
     import ulysses_sequence_attention_repack_b200 as U
     from ulysses_sequence_attention_repack_b200 import inputs
-    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu, causal=causal)
+    plan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu, causal=causal, deterministic=deterministic)
     Np, Nl, Hl = plan.padded_tokens, plan.rows_per_rank, H // P
     S = inputs.qkv_seq(N, H, P, C, seed, gpu)
     shards = [S[q * Nl:(q + 1) * Nl].clone() for q in range(P)]
@@ -139,7 +139,7 @@ dist.init_process_group("nccl", init_method="tcp://127.0.0.1:%d" % int(sys.argv[
 dev = torch.device("cuda", 0)
 torch.cuda.set_device(dev)
 N, H, C = 1000, 4, 3
-plan = U.ulysses_plan(N, H, 128, 1, C)
+plan = U.ulysses_plan(N, H, 128, 1, C, deterministic=True)   # gradients compared bit for bit
 layer = peer.PeerLayer(plan)
 S = inputs.qkv_seq(N, H, 1, C, 68, dev)
 out = layer(S).clone()
@@ -208,15 +208,19 @@ TRAIN_CASES = [
 ]
 
 
+@pytest.mark.parametrize("deterministic", [pytest.param(True, id="two-pass"), pytest.param(False, id="one-pass")])
 @pytest.mark.parametrize("P,N,H,C,cu,causal,seed", TRAIN_CASES)
-def test_push_training_path_equals_one_gpu_backward(gpu, P, N, H, C, cu, causal, seed):
+def test_push_training_path_equals_one_gpu_backward(gpu, P, N, H, C, cu, causal, seed, deterministic):
     """The multi-GPU training path with the ranks emulated: per-slab attention
     with lse, output pushed back, dO pushed into the slabs, the per-slab
     backward, gradients pushed to their owners.  Output, lse and gradients
-    equal the one-GPU layer and ulysses_layer_bwd bit for bit."""
+    equal the one-GPU layer and ulysses_layer_bwd bit for bit with the
+    deterministic backward; with the one-pass backward dK and dV still do, and
+    dQ (summed by L2 reductions in a varying order) agrees to within
+    rounding."""
     import torch
     import ulysses_sequence_attention_repack_b200 as U
-    plan, S, shards, T = _setup(gpu, P, N, H, C, cu, causal, seed)
+    plan, S, shards, T = _setup(gpu, P, N, H, C, cu, causal, seed, deterministic=deterministic)
     Np, Nl, Hl = plan.padded_tokens, plan.rows_per_rank, H // P
     scale = 1.0 / math.sqrt(128)
     g = torch.Generator(device=gpu)
@@ -264,7 +268,15 @@ def test_push_training_path_equals_one_gpu_backward(gpu, P, N, H, C, cu, causal,
         assert np.array_equal(mine, lse_h[r]), f"lse of rank {r}"
         assert np.array_equal(_bits(OTr[r]), _bits(OT[r])), f"output slab of rank {r}"
     got = np.concatenate([_bits(x) for x in G], 0)
-    assert np.array_equal(got, _bits(dS)[:, :3])
+    want = _bits(dS)[:, :3]
+    if deterministic:
+        assert np.array_equal(got, want)
+    else:
+        assert np.array_equal(got[:, 1:], want[:, 1:])
+        x = torch.cat(G, 0)[:, 0].double()
+        y = dS[:, 0].double()
+        tol = 2.0 ** -7 * torch.maximum(x.abs(), y.abs()) + 1e-6 * y.abs().max()
+        assert ((x - y).abs() <= tol).all()
 
 
 @pytest.mark.parametrize("P,N,H,C,seed", [pytest.param(4, 1001, 8, 3, 73, id="P4-N1001"),

@@ -26,6 +26,7 @@ ULYSSES_ERR_DEVICE = 7
 ULYSSES_ERR_UNSUPPORTED = 8
 ULYSSES_PLAN_CAUSAL = 1
 ULYSSES_PLAN_PAIR_ATTENTION = 2
+ULYSSES_PLAN_DETERMINISTIC = 4
 MAX_SEQS = 64
 MAX_WINDOW_BYTES = 1024 ** 3
 
@@ -254,9 +255,11 @@ class Plan:
 
 
 def ulysses_plan(N: int, H: int, D: int, P: int, planes: int, token_stride: int = 0, plane_stride: int = 0,
-                 plane_chunk: int = 0, cu_seqlens=None, causal: bool = False, pair_cta: bool = False) -> Plan:
+                 plane_chunk: int = 0, cu_seqlens=None, causal: bool = False, pair_cta: bool = False,
+                 deterministic: bool = False) -> Plan:
     """ulysses_plan (or ulysses_plan_ex with ULYSSES_PLAN_CAUSAL when causal,
-    ULYSSES_PLAN_PAIR_ATTENTION when pair_cta)."""
+    ULYSSES_PLAN_PAIR_ATTENTION when pair_cta, ULYSSES_PLAN_DETERMINISTIC when
+    deterministic)."""
     lib = load()
     h = ctypes.c_void_p()
     if cu_seqlens is None:
@@ -265,7 +268,8 @@ def ulysses_plan(N: int, H: int, D: int, P: int, planes: int, token_stride: int 
         vals = [int(x) for x in cu_seqlens]
         arr = (ctypes.c_int32 * len(vals))(*vals)
         ns = len(vals) - 1
-    flags = (ULYSSES_PLAN_CAUSAL if causal else 0) | (ULYSSES_PLAN_PAIR_ATTENTION if pair_cta else 0)
+    flags = ((ULYSSES_PLAN_CAUSAL if causal else 0) | (ULYSSES_PLAN_PAIR_ATTENTION if pair_cta else 0)
+             | (ULYSSES_PLAN_DETERMINISTIC if deterministic else 0))
     if flags:
         code = lib.ulysses_plan_ex(ctypes.byref(h), int(N), int(H), int(D), int(P), int(planes), int(token_stride),
                                    int(plane_stride), int(plane_chunk), arr, ns, flags)

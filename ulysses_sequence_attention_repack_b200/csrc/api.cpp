@@ -406,7 +406,8 @@ int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32
                     int32_t num_seqs, uint32_t flags) {
   if (!out) return ULYSSES_ERR_ARG;
   *out = nullptr;
-  if (flags & ~(ULYSSES_PLAN_CAUSAL | ULYSSES_PLAN_PAIR_ATTENTION)) return ULYSSES_ERR_ARG;
+  if (flags & ~(ULYSSES_PLAN_CAUSAL | ULYSSES_PLAN_PAIR_ATTENTION | ULYSSES_PLAN_DETERMINISTIC))
+    return ULYSSES_ERR_ARG;
   if (D != kHeadDim) return ULYSSES_ERR_UNSUPPORTED;
   if (N < 1 || H < 1 || P < 1 || planes < 1 || planes > kMaxPlanes) return ULYSSES_ERR_ARG;
   if (H > kMaxHeads) return ULYSSES_ERR_UNSUPPORTED;
@@ -471,6 +472,7 @@ int ulysses_plan_ex(ulysses_plan_t** out, int64_t N, int32_t H, int32_t D, int32
   p->num_seqs = nseq;
   p->causal = (flags & ULYSSES_PLAN_CAUSAL) ? 1 : 0;
   p->pair_cta = (flags & ULYSSES_PLAN_PAIR_ATTENTION) ? 1 : 0;
+  p->deterministic = (flags & ULYSSES_PLAN_DETERMINISTIC) ? 1 : 0;
   std::memcpy(p->segs, segs, sizeof(ulysses::Segment) * nseq);
   p->device = -1;
   p->dev_err = nullptr;
@@ -660,8 +662,18 @@ int ulysses_attn_fwd_lse(const ulysses_plan_t* plan, const void* qkv_heads, void
                    static_cast<float*>(lse));
 }
 
+// The one-pass backward's fp32 dQ accumulator [P*Hl][Np][D] (none for a
+// deterministic plan), placed after the row terms at a 256-byte boundary.
+// The offset rounds to 256 * P bytes so that the workspace is exactly P times
+// that of one rank's slab (ulysses_attn_bwd_slab takes 1/P of it).
+static int64_t dq_acc_offset(const ulysses_plan_t* plan) { return align_up(2 * lse_bytes(plan), 256 * plan->P); }
+static int64_t dq_acc_bytes(const ulysses_plan_t* plan) {
+  return plan->deterministic ? 0 : static_cast<int64_t>(plan->P) * plan->Hl * plan->Np * plan->D * 4;
+}
+
 size_t ulysses_attn_bwd_workspace_bytes(const ulysses_plan_t* plan) {
-  return plan ? static_cast<size_t>(2 * lse_bytes(plan)) : 0;
+  if (!plan) return 0;
+  return static_cast<size_t>(plan->deterministic ? 2 * lse_bytes(plan) : dq_acc_offset(plan) + dq_acc_bytes(plan));
 }
 
 int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads,
@@ -674,7 +686,8 @@ int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const vo
   const void* ptrs[] = {qkv_heads, out_heads, dout_heads, lse, dqkv_heads, workspace};
   for (const void* q : ptrs)
     if (!aligned16(q)) return ULYSSES_ERR_ALIGN;
-  const int64_t dq = heads_bytes(plan, 3), lb = lse_bytes(plan), ws = 2 * lb;
+  const int64_t dq = heads_bytes(plan, 3), lb = lse_bytes(plan),
+                ws = static_cast<int64_t>(ulysses_attn_bwd_workspace_bytes(plan));
   if (overlap(dqkv_heads, dq, qkv_heads, heads_bytes(plan, plan->C)) || overlap(dqkv_heads, dq, out_heads, heads_bytes(plan, 1)) ||
       overlap(dqkv_heads, dq, dout_heads, heads_bytes(plan, 1)) || overlap(dqkv_heads, dq, lse, lb) ||
       overlap(workspace, ws, dqkv_heads, dq) || overlap(workspace, ws, lse, lb) ||
@@ -689,6 +702,9 @@ int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const vo
   a.dout = dout_heads;
   a.lse = static_cast<const float*>(lse);
   a.delta = static_cast<float*>(workspace);
+  a.dq_acc = plan->deterministic
+                 ? nullptr
+                 : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dq_acc_offset(plan));
   a.dqkv = dqkv_heads;
   a.scale = softmax_scale;
   a.plan = plan;
@@ -698,7 +714,7 @@ int ulysses_attn_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const vo
 size_t ulysses_layer_bwd_workspace_bytes(const ulysses_plan_t* plan) {
   if (!plan) return 0;
   return static_cast<size_t>(align_up(heads_bytes(plan, 1), 256) + align_up(heads_bytes(plan, 3), 256) +
-                             align_up(2 * lse_bytes(plan), 256));
+                             align_up(static_cast<int64_t>(ulysses_attn_bwd_workspace_bytes(plan)), 256));
 }
 
 int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const void* out_heads, const void* lse,
@@ -734,6 +750,8 @@ int ulysses_layer_bwd(const ulysses_plan_t* plan, const void* qkv_heads, const v
   a.dout = dOT;
   a.lse = static_cast<const float*>(lse);
   a.delta = delta;
+  a.dq_acc = plan->deterministic ? nullptr
+                                 : reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(delta) + dq_acc_offset(plan));
   a.dqkv = dT;
   a.scale = 1.0f / std::sqrt(static_cast<float>(plan->D));
   a.plan = plan;

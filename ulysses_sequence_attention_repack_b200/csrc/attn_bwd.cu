@@ -11,17 +11,24 @@
 // forward's plan ("hao-ai-lab FastVideo, compare main...perf/ulysses-h3-
 // adaptive", ulysses_a2a.py).
 //
-// Two passes, no atomics:
-//   pass A (one CTA unit = 128 keys of one head and sequence, loop over query
-//           blocks): S^T = K Q^T and dP^T = V dO^T into TMEM, then
-//           P^T and dS^T (bf16, aliased over them), then
-//           dV += P^T dO and dK += dS^T Q with A read from TMEM;
-//   pass B (unit = 128 queries, loop over key blocks): S = Q K^T and
+// Default, one pass over the keys (kModeAQ): one CTA unit = 128 keys of one
+// head and sequence, looping over the query blocks: S^T = K Q^T and
+// dP^T = V dO^T into TMEM, then P^T and dS^T (bf16, aliased over them),
+// dV += P^T dO and dK += dS^T Q with A read from TMEM, and dQ^T = K^T dS^T
+// with dS also stored to shared memory; a fourth warpgroup adds each dQ^T
+// block into an fp32 accumulator in global memory (reductions performed in
+// L2, so the order of the additions, and the last bits of dQ, vary from run
+// to run), which a last kernel scales and rounds to bf16.
+//
+// Deterministic, two passes, no atomics (plan flag DETERMINISTIC):
+//   pass A (kModeA, the loop above without dQ), then
+//   pass B (kModeB, unit = 128 queries, loop over key blocks): S = Q K^T and
 //           dP = dO V^T, then dS (bf16, over dP), then dQ += dS K.
-// Both reuse the forward's machinery: TMA-fed 128B-swizzled tiles, grouped
+// All reuse the forward's machinery: TMA-fed 128B-swizzled tiles, grouped
 // tcgen05 MMAs issued by one thread, bounded mbarrier waits.  Warps: 0-7
 // elementwise and epilogue (two warpgroups, each one thread per TMEM lane and
-// 64 of the 128 columns), 8 MMA issuer, 9 TMA producer.
+// 64 of the 128 columns), 8 MMA issuer, 9 TMA producer; kModeAQ adds warps
+// 12-15 (dQ reduction; 10 and 11 only complete their warpgroup).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,16 +37,28 @@
 #include <cstdint>
 #include <cstring>
 
+#include "bounds.cuh"
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
 namespace ulysses {
 namespace {
 
+constexpr int kModeA = 0;    // dK, dV (loop over query blocks)
+constexpr int kModeB = 1;    // dQ (loop over key blocks)
+constexpr int kModeAQ = 2;   // dK, dV and dQ in one loop over query blocks
 constexpr int kEwWarps = 8;                           // two warpgroups, 64 columns each
-constexpr int kThreads = 32 * (kEwWarps + 2);         // + the MMA and TMA warps
 constexpr int kMmaWarp = kEwWarps;
 constexpr int kTmaWarp = kEwWarps + 1;
+constexpr int kDqWarp0 = 12;                          // kModeAQ: warps 12-15 reduce dQ
+template <int kMode>
+constexpr int threads_of() {
+  return kMode == kModeAQ ? 512 : 32 * (kEwWarps + 2);
+}
+// kModeAQ register split (setmaxnreg), against the 128 per thread a 512-thread
+// CTA is launched with: 256 x 168 + 128 x 80 + 128 x 96 = 512 x 128.
+constexpr uint32_t kEwRegs = 168, kCtlRegs = 80, kDqRegs = 96;
+static_assert(256 * kEwRegs + 128 * kCtlRegs + 128 * kDqRegs == 512 * 128, "register split");
 constexpr int BT = 128;                               // rows per tile (keys or queries)
 constexpr int HD = 128;
 constexpr uint32_t kHalfBytes = BT * 64 * 2;          // 16 KB swizzled box
@@ -56,23 +75,45 @@ constexpr uint32_t kOffX = 2 * kTileBytes;                    // [stage][X0, X1]
 constexpr uint32_t kRowFloats = 132;
 constexpr uint32_t kRowStageBytes = 2 * kRowFloats * 4;                // 1056
 constexpr uint32_t kOffRow = kOffX + kStages * 2 * kTileBytes;
-constexpr uint32_t kOffBar = kOffRow + kStages * kRowStageBytes;
+// kModeAQ only: 64 rows of 512 bytes (fp32 dQ of 64 queries) staged for the
+// bulk reduce-adds, after the row stages.
+constexpr uint32_t kOffDqStage = (kOffRow + kStages * kRowStageBytes + 127) / 128 * 128;
+constexpr uint32_t kDqStageRows = 64;
+constexpr uint32_t kDqStageBytes = kDqStageRows * HD * 4;
 // Streamed tiles: X0 (pass A: Q, pass B: K) and X1 (dO / V) arrive on their
 // own barriers, so the MMA that needs X0 first does not wait for X1.  Pass A
 // frees both with one commit after dK; pass B frees V as soon as dP is done
 // (an elementwise thread arrives) and K with a commit after dQ.
 enum {
   B_FFULL = 0, B_FEMPTY, B_X0FULL0, B_X0FULL1, B_X1FULL0, B_X1FULL1, B_X0EMPTY0, B_X0EMPTY1, B_X1EMPTY0,
-  B_X1EMPTY1, B_SFULL, B_DPFULL, B_PFULL, B_DSFULL, B_OFULL, B_OEMPTY, B_DONE, B_COUNT
+  B_X1EMPTY1, B_SFULL, B_DPFULL, B_PFULL, B_DSFULL, B_OFULL, B_OEMPTY, B_DONE,
+  B_DVDONE, B_DQFULL, B_DQEMPTY,   // kModeAQ: dV has read dO; dQ^T is in TMEM; dQ^T has been read out
+  B_DQSTAGED,                      // kModeAQ: every dQ warp has written its channels of the staged rows
+  B_DQFREE,                        // kModeAQ: every dQ warp's bulk copies have read the staged rows
+  B_COUNT
 };
-constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;
-constexpr uint32_t kOffAbort = kOffSlot + 4;
-constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;
+// Barriers, TMEM slot and abort flag after the tiles.  Modes A and B leave
+// 1 KB of slack to round the dynamic shared memory base up to 1024 bytes;
+// kModeAQ needs that kilobyte for its staging rows, so it runs only on a
+// base that is already 1024-byte aligned (checked; error bit kErrSmemAlign).
+template <int kMode>
+__host__ __device__ constexpr uint32_t off_bar() {
+  return kMode == kModeAQ ? kOffDqStage + kDqStageBytes : kOffRow + kStages * kRowStageBytes;
+}
+template <int kMode>
+__host__ __device__ constexpr uint32_t smem_bytes() {
+  return off_bar<kMode>() + B_COUNT * 8 + 8 + (kMode == kModeAQ ? 0u : 1024u);
+}
+static_assert(smem_bytes<kModeAQ>() <= 232448, "kModeAQ shared memory");
+static_assert(smem_bytes<kModeA>() <= 232448, "pass shared memory");
 
 // TMEM columns: A0 (S or S^T, then P^T / dS bf16), A1 (dP or dP^T, then dS^T), accumulators
 constexpr uint32_t kColA0 = 0, kColA1 = 128, kColAcc0 = 256, kColAcc1 = 384;
 constexpr uint32_t kIdescSS = idesc_bf16_f32(BT, BT, 0, 0);
 constexpr uint32_t kIdescTS = idesc_bf16_f32(BT, HD, 0, 1);
+// dQ^T = K^T dS^T: M = D (A = K^T, MN-major in the K tile), N = 128 queries
+// (B = dS^T, MN-major: key rows of 128 query columns)
+constexpr uint32_t kIdescDq = idesc_bf16_f32(HD, BT, 1, 1);
 
 struct SegB {
   int32_t start, end;      // the segment's rows [start, end)
@@ -86,6 +127,9 @@ struct BwdParams {
   __nv_bfloat16* dqkv;     // [P, 3, Np, Hl, D]
   const float* nlse;       // [P*Hl][ls]: -lse
   const float* nd;         // [P*Hl][ls]: -rowsum(dO o O)
+  float* dqacc;            // kModeAQ: [P*Hl][Np][D] fp32 sum of dS K (zeroed by bwd_delta_kernel)
+  int64_t dqkv_ext;        // elements of dqkv (range checks of the bounds-checked build)
+  int64_t dqacc_ext;       // elements of dqacc
   int64_t ls;              // row stride of both
   unsigned int* err;
   int32_t N, Np, Hl, P, causal;
@@ -157,6 +201,20 @@ __device__ __forceinline__ void stream_range(const BwdParams& p, const SegB& sd,
   }
 }
 
+// kModeAQ starts a unit's loop over query blocks at its own key-tile index
+// (mod the block count), so the CTAs working on one head add into different
+// dQ tiles at any moment rather than all into the same one.  Block i of the
+// loop is query block first + rot_block(i, rot, count).
+template <int kMode>
+__device__ __forceinline__ int block_rot(const SegB& sd, const UnitB& w, int count) {
+  if (kMode != kModeAQ || count <= 0) return 0;
+  return ((w.row0 - sd.start) / BT) % count;
+}
+__device__ __forceinline__ int rot_block(int i, int rot, int count) {
+  const int k = i + rot;
+  return k >= count ? k - count : k;
+}
+
 __device__ __forceinline__ bool drain_wait_b(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
@@ -167,12 +225,14 @@ __device__ __forceinline__ bool drain_wait_b(uint32_t bar, uint32_t parity) {
 
 // nd[(r*Hl + j) * ls + n] = -sum_d dO[r, n, j, d] * O[r, n, j, d] and
 // nlse[...] = -lse[...] for n < Np: the row terms the elementwise step
-// subtracts, stored negated so that it adds them.  One half-warp per row:
-// 16 lanes x 8 channels.
+// subtracts, stored negated so that it adds them.  With dqacc (one-pass
+// backward) it also zeroes the row's fp32 dQ accumulator
+// dqacc[((r*Hl + j) * Np + n) * D ..].  One half-warp per row: 16 lanes x 8
+// channels.
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const int4* __restrict__ out, const int4* __restrict__ dout,
                                                         const float* __restrict__ lse, float* __restrict__ nd,
-                                                        float* __restrict__ nlse, int64_t rows, int32_t Np,
-                                                        int32_t Hl, int64_t ls) {
+                                                        float* __restrict__ nlse, float4* __restrict__ dqacc,
+                                                        int64_t rows, int32_t Np, int32_t Hl, int64_t ls) {
   const int64_t hw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
   const int64_t nhw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
   const int ch = threadIdx.x & 15;
@@ -195,14 +255,41 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const int4* __restrict__
     acc += __shfl_xor_sync(hmask, acc, 4);
     acc += __shfl_xor_sync(hmask, acc, 2);
     acc += __shfl_xor_sync(hmask, acc, 1);
+    const int64_t j = row % Hl;
+    const int64_t rn = row / Hl;
+    const int64_t n = rn % Np, r = rn / Np;
+    if (dqacc) {
+      float4* z = dqacc + ((r * Hl + j) * Np + n) * (HD / 4) + 2 * ch;
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if (ch == 0) {
-      const int64_t j = row % Hl;
-      const int64_t rn = row / Hl;
-      const int64_t n = rn % Np, r = rn / Np;
       const int64_t o = (r * Hl + j) * ls + n;
       nd[o] = -acc;
       nlse[o] = -lse[o];
     }
+  }
+}
+
+// dQ = scale * dqacc, rounded to bf16, into plane 0 of dqkv [P, 3, Np, Hl, D];
+// dqacc is [P*Hl][Np][D] fp32.  One thread per 8 channels.
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restrict__ dqacc, uint4* __restrict__ dqkv,
+                                                         int64_t rows, int32_t Np, int32_t Hl, float scale) {
+  const int64_t total = rows * 16;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = t >> 4;    // (r*Hl + j)*Np + n
+    const int ch = static_cast<int>(t & 15);
+    const int64_t n = row % Np, rj = row / Np;
+    const int64_t j = rj % Hl, r = rj / Hl;
+    const float4 a = dqacc[row * 32 + 2 * ch];
+    const float4 b = dqacc[row * 32 + 2 * ch + 1];
+    uint4 q;
+    q.x = pack_bf16x2(a.x * scale, a.y * scale);
+    q.y = pack_bf16x2(a.z * scale, a.w * scale);
+    q.z = pack_bf16x2(b.x * scale, b.y * scale);
+    q.w = pack_bf16x2(b.z * scale, b.w * scale);
+    dqkv[(((r * 3) * Np + n) * Hl + j) * 16 + ch] = q;
   }
 }
 
@@ -280,11 +367,20 @@ __device__ __forceinline__ void ds_half(const uint32_t (&dv)[32], const float* p
   }
 }
 
-template <bool kPassA>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kMode>
+__global__ void __launch_bounds__(threads_of<kMode>(), 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ BwdParams p) {
+  constexpr bool kPassA = kMode != kModeB;
+  constexpr bool kDq = kMode == kModeAQ;
+  constexpr uint32_t kOffBar = off_bar<kMode>();
+  constexpr uint32_t kOffSlot = kOffBar + B_COUNT * 8;
+  constexpr uint32_t kOffAbort = kOffSlot + 4;
   extern __shared__ uint8_t smem_raw[];
+  if (kDq && (smem_u32(smem_raw) & 1023u) != 0) {   // the layout has no slack to align it
+    if (threadIdx.x == 0 && p.err) atomicOr(p.err, kErrSmemAlign);
+    return;
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + kOffBar;
@@ -312,6 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(BAR(B_OFULL), 1);
     mbar_init(BAR(B_OEMPTY), kEwWarps);
     mbar_init(BAR(B_DONE), 1);
+    mbar_init(BAR(B_DVDONE), 1);
+    mbar_init(BAR(B_DQFULL), 1);
+    mbar_init(BAR(B_DQEMPTY), 4);           // one elected arrival per dQ warp
+    mbar_init(BAR(B_DQSTAGED), 4);
+    mbar_init(BAR(B_DQFREE), 4);
     fence_mbar_init();
   }
   if (warp == kTmaWarp && lane == 0) {
@@ -326,9 +427,108 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (kDq) {   // whole warpgroups: 0-1 elementwise, 2 MMA / TMA (+ two idle warps), 3 dQ
+    if (warp < kEwWarps)
+      regs_inc<kEwRegs>();
+    else if (warp < kDqWarp0)
+      regs_dec<kCtlRegs>();
+    else
+      regs_dec<kDqRegs>();
+  }
 
-
-  if (warp >= kEwWarps) {
+  if (kDq && warp >= kDqWarp0) {
+    // ------------------------------------------------------------ dQ reduction (kModeAQ)
+    // Thread (warp w, lane l) owns TMEM lane d = 32 (w % 4) + l of dQ^T, i.e.
+    // channel d of the block's 128 queries.  dQ^T goes out in two rounds of 64
+    // queries through a 32 KB staging area of fp32 rows [q][d] (512 bytes per
+    // query): the first round's columns are read from TMEM and stored, the
+    // second's read into registers, after which A1 is free for the next dP;
+    // each round is then handed to the TMA engine as bulk reduce-adds into
+    // dqacc[(r*Hl + j)*Np + q][..] (warp w: 16 of the 64 queries, those inside
+    // the segment).  A round's rows are overwritten only after every warp's
+    // bulk copies of the previous round have read them (B_DQFREE).
+    const int dq_w = warp - kDqWarp0;
+    const int dl = 32 * (warp & 3) + lane;
+    const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kColA1;
+    const uint32_t sbuf = sbase + kOffDqStage;
+    uint32_t qc = 0, rc = 0;   // blocks, staging rounds
+    bool ok = true;
+    // Before staging round n: every warp's bulk copies of round n - 1 have read the rows.
+    auto dq_rows_free = [&](uint32_t n) -> bool {
+      if (n == 0) return true;
+      if (lane == 0) {
+        bulk_wait_read();
+        mbar_arrive(BAR(B_DQFREE));
+      }
+      return mbar_wait_warp(BAR(B_DQFREE), (n - 1) & 1, g);
+    };
+    // After staging round n (queries q0 .. q0 + 63): once every warp's channels
+    // are in place, warp w reduce-adds queries q0 + 16w .. + 15 (those before
+    // `end`) into dqacc.
+    auto dq_rows_reduce = [&](uint32_t n, int q0, int end, int64_t head_row) -> bool {
+      fence_proxy_async_smem();                      // the rows are for the TMA engine to read
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(B_DQSTAGED));
+      if (!mbar_wait_warp(BAR(B_DQSTAGED), n & 1, g)) return false;   // every channel is in place
+      if (lane == 0) {
+        const int qw = q0 + 16 * dq_w;
+        const int nq = min(16, end - qw);            // rows of this warp inside the segment
+        if (nq > 0) {
+          const int64_t off = (head_row + qw) * HD;
+          if (in_bounds(off, static_cast<int64_t>(nq) * HD, p.dqacc_ext, p.err))
+            bulk_reduce_add_f32(p.dqacc + off, sbuf + dq_w * 16 * 512, static_cast<uint32_t>(nq) * 512);
+        }
+        bulk_commit();
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int k = 0; ok; ++k) {
+      UnitB w;
+      const int st = unit_of_cta_b(p, k, w);
+      if (st == 0 || st < 0) break;
+      if (st == 2) continue;
+      const SegB& sd = p.seg[w.seg];
+      int first, count;
+      stream_range<true>(p, sd, w, first, count);
+      const int rot = block_rot<kMode>(sd, w, count);
+      const int64_t head_row = (static_cast<int64_t>(w.r) * p.Hl + w.j) * p.Np;
+      for (int i = 0; ok && i < count; ++i) {
+        const int r0 = sd.start + (first + rot_block(i, rot, count)) * BT;
+        if (!(ok = mbar_wait_warp(BAR(B_DQFULL), qc & 1, g))) break;
+        ++qc;
+        tc_fence_after();
+        // round 0 (queries 0-63): into the staging rows once the previous round's
+        // bulk copies have read them
+        uint32_t v[2][32];
+        tmem_ld32(tq, v[0]);
+        tmem_ld32(tq + 32, v[1]);
+        tmem_wait_ld();
+        tmem_regs_ready(v[0]);
+        tmem_regs_ready(v[1]);
+        if (!(ok = dq_rows_free(rc))) break;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sts32(sbuf + c * 512 + 4 * dl, v[c >> 5][c & 31]);
+        // round 1 (queries 64-127) into registers: all of dQ^T is out of TMEM
+        tmem_ld32(tq + 64, v[0]);
+        tmem_ld32(tq + 96, v[1]);
+        tmem_wait_ld();
+        tmem_regs_ready(v[0]);
+        tmem_regs_ready(v[1]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_DQEMPTY));   // A1 may take the next dP
+        if (!(ok = dq_rows_reduce(rc, r0, sd.end, head_row))) break;
+        ++rc;
+        if (!(ok = dq_rows_free(rc))) break;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sts32(sbuf + c * 512 + 4 * dl, v[c >> 5][c & 31]);
+        if (!(ok = dq_rows_reduce(rc, r0 + 64, sd.end, head_row))) break;
+        ++rc;
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  } else if (warp >= kEwWarps) {
    if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -346,6 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const SegB& sd = p.seg[w.seg];
         int first, count;
         stream_range<kPassA>(p, sd, w, first, count);
+        const int rot = block_rot<kMode>(sd, w, count);
         if (uc > 0 && !(ok = mbar_wait(BAR(B_FEMPTY), (uc - 1) & 1, g))) break;
         mbar_arrive_expect_tx(BAR(B_FFULL), 2 * kTileBytes);
         for (int h = 0; h < 2; ++h) {
@@ -358,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         for (int i = 0; i < count; ++i) {
-          const int r0 = sd.start + (first + i) * BT;
+          const int r0 = sd.start + (first + rot_block(i, rot, count)) * BT;
           const uint32_t s = xc % kStages, ph = (xc / kStages) & 1;
           const uint32_t x0 = sbase + kOffX + s * 2 * kTileBytes, x1 = x0 + kTileBytes;
           if (kPassA) {   // streamed: Q with its -lse / -D rows, then dO, of a query block
@@ -402,15 +603,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ tcgen05 issuer
     // Per block i (pass A):  [P^T(i) ready] dV += P^T dO, S(i+1), [dS^T(i) ready] dK += dS^T Q, dP(i+1)
     //           (pass B):  [S(i) read]      S(i+1),          [dS(i) ready]   dQ += dS K,   dP(i+1)
+    //          (kModeAQ):  [P^T(i) ready] dV += P^T dO, S(i+1), [dS(i) ready] dK += dS^T Q,
+    //                      dQ^T = K^T dS^T over A1, [dQ^T read out] dP(i+1)
     // so the next block's S is computed while the elementwise warps form dS.
     // The bf16 operands P^T / dS come in two halves of 32 TMEM columns, one per
     // elementwise warpgroup, at column offsets 0 and 64 of their region.
     if (lane == 0) {
-      uint32_t xc = 0, uc = 0, pc = 0;
+      uint32_t xc = 0, uc = 0, pc = 0, qfull = 0, qempty = 0;
       bool ok = true;
       const uint64_t dF0 = desc_sw128(sbase + kOffF0, 16, 1024), dF1 = desc_sw128(sbase + kOffF1, 16, 1024);
+      const uint64_t dKT = desc_sw128(sbase + kOffF0, kHalfBytes, 1024);   // K^T as an MN-major A operand
       auto xdesc = [&](uint32_t s, int t, uint32_t lbo) {
         return desc_sw128(sbase + kOffX + s * 2 * kTileBytes + t * kTileBytes, lbo, 1024);
+      };
+      // kModeAQ: A1 may take the next dP only once the last dQ^T has been read out of it
+      auto a1_free = [&]() -> bool {
+        if (!kDq || qempty == qfull) return true;
+        if (!mbar_wait(BAR(B_DQEMPTY), qempty & 1, g)) return false;
+        ++qempty;
+        tc_fence_after();
+        return true;
       };
       for (int k = 0; ok; ++k) {
         UnitB w;
@@ -431,6 +643,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // pass A: S^T = K Q^T, dP^T = V dO^T;  pass B: S = Q K^T, dP = dO V^T
           mma_ss_k128(tmem + kColA0, dF0, xdesc(s, 0, 16), kIdescSS, 0);
           mma_commit(BAR(B_SFULL));
+          ok = a1_free();
+          if (!ok) break;
           if (!(ok = mbar_wait(BAR(B_X1FULL0 + s), ph, g))) break;
           tc_fence_after();
           mma_ss_k128(tmem + kColA1, dF1, xdesc(s, 1, 16), kIdescSS, 0);
@@ -444,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kPassA) {   // dV += P^T dO (B: dO read MN-major from the stage)
             mma_ts_k64(tmem + kColAcc0, tmem + kColA0, xdesc(s, 1, kHalfBytes), kIdescTS, i > 0);
             mma_ts_k64(tmem + kColAcc0, tmem + kColA0 + 64, xdesc(s, 1, kHalfBytes) + 512, kIdescTS, 1);
+            if (kDq) mma_commit(BAR(B_DVDONE));   // dO's slot may now take dS
           }
           if (more) {     // S of the next block over A0 (in order after the MMAs that read it)
             if (!(ok = mbar_wait(BAR(B_X0FULL0 + sn), ((xi + 1) / kStages) & 1, g))) break;
@@ -458,8 +673,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t acc = kPassA ? kColAcc1 : kColAcc0;
           mma_ts_k64(tmem + acc, tmem + kColA1, xdesc(s, 0, kHalfBytes), kIdescTS, i > 0);
           mma_ts_k64(tmem + acc, tmem + kColA1 + 64, xdesc(s, 0, kHalfBytes) + 512, kIdescTS, 1);
-          mma_commit(BAR(B_X0EMPTY0 + s));
+          if (kDq) {      // dQ^T = K^T dS^T over A1 (after dK has read dS^T), dS from dO's slot
+            mma_ss_k128_mn(tmem + kColA1, dKT, xdesc(s, 1, kHalfBytes), kIdescDq, 0);
+            mma_commit(BAR(B_X0EMPTY0 + s));
+            mma_commit(BAR(B_DQFULL));
+            ++qfull;
+          } else {
+            mma_commit(BAR(B_X0EMPTY0 + s));
+          }
           if (more) {     // dP of the next block over A1
+            ok = a1_free();
+            if (!ok) break;
             if (!(ok = mbar_wait(BAR(B_X1FULL0 + sn), ((xi + 1) / kStages) & 1, g))) break;
             tc_fence_after();
             mma_ss_k128(tmem + kColA1, dF1, xdesc(sn, 1, 16), kIdescSS, 0);
@@ -487,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tA0 = tmem + lane_base + kColA0 + c0, tA1 = tmem + lane_base + kColA1 + c0;
     const float sl2 = p.scale_log2;
     const float* srow = reinterpret_cast<const float*>(smem + kOffRow);
-    uint32_t sc = 0, uc = 0, xc = 0;
+    uint32_t sc = 0, uc = 0, xc = 0, dvc = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
       UnitB w;
@@ -498,6 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int end = sd.end;
       int first, count;
       stream_range<kPassA>(p, sd, w, first, count);
+      const int rot = block_rot<kMode>(sd, w, count);
       const int my = w.row0 + row;                     // key (pass A) or query (pass B) index
       float nl_row = 0.f, nd_row = 0.f;               // pass B: -lse and -D of this thread's query
       if (!kPassA && my < p.Np) {
@@ -509,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait_warp(BAR(B_SFULL), sc & 1, g))) break;
         ++sc;
         tc_fence_after();
-        const int r0 = sd.start + (first + i) * BT;    // first streamed index of this block
+        const int r0 = sd.start + (first + rot_block(i, rot, count)) * BT;    // first streamed index of this block
         const uint32_t s = xc % kStages;
         // pass A reads the block's lse / D rows, which arrive with the stage
         const uint32_t ph = (xc / kStages) & 1;
@@ -554,18 +779,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait_warp(BAR(B_DPFULL), (sc - 1) & 1, g))) break;
         tc_fence_after();
         if (!kPassA && threadIdx.x == 0) mbar_arrive(BAR(B_X1EMPTY0 + s));   // dP done: V's slot is free
+        uint32_t dsk[2][16];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {    // two halves of 32 columns: dS of half 0 lands before half 1 is read
           uint32_t dv[32];
           tmem_ld32(tA1 + 32 * h, dv);
           tmem_wait_ld();
           tmem_regs_ready(dv);
-          uint32_t pk[16];
           if (full)
-            ds_half<kPassA, false>(dv, pr + 32 * h, nd_s + 32 * h, nd_sa + 128 * h, nd_row, pk);
+            ds_half<kPassA, false>(dv, pr + 32 * h, nd_s + 32 * h, nd_sa + 128 * h, nd_row, dsk[h]);
           else
-            ds_half<kPassA, true>(dv, pr + 32 * h, nd_s + 32 * h, nd_sa + 128 * h, nd_row, pk);
-          tmem_st16(tA1 + 16 * h, pk);
+            ds_half<kPassA, true>(dv, pr + 32 * h, nd_s + 32 * h, nd_sa + 128 * h, nd_row, dsk[h]);
+          tmem_st16(tA1 + 16 * h, dsk[h]);
+        }
+        if (kDq) {
+          // dS (bf16) also into shared memory for dQ^T = K^T dS^T, over the block's
+          // dO tile once dV has read it: key row `row` of the warpgroup's 64-query
+          // half, 128 bytes in 16-byte chunks at the 128B-swizzled positions
+          if (!(ok = mbar_wait_warp(BAR(B_DVDONE), dvc & 1, g))) break;
+          ++dvc;
+          const uint32_t drow = sbase + kOffX + s * 2 * kTileBytes + kTileBytes + wg * kHalfBytes + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            sts128(drow + ((c ^ (row & 7)) << 4), dsk[c >> 2][4 * (c & 3)], dsk[c >> 2][4 * (c & 3) + 1],
+                   dsk[c >> 2][4 * (c & 3) + 2], dsk[c >> 2][4 * (c & 3) + 3]);
+          fence_proxy_async_smem();
         }
         tmem_wait_st();
         tc_fence_before();
@@ -590,9 +828,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tmem_regs_ready(ov[0]);
         tmem_regs_ready(ov[1]);
-        if (write) {
-          uint4* dst = reinterpret_cast<uint4*>(
-              p.dqkv + ((((static_cast<int64_t>(w.r) * 3 + plane) * p.Np + my) * p.Hl + w.j) * HD + c0));
+        const int64_t doff = (((static_cast<int64_t>(w.r) * 3 + plane) * p.Np + my) * p.Hl + w.j) * HD + c0;
+        if (write && in_bounds(doff, 64, p.dqkv_ext, p.err)) {
+          uint4* dst = reinterpret_cast<uint4*>(p.dqkv + doff);
           const float* o = reinterpret_cast<const float*>(&ov[0][0]);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
@@ -654,18 +892,19 @@ bool head_map(CUtensorMap* m, const void* base, int64_t P, int64_t C, int64_t Np
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kPassA>
+template <int kMode>
 cudaError_t launch_pass(const CUtensorMap& tq, const CUtensorMap& td, const BwdParams& p, int sms,
                         cudaStream_t stream) {
   static PerDeviceOnce setup;
   int dev = 0;
   cudaGetDevice(&dev);
   cudaError_t e = setup.run(dev, [] {
-    return cudaFuncSetAttribute(attn_bwd_kernel<kPassA>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    return cudaFuncSetAttribute(attn_bwd_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem_bytes<kMode>());
   });
   if (e != cudaSuccess) return e;
   const int grid = std::min(p.num_units, sms);
-  attn_bwd_kernel<kPassA><<<grid, kThreads, kSmemBytes, stream>>>(tq, td, p);
+  attn_bwd_kernel<kMode><<<grid, threads_of<kMode>(), smem_bytes<kMode>(), stream>>>(tq, td, p);
   return cudaGetLastError();
 }
 
@@ -686,7 +925,8 @@ cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
     const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
     if (grid > 0)
       bwd_delta_kernel<<<grid, 256, 0, stream>>>(static_cast<const int4*>(a.out), static_cast<const int4*>(a.dout),
-                                                 a.lse, a.delta, a.delta + P * Hl * ls, rows,
+                                                 a.lse, a.delta, a.delta + P * Hl * ls,
+                                                 reinterpret_cast<float4*>(a.dq_acc), rows,
                                                  static_cast<int32_t>(Np), static_cast<int32_t>(Hl), ls);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -700,6 +940,9 @@ cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
   p.dqkv = static_cast<__nv_bfloat16*>(a.dqkv);
   p.nd = a.delta;
   p.nlse = a.delta + P * Hl * ls;
+  p.dqacc = a.dq_acc;
+  p.dqkv_ext = P * 3 * Np * Hl * HD;
+  p.dqacc_ext = a.dq_acc ? P * Hl * Np * HD : 0;
   p.ls = ls;
   p.err = pl->dev_err;
   p.N = static_cast<int32_t>(pl->N);
@@ -735,9 +978,19 @@ cudaError_t launch_attn_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
   p.num_pairs = pairs;
   p.paired = (p.causal && units >= 2 * sms) ? 1 : 0;   // two units per SM at least, or the pairs idle SMs
   if (units == 0) return cudaSuccess;
-  cudaError_t e = launch_pass<true>(tq, td, p, sms, stream);    // dK, dV
+  if (!a.dq_acc) {   // deterministic: two passes
+    cudaError_t e = launch_pass<kModeA>(tq, td, p, sms, stream);    // dK, dV
+    if (e != cudaSuccess) return e;
+    return launch_pass<kModeB>(tq, td, p, sms, stream);            // dQ
+  }
+  cudaError_t e = launch_pass<kModeAQ>(tq, td, p, sms, stream);     // dK, dV, and dQ into dq_acc
   if (e != cudaSuccess) return e;
-  return launch_pass<false>(tq, td, p, sms, stream);           // dQ
+  const int64_t rows = P * Hl * Np;
+  const int grid = static_cast<int>(std::min<int64_t>((rows * 16 + 255) / 256, static_cast<int64_t>(sms) * 8));
+  dq_convert_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
+                                              static_cast<uint4*>(a.dqkv), rows, static_cast<int32_t>(Np),
+                                              static_cast<int32_t>(Hl), a.scale);
+  return cudaGetLastError();
 }
 
 }  // namespace ulysses

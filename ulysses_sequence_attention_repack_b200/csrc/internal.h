@@ -49,6 +49,7 @@ struct ulysses_plan_s {
   int32_t num_seqs;
   int32_t causal;                       // attention sees keys m <= n only
   int32_t pair_cta;                     // bf16 attention on CTA pairs (clusters of two) instead of one CTA per SM
+  int32_t deterministic;                // backward in two passes without atomics (bit-reproducible)
   ulysses::Segment segs[ULYSSES_MAX_SEQS];
   int32_t device;                       // device the plan's scratch lives on (-1: none)
   unsigned int* dev_err;                // device error word (16 bytes allocated)
@@ -128,6 +129,7 @@ struct AttnBwdLaunch {
   const void* dout;     // dO_T [P, Np, Hl, D]
   const float* lse;     // [P*Hl][lse_stride] from the forward
   float* delta;         // workspace: -rowsum(dO o O), then -lse, each [P*Hl][lse_stride]
+  float* dq_acc;        // one-pass backward: fp32 [P*Hl][Np][D] dQ accumulator (workspace); null = two passes
   void* dqkv;           // [P, 3, Np, Hl, D]
   float scale;
   const ulysses_plan_t* plan;

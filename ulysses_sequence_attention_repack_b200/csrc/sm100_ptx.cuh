@@ -13,6 +13,7 @@ namespace ulysses {
 enum : uint32_t {
   kErrWaitTimeout = 1u,   // an mbarrier wait gave up
   kErrBadUnit = 2u,       // a work-unit index decoded outside the problem
+  kErrSmemAlign = 8u,     // dynamic shared memory not at the alignment a kernel's layout assumes
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -316,6 +317,33 @@ __device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Eight MMAs over K = 128 with BOTH operands MN-major in 128B-swizzled shared
+// memory: every k-step covers 16 K-rows of 128 bytes (2048 bytes, +128
+// descriptor units) in each.
+__device__ __forceinline__ void mma_ss_k128_mn(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, t;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 a, %1, 128;\n\tadd.s64 b, %2, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 256;\n\tadd.s64 b, %2, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 384;\n\tadd.s64 b, %2, 384;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 512;\n\tadd.s64 b, %2, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 640;\n\tadd.s64 b, %2, 640;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 768;\n\tadd.s64 b, %2, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.s64 a, %1, 896;\n\tadd.s64 b, %2, 896;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Four MMAs over K = 64 (A in TMEM, B MN-major in shared memory): half of
 // mma_ts_k128.  a_tmem / bdesc point at the first of the four k-steps.
 __device__ __forceinline__ void mma_ts_k64(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
@@ -520,6 +548,38 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 16-byte shared-memory store at a shared-window address.
+__device__ __forceinline__ void sts128(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Make this thread's ordinary shared-memory stores visible to the async proxy
+// (the tensor core reading a descriptor operand) before a barrier hands the
+// buffer over.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Bulk fp32 reduce-add of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from this CTA's shared memory into global memory, performed at L2
+// by the TMA engine; tracked by the issuing thread's bulk async-group.  No
+// multicast.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The shared-memory sources of this thread's committed bulk groups have been read.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// This thread's committed bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 4-byte shared-memory store at a shared-window address.
+__device__ __forceinline__ void sts32(uint32_t saddr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
 }
 
 // 16-byte shared-memory load at a shared-window address (volatile: stays after

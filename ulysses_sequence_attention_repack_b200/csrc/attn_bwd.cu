@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(threads_of<kMode>(), 1)
       mbar_init(BAR(B_X0FULL0 + s), 1);
       mbar_init(BAR(B_X1FULL0 + s), 1);
       mbar_init(BAR(B_X0EMPTY0 + s), 1);
-      mbar_init(BAR(B_X1EMPTY0 + s), 1);
+      mbar_init(BAR(B_X1EMPTY0 + s), kDq ? 4 : 1);   // kModeAQ: the dQ warps release dO's slot
     }
     mbar_init(BAR(B_SFULL), 1);
     mbar_init(BAR(B_DPFULL), 1);
@@ -439,33 +439,25 @@ __global__ void __launch_bounds__(threads_of<kMode>(), 1)
   if (kDq && warp >= kDqWarp0) {
     // ------------------------------------------------------------ dQ reduction (kModeAQ)
     // Thread (warp w, lane l) owns TMEM lane d = 32 (w % 4) + l of dQ^T, i.e.
-    // channel d of the block's 128 queries.  dQ^T goes out in two rounds of 64
-    // queries through a 32 KB staging area of fp32 rows [q][d] (512 bytes per
-    // query): the first round's columns are read from TMEM and stored, the
-    // second's read into registers, after which A1 is free for the next dP;
-    // each round is then handed to the TMA engine as bulk reduce-adds into
+    // channel d of the block's 128 queries.  dQ^T goes out as fp32 rows [q][d]
+    // (512 bytes per query) in two rounds of 64 queries: round 0 into the
+    // block's dO slot (free once dQ^T is complete: it held dS), round 1 into
+    // registers, after which A1 is free for the next dP; then round 1 into a
+    // 32 KB staging area once the previous block's round 1 has been read out
+    // of it.  Each round is handed to the TMA engine as bulk reduce-adds into
     // dqacc[(r*Hl + j)*Np + q][..] (warp w: 16 of the 64 queries, those inside
-    // the segment).  A round's rows are overwritten only after every warp's
-    // bulk copies of the previous round have read them (B_DQFREE).
+    // the segment); dO's slot returns to the producer when round 0 has been
+    // read.
     const int dq_w = warp - kDqWarp0;
     const int dl = 32 * (warp & 3) + lane;
     const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kColA1;
     const uint32_t sbuf = sbase + kOffDqStage;
-    uint32_t qc = 0, rc = 0;   // blocks, staging rounds
+    uint32_t qc = 0, rc = 0, xc = 0;   // blocks, staged rounds, stage slots used
     bool ok = true;
-    // Before staging round n: every warp's bulk copies of round n - 1 have read the rows.
-    auto dq_rows_free = [&](uint32_t n) -> bool {
-      if (n == 0) return true;
-      if (lane == 0) {
-        bulk_wait_read();
-        mbar_arrive(BAR(B_DQFREE));
-      }
-      return mbar_wait_warp(BAR(B_DQFREE), (n - 1) & 1, g);
-    };
-    // After staging round n (queries q0 .. q0 + 63): once every warp's channels
-    // are in place, warp w reduce-adds queries q0 + 16w .. + 15 (those before
-    // `end`) into dqacc.
-    auto dq_rows_reduce = [&](uint32_t n, int q0, int end, int64_t head_row) -> bool {
+    // Round n of 64 rows staged at `rows` (queries q0 .. q0 + 63): once every
+    // warp's channels are in place, warp w reduce-adds its 16 rows (those
+    // before `end`) into dqacc.
+    auto dq_rows_reduce = [&](uint32_t n, uint32_t rows, int q0, int end, int64_t head_row) -> bool {
       fence_proxy_async_smem();                      // the rows are for the TMA engine to read
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(B_DQSTAGED));
@@ -476,7 +468,7 @@ __global__ void __launch_bounds__(threads_of<kMode>(), 1)
         if (nq > 0) {
           const int64_t off = (head_row + qw) * HD;
           if (in_bounds(off, static_cast<int64_t>(nq) * HD, p.dqacc_ext, p.err))
-            bulk_reduce_add_f32(p.dqacc + off, sbuf + dq_w * 16 * 512, static_cast<uint32_t>(nq) * 512);
+            bulk_reduce_add_f32(p.dqacc + off, rows + dq_w * 16 * 512, static_cast<uint32_t>(nq) * 512);
         }
         bulk_commit();
       }
@@ -493,23 +485,21 @@ __global__ void __launch_bounds__(threads_of<kMode>(), 1)
       stream_range<true>(p, sd, w, first, count);
       const int rot = block_rot<kMode>(sd, w, count);
       const int64_t head_row = (static_cast<int64_t>(w.r) * p.Hl + w.j) * p.Np;
-      for (int i = 0; ok && i < count; ++i) {
+      for (int i = 0; ok && i < count; ++i, ++xc) {
         const int r0 = sd.start + (first + rot_block(i, rot, count)) * BT;
+        const uint32_t s = xc % kStages;
+        const uint32_t dslot = sbase + kOffX + s * 2 * kTileBytes + kTileBytes;
         if (!(ok = mbar_wait_warp(BAR(B_DQFULL), qc & 1, g))) break;
         ++qc;
         tc_fence_after();
-        // round 0 (queries 0-63): into the staging rows once the previous round's
-        // bulk copies have read them
         uint32_t v[2][32];
         tmem_ld32(tq, v[0]);
         tmem_ld32(tq + 32, v[1]);
         tmem_wait_ld();
         tmem_regs_ready(v[0]);
         tmem_regs_ready(v[1]);
-        if (!(ok = dq_rows_free(rc))) break;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) sts32(sbuf + c * 512 + 4 * dl, v[c >> 5][c & 31]);
-        // round 1 (queries 64-127) into registers: all of dQ^T is out of TMEM
+        for (int c = 0; c < 64; ++c) sts32(dslot + c * 512 + 4 * dl, v[c >> 5][c & 31]);
         tmem_ld32(tq + 64, v[0]);
         tmem_ld32(tq + 96, v[1]);
         tmem_wait_ld();
@@ -517,14 +507,23 @@ __global__ void __launch_bounds__(threads_of<kMode>(), 1)
         tmem_regs_ready(v[1]);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(B_DQEMPTY));   // A1 may take the next dP
-        if (!(ok = dq_rows_reduce(rc, r0, sd.end, head_row))) break;
-        ++rc;
-        if (!(ok = dq_rows_free(rc))) break;
+        if (lane == 0) mbar_arrive(BAR(B_DQEMPTY));   // all of dQ^T is out of TMEM: A1 may take the next dP
+        if (!(ok = dq_rows_reduce(rc++, dslot, r0, sd.end, head_row))) break;
+        if (qc > 1) {   // the previous block's round 1 must have been read out of the staging area
+          if (lane == 0) {
+            bulk_wait_read_but_newest();
+            mbar_arrive(BAR(B_DQFREE));
+          }
+          if (!(ok = mbar_wait_warp(BAR(B_DQFREE), (qc - 2) & 1, g))) break;
+        }
 #pragma unroll
         for (int c = 0; c < 64; ++c) sts32(sbuf + c * 512 + 4 * dl, v[c >> 5][c & 31]);
-        if (!(ok = dq_rows_reduce(rc, r0 + 64, sd.end, head_row))) break;
-        ++rc;
+        if (!(ok = dq_rows_reduce(rc++, sbuf, r0 + 64, sd.end, head_row))) break;
+        if (lane == 0) {   // round 0 has been read: dO's slot goes back to the producer
+          bulk_wait_read_but_newest();
+          mbar_arrive(BAR(B_X1EMPTY0 + s));
+        }
+        __syncwarp();
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -572,6 +571,8 @@ __global__ void __launch_bounds__(threads_of<kMode>(), 1)
             bulk_load(sbase + kOffRow + s * kRowStageBytes + kRowFloats * 4, p.nd + roff, kRowFloats * 4,
                       BAR(B_X0FULL0 + s));
             ++x0c;
+            // kModeAQ: dO's slot also stages half of a dQ^T block and comes back later
+            if (kDq && xc >= kStages && !(ok = mbar_wait(BAR(B_X1EMPTY0 + s), ph ^ 1, g))) break;
             mbar_arrive_expect_tx(BAR(B_X1FULL0 + s), kTileBytes);
             for (int h = 0; h < 2; ++h)
               tma_load_5d(x1 + h * kHalfBytes, &tm_do, BAR(B_X1FULL0 + s), 64 * h, w.j, r0, 0, w.r);

@@ -675,8 +675,8 @@ __global__ void __launch_bounds__(threads_of<kMode>(), 1)
           mma_ts_k64(tmem + acc, tmem + kColA1, xdesc(s, 0, kHalfBytes), kIdescTS, i > 0);
           mma_ts_k64(tmem + acc, tmem + kColA1 + 64, xdesc(s, 0, kHalfBytes) + 512, kIdescTS, 1);
           if (kDq) {      // dQ^T = K^T dS^T over A1 (after dK has read dS^T), dS from dO's slot
+            mma_commit(BAR(B_X0EMPTY0 + s));       // dK was the last reader of the Q slot
             mma_ss_k128_mn(tmem + kColA1, dKT, xdesc(s, 1, kHalfBytes), kIdescDq, 0);
-            mma_commit(BAR(B_X0EMPTY0 + s));
             mma_commit(BAR(B_DQFULL));
             ++qfull;
           } else {

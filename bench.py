@@ -383,6 +383,21 @@ def run_ours(args, rank, world, local_rank):
     bwd_ms = b0.elapsed_time(b1) / nbw
     if U.ulysses_last_device_error(plan) != 0:
         raise RuntimeError("a kernel reported a device error in the backward")
+    # the deterministic two-pass backward (ULYSSES_PLAN_DETERMINISTIC) on the same inputs
+    dplan = U.ulysses_plan(N, H, 128, P, C, 0, 0, 0, cu, causal=causal, deterministic=True)
+    del bws
+    bws = torch.empty(dplan.attn_bwd_workspace_bytes, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        U.ulysses_attn_bwd(dplan, T, OT, dO, lse, dT, bws, scale, stream=stream)
+    b0.record(stream)
+    for _ in range(nbw):
+        U.ulysses_attn_bwd(dplan, T, OT, dO, lse, dT, bws, scale, stream=stream)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    bwd_det_ms = b0.elapsed_time(b1) / nbw
+    if U.ulysses_last_device_error(dplan) != 0:
+        raise RuntimeError("a kernel reported a device error in the deterministic backward")
+    del bws
 
     # end to end through the C ABI from pinned host buffers
     host_in = S.cpu().pin_memory()
@@ -407,7 +422,7 @@ def run_ours(args, rank, world, local_rank):
     # the other layer workloads, a few steps each (outside the timed region)
     others = {}
     if not args.no_other_workloads:
-        del host_in, host_out, dev_in, ws, lse, dO, dT, bws
+        del host_in, host_out, dev_in, ws, lse, dO, dT
         for name in OTHER_WORKLOADS:
             if name != args.config:
                 others[name] = time_layer_workload(U, inputs, name, dev, stream, steps=max(3, min(args.steps, 10)))
@@ -473,6 +488,7 @@ def run_ours(args, rank, world, local_rank):
         "push_repack_fwd_gbs": round(rf_bytes / (push_rf_ms * 1e-3) / 1e9, 1),
         "attn_bwd_us": round(bwd_ms * 1000, 2),
         "attn_bwd_tflops": round(2.5 * flops / (bwd_ms * 1e-3) / 1e12, 1),
+        "attn_bwd_deterministic_us": round(bwd_det_ms * 1000, 2),
         "prologue_repack_fwd_us": round(prologue_ms * 1000, 2),
         "prologue_repack_fwd_gbs": round(rf_bytes / (prologue_ms * 1e-3) / 1e9, 1),
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_pair_kernel" if args.pair_attention else "attn_fwd_kernel",

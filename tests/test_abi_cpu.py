@@ -111,6 +111,33 @@ def test_plan_sizes_agree_with_oracle(N, H, P, C):
     assert plan.workspace_bytes == up(P * C * Np * Hl * 128 * 2) + up(P * Np * Hl * 128 * 2)
 
 
+@pytest.mark.parametrize("N,H,P", [(19_394, 56, 4), (104_448, 56, 8), (1024, 8, 2), (5, 4, 4), (300, 2, 1),
+                                   (4, 56, 56)])
+def test_backward_workspace_sizes(N, H, P):
+    """The deterministic backward needs the two row-term arrays; the one-pass
+    form adds the fp32 dQ accumulator [P*Hl][Np][D] after them, placed so that
+    a rank's slab workspace (ulysses_attn_bwd_slab) is exactly 1/P of the
+    whole; the layer backward's workspace grows by the same amount."""
+    det = U.ulysses_plan(N, H, 128, P, 3, deterministic=True)
+    one = U.ulysses_plan(N, H, 128, P, 3)
+    Np, Hl = orc.padded_tokens(N, P), H // P
+    rows = 2 * det.lse_bytes
+    assert det.attn_bwd_workspace_bytes == rows
+    acc = P * Hl * Np * 128 * 4
+    want = (rows + 256 * P - 1) // (256 * P) * (256 * P) + acc
+    assert one.attn_bwd_workspace_bytes == want
+    assert want % P == 0 and (want // P) % 256 == 0
+    # a rank's slab is the same problem on one rank with Hl heads
+    slab_rows = 2 * (det.lse_bytes // P)
+    assert one.slab_attn_bwd_workspace_bytes == (slab_rows + 255) // 256 * 256 + Hl * Np * 128 * 4
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    for plan in (det, one):
+        assert plan.layer_bwd_workspace_bytes == (up(P * Np * Hl * 128 * 2) + up(3 * P * Np * Hl * 128 * 2) +
+                                                  up(plan.attn_bwd_workspace_bytes))
+
+
 def test_window_bytes_printed_on_the_pages():
     # 250,000 tokens, 56 heads, head dim 128, SP 4: 896,000,000 bytes per plane, one plane per launch
     plan = U.ulysses_plan(250_000, 56, 128, 4, 4)

@@ -1,13 +1,15 @@
 """The bounds-checked build (libulysses_debug.so, compiled with -DULYSSES_DEBUG).
 
 In that build every global access of the repack, prologue and push kernels,
-and every store of the attention epilogue, checks that its 16-byte vector
-lies inside the buffer the launch geometry describes; an access outside is
-skipped and bit 4 of the device error word is set.  It stands in for a
-memory checker on this GPU.  Here the debug library runs the tiny and
-ragged workloads through every kernel family with the error word staying
-zero and outputs equal, bit for bit, to the default library's.  The check
-itself is exercised by a self-test hook that touches no memory.
+and every store of the attention epilogues and of the backward (its dK/dV
+stores and dQ reduce-adds), checks that it lies inside the buffer the launch
+geometry describes; an access outside is skipped and bit 4 of the device
+error word is set.  It stands in for a memory checker on this GPU.  Here the
+debug library runs the tiny and ragged workloads through every kernel family
+with the error word staying zero and outputs equal, bit for bit, to the
+default library's (for the one-pass backward, whose dQ is summed in a
+varying order, dK and dV).  The check itself is exercised by a self-test hook
+that touches no memory.
 """
 import os
 import subprocess
@@ -68,10 +70,25 @@ for r in range(P):
 back_push = [torch.empty((Nl, 1, H, 128), dtype=torch.bfloat16, device=dev) for _ in range(P)]
 for r in range(P):
     U.ulysses_repack_bwd_push(plan, r, OT[r], back_push, 1)
+# attention backward in both forms (the one-pass dQ sums in a varying order:
+# its dK and dV are compared, and all of the deterministic form's output)
+lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=dev)
+U.ulysses_attn_fwd_lse(plan, T, OT, lse, scale)
+g.manual_seed(92)
+dO = torch.randn(OT.shape, generator=g, device=dev).to(torch.bfloat16)
+dO[:, N:] = 0
+dT = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=dev)
+U.ulysses_attn_bwd(plan, T, OT, dO, lse, dT, torch.empty(plan.attn_bwd_workspace_bytes, dtype=torch.uint8,
+                                                          device=dev), scale)
+dplan = U.ulysses_plan(N, H, 128, P, C, deterministic=True)
+dTd = torch.empty_like(dT)
+U.ulysses_attn_bwd(dplan, T, OT, dO, lse, dTd, torch.empty(dplan.attn_bwd_workspace_bytes, dtype=torch.uint8,
+                                                            device=dev), scale)
 torch.cuda.synchronize()
-out["err"] = np.array([U.ulysses_last_device_error(plan)])
+out["err"] = np.array([U.ulysses_last_device_error(plan) | U.ulysses_last_device_error(dplan)])
 for name, t in (("T", T), ("OT", OT), ("OS", OS), ("OSf", OSf), ("back", back), ("T8", T8), ("Tp", Tp),
-                ("slabs", torch.stack(slabs)), ("shards", torch.cat(shards)), ("back_push", torch.cat(back_push))):
+                ("slabs", torch.stack(slabs)), ("shards", torch.cat(shards)), ("back_push", torch.cat(back_push)),
+                ("dKV_one_pass", dT[:, 1:]), ("dQKV_two_pass", dTd)):
     out[name] = t.contiguous().view(torch.uint8).cpu().numpy()
 np.savez(sys.argv[1], **out)
 """

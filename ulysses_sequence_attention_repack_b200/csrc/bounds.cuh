@@ -1,9 +1,9 @@
 // Range checks of computed global offsets, for the bounds-checked build.
 //
 // Built with -DULYSSES_DEBUG, every global access of the repack, prologue and
-// push kernels (and the attention epilogue's stores) first checks that the
-// 16-byte vector it touches lies inside the buffer the launch geometry
-// describes.  An access outside is skipped and bit kErrBounds is set in the
+// push kernels (and the stores of the attention epilogue and of the backward)
+// first checks that the span it touches lies inside the buffer the launch
+// geometry describes.  An access outside is skipped and bit kErrBounds is set in the
 // device error word, which ulysses_last_device_error reports; the kernel
 // carries on (no trap, no assert), so the context stays usable.  In the
 // default build the check is a compile-time `true` and costs nothing.

@@ -572,9 +572,8 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, uint32_t ssrc, 
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// The shared-memory sources of this thread's committed bulk groups have been
-// read (all of them, or all but the newest one).
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// The shared-memory sources of all but the newest of this thread's committed
+// bulk groups have been read.
 __device__ __forceinline__ void bulk_wait_read_but_newest() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }

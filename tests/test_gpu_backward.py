@@ -250,3 +250,56 @@ def test_backward_repeatability(gpu, P, N, H, cu, causal):
         x, y = a[:, 0].double(), b[:, 0].double()
         tol = 2.0 ** -7 * torch.maximum(x.abs(), y.abs()) + 1e-6 * x.abs().max()
         assert ((x - y).abs() <= tol).all()
+
+
+@pytest.mark.slow
+def test_attention_backward_long104k(gpu):
+    """The largest layer (P=8, N=104,448, H=56) through the default one-pass
+    backward, whose fp32 dQ accumulator is 2.99 GB here.  Every head: the
+    invariants sum_k dK[k] = 0 and sum_k dV[k] = sum_q dO[q]; pad rows zero;
+    dQ at 34 sampled query rows of one head per rank against fp64."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    P, N, H = 8, 104_448, 56
+    plan = U.ulysses_plan(N, H, 128, P, 3)
+    Np, Hl = plan.padded_tokens, H // P
+    scale = 1.0 / math.sqrt(128)
+    S = inputs.qkv_seq(N, H, P, 3, 3, gpu)
+    T = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_repack_fwd(plan, S, T)
+    del S
+    OT = torch.empty((P, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    lse = torch.empty(plan.lse_bytes // 4, dtype=torch.float32, device=gpu)
+    U.ulysses_attn_fwd_lse(plan, T, OT, lse, scale)
+    dO = _grad(gpu, (P, Np, Hl, 128), 230)
+    dO[:, N:] = 0
+    dT = torch.empty((P, 3, Np, Hl, 128), dtype=torch.bfloat16, device=gpu)
+    ws = torch.empty(plan.attn_bwd_workspace_bytes, dtype=torch.uint8, device=gpu)
+    U.ulysses_attn_bwd(plan, T, OT, dO, lse, dT, ws, scale)
+    torch.cuda.synchronize()
+    assert U.ulysses_last_device_error(plan) == 0
+    del ws, OT
+    assert not dT[:, :, N:].any()
+    for r in range(P):
+        dK = dT[r, 1, :N].double()
+        dV = dT[r, 2, :N].double()
+        g = dO[r, :N].double()
+        assert (dK.sum(0).abs() <= 1e-3 * dK.abs().sum(0) + 1e-6).all(), r
+        assert ((dV.sum(0) - g.sum(0)).abs() <= 1e-3 * g.abs().sum(0) + 1e-6).all(), r
+        del dK, dV, g
+    rng = np.random.default_rng(31)
+    qr = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 32, replace=False)]))
+    iq = torch.from_numpy(qr).to(gpu)
+    got_l, ref_l = [], []
+    for r in range(P):
+        j = r % Hl
+        q, k, v = (orc.bf16_bits_to_f64(inputs.host_bits(T[r, c, :N, j])) for c in range(3))
+        g_h = orc.bf16_bits_to_f64(inputs.host_bits(dO[r, :N, j]))
+        dq, _, _ = orc.attention_bwd_sampled(q, k, v, g_h, scale, qr, qr[:0])
+        got = dT[r, 0, :, j].index_select(0, iq).double().cpu().numpy()
+        _close(got, dq, f"dQ long104k {r},{j}", record=False)
+        got_l.append(got)
+        ref_l.append(dq)
+    check_attention("backward long104k one-pass dQ (sampled rows)", np.stack(got_l), np.stack(ref_l),
+                    max_abs=None, mean_abs=None)

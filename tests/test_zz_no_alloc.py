@@ -75,6 +75,38 @@ def test_no_alloc_leaves_device_memory_untouched(gpu):
         assert stats1.get(key, 0) == stats0.get(key, 0), key
 
 
+def test_no_alloc_call_in_a_cuda_graph(gpu):
+    """After a first call in this context (the header's rule), an asynchronous
+    call (host_status NULL) can be captured into a CUDA graph on a side
+    stream; each replay reproduces the fused layer bit for bit."""
+    import torch
+    import ulysses_sequence_attention_repack_b200 as U
+    from ulysses_sequence_attention_repack_b200 import inputs
+    lib = U.load()
+    P, N, H, C = 2, 1000, 8, 3
+    S = inputs.qkv_seq(N, H, P, C, 34, gpu)
+    Np = S.shape[0]
+    plan = U.ulysses_plan(N, H, 128, P, C)
+    ref = torch.empty((Np, H, 128), dtype=torch.bfloat16, device=gpu)
+    U.ulysses_layer_fwd(plan, S, ref, None, fused=1)
+    out = torch.empty_like(ref)
+    assert _call(lib, S, out, N, H, P, C, None) == (0, 0)      # the first call, outside any capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=side):
+        code = lib.ulysses_layer_fwd_fused_noalloc(S.data_ptr(), out.data_ptr(), N, H, 128, P, C, 0, 0, None, 0,
+                                                   None, side.cuda_stream)
+    assert code == 0
+    for _ in range(2):
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    del graph
+
+
 def test_no_alloc_rejects_bad_arguments(gpu):
     import ulysses_sequence_attention_repack_b200 as U
     lib = U.load()

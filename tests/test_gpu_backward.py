@@ -34,6 +34,9 @@ CASES = [
     pytest.param(2, 1024, 8, None, True, 4, id="causal"),
     pytest.param(2, 700, 4, [0, 256, 300, 700], True, 5, id="causal-varlen"),
     pytest.param(2, 1000, 4, [0, 0, 300, 300, 1000], False, 6, id="varlen-empty-segments"),
+    pytest.param(4, 5, 4, None, False, 7, id="N5"),
+    pytest.param(56, 1000, 56, None, False, 8, id="P56-Hl1"),
+    pytest.param(1, 129, 2, None, True, 9, id="causal-N129"),
 ]
 
 

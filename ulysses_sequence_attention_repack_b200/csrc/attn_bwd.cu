@@ -82,8 +82,11 @@ constexpr uint32_t kDqStageRows = 64;
 constexpr uint32_t kDqStageBytes = kDqStageRows * HD * 4;
 // Streamed tiles: X0 (pass A: Q, pass B: K) and X1 (dO / V) arrive on their
 // own barriers, so the MMA that needs X0 first does not wait for X1.  Pass A
-// frees both with one commit after dK; pass B frees V as soon as dP is done
-// (an elementwise thread arrives) and K with a commit after dQ.
+// frees both with one commit after dK; kModeAQ frees Q with that commit and
+// dO's slot (which then holds dS, and after dQ^T the first half of the
+// block's dQ rows) when the dQ warps' bulk copies have read it; pass B frees
+// V as soon as dP is done (an elementwise thread arrives) and K with a commit
+// after dQ.
 enum {
   B_FFULL = 0, B_FEMPTY, B_X0FULL0, B_X0FULL1, B_X1FULL0, B_X1FULL1, B_X0EMPTY0, B_X0EMPTY1, B_X1EMPTY0,
   B_X1EMPTY1, B_SFULL, B_DPFULL, B_PFULL, B_DSFULL, B_OFULL, B_OEMPTY, B_DONE,

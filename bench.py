@@ -6,7 +6,10 @@ One step = one pass of the whole layer over the workload's synthetic input:
 ulysses_repack_fwd (all planes) -> ulysses_attn_fwd -> ulysses_repack_bwd
 (output plane), each a C-ABI call on one stream with CUDA events between
 them.  Rank 0 prints one JSON line.  N > 1 runs N independent replicas (the
-layer has no exchange between GPUs in this build), launched with torchrun.
+layer has no exchange between GPUs in this build), launched with torchrun;
+the job then processes N layers per step, so ``value`` (and ``e2e.value``)
+is the slowest rank's step time divided by N, the whole job's time per
+layer, with the per-replica time in ``per_replica_us``.
 
 The default workload is the largest one that fits one GPU, the long clip
 (P=8, N=104,448, H=56).  The line also carries the other layer workloads
@@ -454,9 +457,12 @@ def run_ours(args, rank, world, local_rank):
         w["repack_fwd_frac"] = round(w["repack_fwd_gbs"] / pk["hbm_gbs"], 3)
     line = {
         "metric": "Ulysses layer µs; attn TFLOP/s and repack GB/s vs B200 peak",
-        "value": round(ms_per_step * 1000.0, 2),
+        # N replicas process N layers per step: the job's time per layer is the
+        # slowest rank's step time over N (per-replica time in per_replica_us)
+        "value": round(ms_per_step * 1000.0 / world, 2),
         "unit": "us per layer",
         "n_gpus": world,
+        "per_replica_us": round(ms_per_step * 1000.0, 2),
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4),
@@ -497,8 +503,9 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(attn_tflops / tpk, 3),
                      "frac_of_sustained": round(attn_tflops / spk, 3), "traffic": traffic,
                      "algorithmic_flops_per_launch": flops},
-        "e2e": {"value": round(e2e_ms * 1000, 2), "unit": "us per layer", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "path": "ulysses_layer_fwd_host (pinned host in/out)"},
+        "e2e": {"value": round(e2e_ms * 1000 / world, 2), "unit": "us per layer", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "path": "ulysses_layer_fwd_host (pinned host in/out)",
+                "per_replica_us": round(e2e_ms * 1000, 2)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "workloads": others,
@@ -605,7 +612,8 @@ def run_fp8(args, rank, world, local_rank):
     ms_per_step = total_ms / args.steps
     return {
         "metric": "Ulysses layer µs; attn TFLOP/s and repack GB/s vs B200 peak",
-        "value": round(ms_per_step * 1000.0, 2), "unit": "us per layer", "n_gpus": world, "steps": args.steps,
+        "value": round(ms_per_step * 1000.0 / world, 2), "unit": "us per layer", "n_gpus": world,
+        "per_replica_us": round(ms_per_step * 1000.0, 2), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 attention, bf16 in/out",
         "data": "synthetic N(0,1) bf16, seeded",
@@ -624,9 +632,9 @@ def run_fp8(args, rank, world, local_rank):
                                                                             pk["bf16_tflops"])), 3),
                      "traffic": recorded_traffic("attn_fwd_kernel_fp8", args.config),
                      "algorithmic_flops_per_launch": flops},
-        "e2e": {"value": round(e2e_ms * 1000, 2), "unit": "us per layer",
+        "e2e": {"value": round(e2e_ms * 1000 / world, 2), "unit": "us per layer",
                 "h2d_bytes_per_step": host_in.numel() * 2, "d2h_bytes_per_step": host_out.numel() * 2,
-                "path": "ulysses_layer_fwd_fp8_host (pinned host in/out)"},
+                "path": "ulysses_layer_fwd_fp8_host (pinned host in/out)", "per_replica_us": round(e2e_ms * 1000, 2)},
         "gpu_launches": (math.ceil(C / plan.plane_chunk) + 2) * args.steps,
         "clocks": clocks,
     }
